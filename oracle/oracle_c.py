@@ -1,0 +1,93 @@
+"""ctypes loader and builder for the C oracle (test infrastructure only)."""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def library_path():
+    return _LIB
+
+
+def build(force=False):
+    """Compile attn_oracle.c with gcc -O2 -fopenmp into liboracle.so (in place)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    tmp = _LIB + ".tmp%d" % os.getpid()
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
+                           "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        ptr = ctypes.c_void_p
+        for name in ("attn_oracle_f64", "attn_oracle_bf16"):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = [ptr, ptr, ptr, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                           ctypes.c_double, ctypes.c_int, ptr, ctypes.c_int, ptr, ptr, ctypes.c_int]
+        lib.attn_oracle_max_threads.restype = ctypes.c_int
+        lib.attn_oracle_max_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def max_threads():
+    return _load().attn_oracle_max_threads()
+
+
+def _bf16_bits(t):
+    """Raw uint16 patterns of a bf16 torch tensor (CPU, contiguous)."""
+    import torch
+    assert t.dtype == torch.bfloat16
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def attention_rows(q, k, v, scale, causal=False, rows=None, n_threads=0):
+    """Evaluate the oracle on selected query rows.
+
+    q, k, v: [B, H, N, d], either bf16 torch tensors (widened exactly) or
+    float64 arrays.  rows: None (all rows) or an int array [B*H, R] (or [R],
+    shared by every head) of query indices.  Returns (O [B*H, R, d],
+    LSE [B*H, R]) as float64 numpy arrays.
+    """
+    lib = _load()
+    try:
+        import torch
+        is_bf16 = isinstance(q, torch.Tensor) and q.dtype == torch.bfloat16
+    except ImportError:  # pragma: no cover
+        is_bf16 = False
+    B, H, N, d = (int(x) for x in q.shape)
+    if is_bf16:
+        qa, ka, va = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+        fn = lib.attn_oracle_bf16
+    else:
+        qa, ka, va = (np.ascontiguousarray(np.asarray(x, dtype=np.float64)) for x in (q, k, v))
+        fn = lib.attn_oracle_f64
+    if rows is None:
+        n_rows, rows_a, rows_p = N, None, None
+    else:
+        rows_a = np.asarray(rows, dtype=np.int32)
+        if rows_a.ndim == 1:
+            rows_a = np.broadcast_to(rows_a, (B * H, rows_a.shape[0]))
+        rows_a = np.ascontiguousarray(rows_a.reshape(B * H, -1))
+        n_rows = rows_a.shape[1]
+        rows_p = rows_a.ctypes.data
+    o = np.empty((B * H, n_rows, d), dtype=np.float64)
+    lse = np.empty((B * H, n_rows), dtype=np.float64)
+    rc = fn(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, B, H, N, d, float(scale),
+            int(bool(causal)), rows_p, n_rows, o.ctypes.data, lse.ctypes.data, int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments (code %d)" % rc)
+    return o, lse

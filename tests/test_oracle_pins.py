@@ -1,0 +1,238 @@
+"""Pins for the fp64 CPU oracle, against facts fixed by the mathematics.
+
+The oracle follows the plain definition of exact attention (FlashAttention:
+Fast and Memory-Efficient Exact Attention with IO-Awareness, wiki notes,
+section "Problem setting": O = softmax(Q K^T) V, here with an explicit scale
+and an optional square causal mask).  Each test below is chosen so that a
+plausible slip in the oracle -- a dropped scale, a wrong sign, exp vs exp2 or
+log vs log2, an off-by-one in the causal mask, K and V swapped, a missing max
+shift -- fails at least one of them.  None of them re-types the oracle's
+formula: they use closed forms, invariants, special cases and a 40-digit
+decimal evaluation of the naive (unshifted) formulation.
+"""
+import decimal
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_102_b200.inputs import make_qkv, sample_rows
+
+RNG = np.random.default_rng(12345)
+
+
+def _both(q, k, v, scale, causal):
+    """Run the C oracle and the NumPy twin; return both (O, LSE) shaped [B,H,N,...]."""
+    B, H, N, d = q.shape
+    oc, lc = oracle.attention_rows(q, k, v, scale, causal)
+    on, ln = oracle.attention_full(q, k, v, scale, causal)
+    return (oc.reshape(B, H, N, d), lc.reshape(B, H, N)), (on, ln)
+
+
+def _decimal_attention(q, k, v, scale, causal, digits=40):
+    """Naive softmax in 40-digit decimal arithmetic: no max subtraction."""
+    ctx = decimal.Context(prec=digits)
+    D = lambda x: ctx.create_decimal_from_float(float(x))
+    N, d = q.shape
+    o = np.zeros((N, d))
+    lse = np.zeros(N)
+    for i in range(N):
+        visible = range(i + 1) if causal else range(N)
+        w = []
+        for j in visible:
+            s = D(scale) * sum((D(q[i, t]) * D(k[j, t]) for t in range(d)), D(0))
+            w.append((j, ctx.exp(s)))
+        z = sum((x for _, x in w), D(0))
+        lse[i] = float(ctx.ln(z))
+        for t in range(d):
+            o[i, t] = float(sum((x * D(v[j, t]) for j, x in w), D(0)) / z)
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d,scale", [(1, 4, 0.5), (5, 3, 0.37), (16, 8, 1.3)])
+def test_decimal_bruteforce(N, d, scale, causal):
+    q = RNG.normal(size=(1, 1, N, d)) * 2.0
+    k = RNG.normal(size=(1, 1, N, d))
+    v = RNG.normal(size=(1, 1, N, d))
+    o_ref, lse_ref = _decimal_attention(q[0, 0], k[0, 0], v[0, 0], scale, causal)
+    for o, lse in _both(q, k, v, scale, causal):
+        np.testing.assert_allclose(o[0, 0], o_ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[0, 0], lse_ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_probability_rows_sum_to_one(causal):
+    # With V = I (d = N) the output row is the probability row itself.
+    N = 12
+    q = RNG.normal(size=(1, 2, N, N))
+    k = RNG.normal(size=(1, 2, N, N))
+    v = np.broadcast_to(np.eye(N), (1, 2, N, N)).copy()
+    for o, _ in _both(q, k, v, 0.7, causal):
+        p = o[0]
+        assert (p >= 0).all()
+        np.testing.assert_allclose(p.sum(-1), 1.0, rtol=0, atol=1e-12)
+        if causal:
+            upper = np.triu(np.ones((N, N), dtype=bool), 1)
+            assert (p[:, upper] == 0).all()
+            assert (p[:, ~upper] > 0).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_gives_mean_of_visible_values(causal):
+    B, H, N, d = 1, 2, 9, 5
+    q = np.zeros((B, H, N, d))
+    k = RNG.normal(size=(B, H, N, d))
+    v = RNG.normal(size=(B, H, N, d))
+    if causal:
+        counts = np.arange(1, N + 1)
+        mean = np.cumsum(v, axis=2) / counts[None, None, :, None]
+        lse_cf = np.log(counts)[None, None, :].repeat(H, 1)
+    else:
+        mean = np.broadcast_to(v.mean(axis=2, keepdims=True), v.shape)
+        lse_cf = np.full((B, H, N), math.log(N))
+    for o, lse in _both(q, k, v, 0.125, causal):
+        np.testing.assert_allclose(o, mean, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse, lse_cf, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_value_rows(causal):
+    B, H, N, d = 2, 1, 11, 4
+    q = RNG.normal(size=(B, H, N, d)) * 3
+    k = RNG.normal(size=(B, H, N, d))
+    c = np.array([1.5, -2.25, 0.0, 7.0])
+    v = np.broadcast_to(c, (B, H, N, d)).copy()
+    for o, _ in _both(q, k, v, 0.4, causal):
+        np.testing.assert_allclose(o, np.broadcast_to(c, o.shape), rtol=0, atol=1e-13)
+
+
+def test_one_hot_large_logit_selects_that_value_row():
+    N, d, jstar, i = 10, 4, 6, 2
+    q = np.zeros((1, 1, N, d))
+    k = np.zeros((1, 1, N, d))
+    q[0, 0, i, 0] = 10.0
+    k[0, 0, jstar, 0] = 10.0            # s[i, jstar] = 100, every other s[i, j] = 0
+    v = RNG.normal(size=(1, 1, N, d))
+    for o, lse in _both(q, k, v, 1.0, False):
+        np.testing.assert_allclose(o[0, 0, i], v[0, 0, jstar], rtol=0, atol=N * math.exp(-90))
+        assert abs(lse[0, 0, i] - 100.0) < N * math.exp(-90)
+        # the other rows see all-zero scores: mean of V, LSE = ln N
+        np.testing.assert_allclose(o[0, 0, 0], v[0, 0].mean(0), atol=1e-13)
+        assert abs(lse[0, 0, 0] - math.log(N)) < 1e-13
+
+
+def test_single_key():
+    q = RNG.normal(size=(3, 2, 1, 6))
+    k = RNG.normal(size=(3, 2, 1, 6))
+    v = RNG.normal(size=(3, 2, 1, 6))
+    for causal in (False, True):
+        for o, lse in _both(q, k, v, 0.3, causal):
+            np.testing.assert_allclose(o, v, rtol=0, atol=1e-15)
+            np.testing.assert_allclose(lse[..., 0], 0.3 * (q * k).sum(-1)[..., 0], atol=1e-13)
+
+
+def test_permutation_equivariance():
+    B, H, N, d = 1, 1, 13, 6
+    q = RNG.normal(size=(B, H, N, d))
+    k = RNG.normal(size=(B, H, N, d))
+    v = RNG.normal(size=(B, H, N, d))
+    o, lse = oracle.attention_rows(q, k, v, 0.5)
+    perm = RNG.permutation(N)
+    o_kv, lse_kv = oracle.attention_rows(q, k[:, :, perm], v[:, :, perm], 0.5)
+    np.testing.assert_allclose(o_kv, o, atol=1e-13)
+    np.testing.assert_allclose(lse_kv, lse, atol=1e-13)
+    o_q, lse_q = oracle.attention_rows(q[:, :, perm], k, v, 0.5)
+    np.testing.assert_allclose(o_q, o[:, perm], atol=1e-13)
+    np.testing.assert_allclose(lse_q, lse[:, perm], atol=1e-13)
+
+
+def test_score_shift_invariance():
+    # Append a coordinate that adds the same constant c to every score of a
+    # row: O is unchanged and LSE grows by exactly c.
+    B, H, N, d, scale, c = 1, 2, 8, 4, 0.25, 37.5
+    q = RNG.normal(size=(B, H, N, d))
+    k = RNG.normal(size=(B, H, N, d))
+    v = RNG.normal(size=(B, H, N, d))
+    q2 = np.concatenate([q, np.ones((B, H, N, 1))], -1)
+    k2 = np.concatenate([k, np.full((B, H, N, 1), c / scale)], -1)
+    v2 = np.concatenate([v, np.zeros((B, H, N, 1))], -1)   # head size is shared by Q, K, V
+    for causal in (False, True):
+        o, lse = oracle.attention_rows(q, k, v, scale, causal)
+        o2, lse2 = oracle.attention_rows(q2, k2, v2, scale, causal)
+        np.testing.assert_allclose(o2[..., :d], o, atol=1e-12)
+        np.testing.assert_array_equal(o2[..., d], 0.0)
+        np.testing.assert_allclose(lse2, lse + c, atol=1e-12)
+
+
+def test_causal_row_sees_exactly_its_prefix():
+    B, H, N, d = 1, 1, 10, 3
+    q = RNG.normal(size=(B, H, N, d))
+    k = RNG.normal(size=(B, H, N, d))
+    v = RNG.normal(size=(B, H, N, d))
+    o, lse = oracle.attention_rows(q, k, v, 0.6, True)
+    i = 4
+    k2, v2 = k.copy(), v.copy()
+    k2[0, 0, i + 1:] += 5.0
+    v2[0, 0, i + 1:] -= 3.0
+    o2, lse2 = oracle.attention_rows(q, k2, v2, 0.6, True)
+    np.testing.assert_array_equal(o2[0, : i + 1], o[0, : i + 1])
+    np.testing.assert_array_equal(lse2[0, : i + 1], lse[0, : i + 1])
+    v3 = v.copy()
+    v3[0, 0, i] += 1.0                      # key i is visible to query i
+    o3, _ = oracle.attention_rows(q, k, v3, 0.6, True)
+    assert np.abs(o3[0, i] - o[0, i]).max() > 1e-3
+    np.testing.assert_array_equal(o3[0, :i], o[0, :i])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_c_oracle_matches_numpy_twin_on_bf16_inputs(causal):
+    q, k, v = make_qkv(2, 2, 37, 16, seed=3)
+    scale = 0.25
+    o, lse = oracle.attention_rows(q, k, v, scale, causal)
+    qd, kd, vd = (x.double().numpy() for x in (q, k, v))
+    o_np, lse_np = oracle.attention_full(qd, kd, vd, scale, causal)
+    np.testing.assert_allclose(o.reshape(o_np.shape), o_np, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(lse_np.shape), lse_np, rtol=0, atol=1e-12)
+
+
+def test_bf16_widening_is_exact():
+    q, k, v = make_qkv(1, 3, 21, 8, seed=5)
+    o_b, l_b = oracle.attention_rows(q, k, v, 0.3, False)
+    o_f, l_f = oracle.attention_rows(*(x.double().numpy() for x in (q, k, v)), 0.3, False)
+    np.testing.assert_array_equal(o_b, o_f)
+    np.testing.assert_array_equal(l_b, l_f)
+
+
+def test_row_selection_matches_full_evaluation():
+    B, H, N, d = 2, 3, 50, 8
+    q, k, v = make_qkv(B, H, N, d, seed=7)
+    rows = sample_rows(B, H, N, count=9)
+    assert rows.shape == (B * H, 9)
+    assert (rows[:, 0] == 0).all() and (rows[:, -1] == N - 1).all()
+    for causal in (False, True):
+        o_all, l_all = oracle.attention_rows(q, k, v, 0.2, causal)
+        o_sel, l_sel = oracle.attention_rows(q, k, v, 0.2, causal, rows=rows.numpy())
+        idx = rows.numpy()
+        np.testing.assert_array_equal(o_sel, np.take_along_axis(o_all, idx[..., None], 1))
+        np.testing.assert_array_equal(l_sel, np.take_along_axis(l_all, idx, 1))
+
+
+def test_oracle_rejects_bad_rows():
+    q = np.zeros((1, 1, 4, 2))
+    with pytest.raises(ValueError):
+        oracle.attention_rows(q, q, q, 1.0, rows=np.array([[0, 4]]))
+
+
+def test_input_recipe_is_deterministic_and_bf16():
+    a = make_qkv(1, 2, 33, 64, seed=0)
+    b = make_qkv(1, 2, 33, 64, seed=0)
+    for x, y in zip(a, b):
+        assert x.dtype == torch.bfloat16 and x.is_contiguous()
+        assert torch.equal(x, y)
+    q4 = make_qkv(1, 2, 33, 64, seed=0, q_mult=4.0)[0]
+    assert torch.equal(q4.float(), a[0].float() * 4)
+    # Q, K, V come from one stream in that order: K differs from Q
+    assert not torch.equal(a[0], a[1])
