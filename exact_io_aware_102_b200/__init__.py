@@ -1,0 +1,122 @@
+"""Exact, IO-aware attention forward for B200 -- Python binding.
+
+Argument marshalling only: every step of the attention runs in the CUDA
+library ``libattn.so`` (built from ``csrc/attn_fwd.cu`` for sm_100a); PyTorch
+supplies device memory and the current stream.  There is no fallback: if the
+library is missing, every entry point raises.
+
+The C entry points keep their names here (``attn_fwd``,
+``attn_status_string``, ``attn_check_device_status``,
+``attn_selftest_wait_timeout``, ``attn_version``); ``forward`` is the tensor
+convenience wrapper.
+"""
+import ctypes
+import math
+import os
+
+__all__ = [
+    "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_status_string", "attn_check_device_status",
+    "attn_selftest_wait_timeout", "attn_version", "forward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
+    "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
+]
+
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = 0, 1, 2, 3, 4
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+_lib = None
+
+
+class AttnError(RuntimeError):
+    """A library call returned a status other than ATTN_OK."""
+
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (what, attn_status_string(status), status))
+
+
+def library():
+    """The loaded ``libattn.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libattn.so is not built (expected at %s); run "
+                              "`python -c 'import __graft_entry__ as g; g.build()'`" % LIB_PATH)
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i32 = ctypes.c_void_p, ctypes.c_int
+        lib.attn_fwd.restype = i32
+        lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, i32, vp]
+        lib.attn_status_string.restype = ctypes.c_char_p
+        lib.attn_status_string.argtypes = [i32]
+        lib.attn_check_device_status.restype = i32
+        lib.attn_check_device_status.argtypes = [vp]
+        lib.attn_selftest_wait_timeout.restype = i32
+        lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp]
+        lib.attn_version.restype = i32
+        lib.attn_version.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream):
+    """Raw C call: pointers are ints (device addresses), stream an int handle; returns the status."""
+    return library().attn_fwd(q, k, v, o, lse, int(B), int(H), int(N), int(d), float(scale),
+                              int(bool(causal)), stream)
+
+
+def attn_status_string(status):
+    return library().attn_status_string(int(status)).decode()
+
+
+def attn_check_device_status(stream=None):
+    """Synchronise ``stream`` and return (and clear) the device status word."""
+    return library().attn_check_device_status(_stream_handle(stream))
+
+
+def attn_selftest_wait_timeout(limit_ns, stream=None):
+    return library().attn_selftest_wait_timeout(int(limit_ns), _stream_handle(stream))
+
+
+def attn_version():
+    return library().attn_version()
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None):
+    """Exact attention forward on bf16 CUDA tensors [B, H, N, d] (d = 64 or 128).
+
+    Returns (o, lse): o bf16 [B, H, N, d] and lse fp32 [B, H, N] (natural-log
+    log-sum-exp of each row's scaled scores).  ``scale`` defaults to 1/sqrt(d).
+    ``out`` / ``lse`` may be given to write into existing tensors.  The call is
+    asynchronous on ``stream`` (default: the current stream).
+    """
+    import torch
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one shape [B, H, N, d]")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous bf16 CUDA tensor" % name)
+    B, H, N, d = (int(x) for x in q.shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor [B, H, N]")
+    status = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                      B, H, N, d, scale, causal, _stream_handle(stream))
+    if status != ATTN_OK:
+        raise AttnError(status, "attn_fwd")
+    return out, lse

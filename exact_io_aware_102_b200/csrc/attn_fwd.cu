@@ -1,0 +1,846 @@
+// Exact, IO-aware multi-head attention forward for B200 (sm_100a).
+//
+// What is computed (FlashAttention: Fast and Memory-Efficient Exact Attention
+// with IO-Awareness, wiki notes): O = softmax(scale * Q K^T) V per (batch,
+// head), "Problem setting"; Q, K and V are processed in on-chip tiles with a
+// running row maximum m and running row sum l that are updated from tile to
+// tile, so the N x N matrices never reach HBM, "Tiling"; scores, scaling,
+// masking, softmax and both matrix products run in ONE kernel, "Kernel
+// fusion"; only O and the per-row softmax statistics (here as one log-sum-exp)
+// are written, "Recomputation"; with a causal mask only the non-zero key
+// blocks are processed, "Block-sparse FlashAttention".
+//
+// How it maps to sm_100a (the page's A100 design is prior art, not followed):
+//   * persistent grid, one CTA per SM, each CTA walks work units
+//     (b, h, 256 query rows = two 128-row Q tiles);
+//   * warp 8 (one lane) issues TMA loads: the two Q tiles once per unit and a
+//     ring of K / V tiles (128 keys each) guarded by full/empty mbarriers;
+//   * warp 9 (one lane) issues tcgen05.mma: S_t = Q_t K_j^T into TMEM
+//     (fp32, 128 x 128), then O_t += P_t V_j with P_t read from TMEM;
+//   * warps 0-3 and 4-7 are the softmax warpgroups of Q tiles 0 and 1: one
+//     thread per query row reads its S row from TMEM, masks, updates m and l,
+//     rescales its O row in TMEM when m grows, writes P (bf16) back over S,
+//     and at the end normalises O by l and stores O and LSE;
+//   * every mbarrier wait is bounded; on timeout a status word is set, the
+//     CTA drains its in-flight copies and MMAs, frees TMEM and returns.
+//
+// Memory layout: Q, K, V, O bf16 [B, H, N, d] contiguous, LSE fp32 [B, H, N].
+// Shared memory tiles use the 128-byte swizzle (TMA writes them, the tensor
+// cores read them through matrix descriptors); d = 128 tiles are stored as two
+// 64-column halves.  TMEM: S0 cols [0,128), S1 [128,256), O0 [256,256+d),
+// O1 [256+d, 256+2d); P_t overlays the first 64 columns of S_t.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "attn.h"
+
+namespace {
+
+constexpr int kBlockM = 128;           // query rows per Q tile (= TMEM lanes)
+constexpr int kBlockN = 128;           // keys per K / V tile
+constexpr int kUnitRows = 2 * kBlockM;  // query rows per work unit
+constexpr int kThreads = 320;          // 2 softmax warpgroups + load warp + MMA warp
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s per wait
+
+template <int D>
+struct Cfg {
+    static constexpr int kHalfBytes = kBlockN * 64 * 2;       // one 128 x 64 bf16 swizzled half
+    static constexpr int kTileBytes = kBlockN * D * 2;        // one Q, K or V tile
+    static constexpr int kSlots = (D == 64) ? 8 : 4;          // K/V ring depth
+    static constexpr int kQOff = 0;
+    static constexpr int kRingOff = 2 * kTileBytes;
+    static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+    static constexpr int kSmemBytes = kBarOff + 512 + 1024;   // barriers + 1 KB alignment slack
+    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+    static_assert(256 + 2 * D <= (int)kTmemCols, "TMEM budget");
+};
+
+// Barrier block (offsets in bytes from the barrier area).
+struct Bars {
+    static constexpr int kQFull = 0;                 // [2]
+    static constexpr int kQEmpty = 16;               // [1]
+    static constexpr int kSFull = 24;                // [2]
+    static constexpr int kPFull = 40;                // [2]
+    static constexpr int kOFull = 56;                // [2]
+    static constexpr int kOEmpty = 72;               // [2]
+    static constexpr int kDrain = 88;                // [1]
+    static constexpr int kTmemSlot = 96;             // u32: TMEM base address
+    static constexpr int kAbort = 100;               // u32: abort flag
+    static constexpr int kKvFull = 128;              // [slots]
+    static constexpr int kKvEmpty = 128 + 8 * 8;     // [slots]
+};
+
+__device__ int g_attn_status = 0;   // 0 = fine; ATTN_ERR_TIMEOUT after a wait ran out
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait until the phase with parity `parity` of barrier `bar` has completed.
+// Gives up after `limit_ns` (then raises the CTA abort flag and the device
+// status word) or as soon as another thread of the CTA has raised the abort
+// flag.  Returns false when it gave up.
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                       unsigned long long limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    uint32_t n = 0;
+    while (!mbar_try_wait(bar, parity)) {
+        if ((++n & 31u) == 0) {
+            if (abort_flag != nullptr && *abort_flag) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                if (abort_flag != nullptr) *abort_flag = 1u;
+                atomicExch(&g_attn_status, (int)ATTN_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+    return true;
+}
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile uint32_t* abort_flag,
+                                             unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_slow(bar, parity, abort_flag, limit_ns);
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x,
+                                            int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// tcgen05 (5th-generation tensor core + tensor memory)
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc]
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 32 bits, 32 consecutive columns: thread i gets lane (base + i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+// Registers written by tcgen05.ld may only be read after tcgen05.wait::ld.
+// This empty volatile asm "redefines" them and is ordered after the wait, so
+// the compiler cannot hoist their uses above it.
+__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                   "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+                   "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+                   "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+                   "+r"(r[31]));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    // cvt packs its first source into the upper half
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: version
+// field 1 at bit 46, layout type 2 = SWIZZLE_128B at bits 61..63).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, A K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool b_mn_major) {
+    return (1u << 4)                        // D format f32
+           | (1u << 7)                      // A format bf16
+           | (1u << 10)                     // B format bf16
+           | ((b_mn_major ? 1u : 0u) << 16)  // B major
+           | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// ------------------------------------------------------------- the scheduler
+struct Params {
+    int BH, N, n_pairs, n_kv_all, total_units;
+    float scale_log2;  // scale * log2(e)
+    unsigned long long wait_ns;
+};
+
+struct Unit {
+    int bh, q0, n0, n1;  // head, first query row, KV tiles for Q tile 0 / 1
+};
+
+// Work units: (head, pair of Q tiles).  Non-causal: heads-major so the CTAs
+// running at one time share K/V of few heads (L2 reuse).  Causal: the pairs
+// with the most key tiles first, so the short units fill the tail.
+template <bool CAUSAL>
+__device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
+    Unit w;
+    int pair;
+    if (CAUSAL) {
+        pair = p.n_pairs - 1 - u / p.BH;
+        w.bh = u % p.BH;
+    } else {
+        pair = u % p.n_pairs;
+        w.bh = u / p.n_pairs;
+    }
+    w.q0 = pair * kUnitRows;
+    if (CAUSAL) {
+        const int need1 = (w.q0 + kUnitRows) / kBlockN;  // tiles touching rows < q0 + 256
+        const int need0 = w.q0 / kBlockN + 1;            // tiles touching rows < q0 + 128
+        w.n1 = min(p.n_kv_all, need1);
+        w.n0 = min(w.n1, need0);
+    } else {
+        w.n0 = w.n1 = p.n_kv_all;
+    }
+    return w;
+}
+
+// ----------------------------------------------------------------- the kernel
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out_o,
+                float* __restrict__ out_lse, const Params p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;  // 128B-swizzled tiles need 1 KB alignment
+    uint8_t* const gbase = smem_raw + (base - raw);
+    const uint32_t bar = base + C::kBarOff;
+    volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + C::kBarOff + Bars::kAbort);
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kBarOff + Bars::kTmemSlot);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar + Bars::kQFull + 0, 1);
+        mbar_init(bar + Bars::kQFull + 8, 1);
+        mbar_init(bar + Bars::kQEmpty, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar + Bars::kSFull + 8 * t, 1);
+            mbar_init(bar + Bars::kPFull + 8 * t, kBlockM);
+            mbar_init(bar + Bars::kOFull + 8 * t, 1);
+            mbar_init(bar + Bars::kOEmpty + 8 * t, kBlockM);
+        }
+        mbar_init(bar + Bars::kDrain, 1);
+        for (int s = 0; s < C::kSlots; ++s) {
+            mbar_init(bar + Bars::kKvFull + 8 * s, 1);
+            mbar_init(bar + Bars::kKvEmpty + 8 * s, 1);
+        }
+        *abort_flag = 0u;
+        fence_barrier_init();
+        fence_proxy_async();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kLoadWarp) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t kv_i = 0;
+            uint32_t q_issued = 0;
+            bool ok = true;
+            int local = 0;
+            for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++local) {
+                const Unit w = decode_unit<CAUSAL>(u, p);
+                if (!wait_bounded(bar + Bars::kQEmpty, (local & 1) ^ 1, abort_flag, p.wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                for (int t = 0; t < 2; ++t) {
+                    const uint32_t qb = bar + Bars::kQFull + 8 * t;
+                    const uint32_t dst = base + C::kQOff + t * C::kTileBytes;
+                    mbar_expect_tx(qb, C::kTileBytes);
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_3d(dst + h * C::kHalfBytes, &tm_q, qb, h * 64, w.q0 + t * kBlockM, w.bh);
+                }
+                q_issued = local + 1;
+                for (int j = 0; ok && j < w.n1; ++j) {
+                    for (int kv = 0; kv < 2; ++kv) {
+                        const uint32_t slot = kv_i % C::kSlots;
+                        const uint32_t round = kv_i / C::kSlots;
+                        if (!wait_bounded(bar + Bars::kKvEmpty + 8 * slot, (round & 1) ^ 1, abort_flag,
+                                          p.wait_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t fb = bar + Bars::kKvFull + 8 * slot;
+                        const uint32_t dst = base + C::kRingOff + slot * C::kTileBytes;
+                        mbar_expect_tx(fb, C::kTileBytes);
+                        for (int h = 0; h < D / 64; ++h)
+                            tma_load_3d(dst + h * C::kHalfBytes, kv == 0 ? &tm_k : &tm_v, fb, h * 64,
+                                        j * kBlockN, w.bh);
+                        ++kv_i;
+                    }
+                }
+            }
+            if (!ok) {
+                // Drain: every issued copy lands before the CTA may exit.
+                const unsigned long long drain_ns = 100000000ull;
+                for (uint32_t i = (kv_i > (uint32_t)C::kSlots ? kv_i - C::kSlots : 0); i < kv_i; ++i)
+                    wait_bounded(bar + Bars::kKvFull + 8 * (i % C::kSlots), (i / C::kSlots) & 1, nullptr,
+                                 drain_ns);
+                if (q_issued > 0)
+                    for (int t = 0; t < 2; ++t)
+                        wait_bounded(bar + Bars::kQFull + 8 * t, (q_issued - 1) & 1, nullptr, drain_ns);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ----------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN, false);
+            constexpr uint32_t kIdescO = idesc_bf16_f32(kBlockM, D, true);
+            const uint32_t q_smem[2] = {base + C::kQOff, base + C::kQOff + C::kTileBytes};
+            const uint32_t s_col[2] = {C::kColS0, C::kColS1};
+            const uint32_t o_col[2] = {C::kColO0, C::kColO1};
+            uint32_t kv_i = 0;
+            uint32_t p_phase[2] = {0u, 0u};
+            bool ok = true;
+            int local = 0;
+
+            auto wait = [&](uint32_t b, uint32_t parity) {
+                if (ok && !wait_bounded(b, parity, abort_flag, p.wait_ns)) ok = false;
+                return ok;
+            };
+            // S_t = Q_t K^T  (K-major A and B, 16 columns of d per instruction)
+            auto issue_qk = [&](int t, uint32_t k_smem) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk / 4) * C::kHalfBytes + (kk % 4) * 32;
+                    mma_ss(tmem + s_col[t], sdesc_sw128(q_smem[t] + off, 16, 1024),
+                           sdesc_sw128(k_smem + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_t (+)= P_t V  (P from TMEM, V MN-major: 16 keys per instruction)
+            auto issue_pv = [&](int t, uint32_t v_smem, bool accumulate) {
+#pragma unroll
+                for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                    mma_ts(tmem + o_col[t], tmem + s_col[t] + kk * 8,
+                           sdesc_sw128(v_smem + kk * 16 * 128, C::kHalfBytes, 1024), kIdescO,
+                           (accumulate || kk > 0) ? 1u : 0u);
+                }
+            };
+            auto ring_take = [&](uint32_t& slot) {
+                slot = kv_i % C::kSlots;
+                const bool r = wait(bar + Bars::kKvFull + 8 * slot, (kv_i / C::kSlots) & 1);
+                ++kv_i;
+                return r;
+            };
+            auto ring_smem = [&](uint32_t slot) { return base + C::kRingOff + slot * C::kTileBytes; };
+
+            for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++local) {
+                const Unit w = decode_unit<CAUSAL>(u, p);
+                if (!wait(bar + Bars::kQFull + 0, local & 1) || !wait(bar + Bars::kQFull + 8, local & 1))
+                    break;
+                uint32_t ks;
+                if (!ring_take(ks)) break;
+                tc_fence_after();
+                issue_qk(0, ring_smem(ks));
+                tc_commit(bar + Bars::kSFull + 0);
+                issue_qk(1, ring_smem(ks));
+                tc_commit(bar + Bars::kSFull + 8);
+                if (w.n1 == 1) tc_commit(bar + Bars::kQEmpty);
+                tc_commit(bar + Bars::kKvEmpty + 8 * ks);
+
+                for (int j = 0; j < w.n1; ++j) {
+                    uint32_t vs, ks2 = 0;
+                    const bool has_next = j + 1 < w.n1;
+                    if (!ring_take(vs)) break;
+                    if (has_next && !ring_take(ks2)) break;
+                    if (j < w.n0) {
+                        if (!wait(bar + Bars::kPFull + 0, p_phase[0])) break;
+                        p_phase[0] ^= 1u;
+                        if (j == 0 && !wait(bar + Bars::kOEmpty + 0, (local & 1) ^ 1)) break;
+                        tc_fence_after();
+                        issue_pv(0, ring_smem(vs), j > 0);
+                        if (j + 1 < w.n0) {
+                            issue_qk(0, ring_smem(ks2));
+                            tc_commit(bar + Bars::kSFull + 0);
+                        } else {
+                            tc_commit(bar + Bars::kOFull + 0);
+                        }
+                    }
+                    if (!wait(bar + Bars::kPFull + 8, p_phase[1])) break;
+                    p_phase[1] ^= 1u;
+                    if (j == 0 && !wait(bar + Bars::kOEmpty + 8, (local & 1) ^ 1)) break;
+                    tc_fence_after();
+                    issue_pv(1, ring_smem(vs), j > 0);
+                    tc_commit(bar + Bars::kKvEmpty + 8 * vs);
+                    if (has_next) {
+                        issue_qk(1, ring_smem(ks2));
+                        tc_commit(bar + Bars::kSFull + 8);
+                        if (j + 2 == w.n1) tc_commit(bar + Bars::kQEmpty);
+                        tc_commit(bar + Bars::kKvEmpty + 8 * ks2);
+                    } else {
+                        tc_commit(bar + Bars::kOFull + 8);
+                    }
+                }
+            }
+            if (!ok) {
+                // Drain: all issued MMAs retire before TMEM is released.
+                tc_commit(bar + Bars::kDrain);
+                wait_bounded(bar + Bars::kDrain, 0, nullptr, 100000000ull);
+            }
+        }
+        __syncwarp();
+    } else {
+        // -------------------------------------------------- softmax warpgroups
+        const int t = warp >> 2;                  // Q tile of this warpgroup
+        const int quarter = warp & 3;             // TMEM lane quarter of this warp
+        const int r_in_tile = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t t_s = tmem + lane_off + (t == 0 ? C::kColS0 : C::kColS1);
+        const uint32_t t_o = tmem + lane_off + (t == 0 ? C::kColO0 : C::kColO1);
+        const uint32_t b_s = bar + Bars::kSFull + 8 * t;
+        const uint32_t b_p = bar + Bars::kPFull + 8 * t;
+        const uint32_t b_of = bar + Bars::kOFull + 8 * t;
+        const uint32_t b_oe = bar + Bars::kOEmpty + 8 * t;
+        const float sl2 = p.scale_log2;
+        uint32_t s_phase = 0;
+        bool ok = true;
+        int local = 0;
+
+        for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++local) {
+            const Unit w = decode_unit<CAUSAL>(u, p);
+            const int row = w.q0 + t * kBlockM + r_in_tile;
+            const int n_kv = (t == 0) ? w.n0 : w.n1;
+            // last visible key of this row (the row itself when causal)
+            const int last_key = CAUSAL ? min(row, p.N - 1) : p.N - 1;
+            float m = -INFINITY;  // running max of scale*log2(e)*s, log2 units
+            float l = 0.f;        // running sum of exp2(...- m)
+
+            for (int j = 0; j < n_kv; ++j) {
+                bool got = wait_bounded(b_s, s_phase, abort_flag, p.wait_ns);
+                got = __all_sync(0xffffffffu, got);
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                s_phase ^= 1u;
+                tc_fence_after();
+
+                float s[kBlockN];
+                {
+                    uint32_t r[4][32];
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(t_s + c4 * 32, r[c4]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        reg_fence32(r[c4]);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) s[c4 * 32 + c] = __uint_as_float(r[c4][c]);
+                    }
+                }
+                // key-tail and causal mask: keys past last_key get -inf
+                const int lim = last_key - j * kBlockN;
+                if (lim < kBlockN - 1) {
+#pragma unroll
+                    for (int c = 0; c < kBlockN; ++c)
+                        if (c > lim) s[c] = -INFINITY;
+                }
+                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+                for (int c = 4; c < kBlockN; c += 4) {
+                    mx0 = fmaxf(mx0, s[c]);
+                    mx1 = fmaxf(mx1, s[c + 1]);
+                    mx2 = fmaxf(mx2, s[c + 2]);
+                    mx3 = fmaxf(mx3, s[c + 3]);
+                }
+                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+                const float m_new = fmaxf(m, mx);
+                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                const float alpha = ex2(m - m_use);  // 0 on the first tile
+                const bool grow = (j > 0) && (m_new > m);
+                l *= alpha;
+                m = m_new;
+                const float neg_m = -m_use;
+                // P = exp2(scale*log2(e)*s - m), written as bf16 pairs over the S columns
+                float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const float e0 = ex2(fmaf(s[c2 * 64 + 2 * c], sl2, neg_m));
+                        const float e1 = ex2(fmaf(s[c2 * 64 + 2 * c + 1], sl2, neg_m));
+                        sum0 += e0;
+                        sum1 += e1;
+                        pk[c] = pack_bf16x2(e0, e1);
+                    }
+                    tmem_st32(t_s + c2 * 32, pk);
+                }
+                l += sum0 + sum1;
+                // O holds sum over earlier tiles of exp2(.. - m_old) v: bring it to m_new
+                // before the next P V accumulates into it.
+                if (__any_sync(0xffffffffu, grow)) {
+                    const float a = grow ? alpha : 1.f;
+#pragma unroll
+                    for (int c4 = 0; c4 < D / 32; ++c4) {
+                        uint32_t r[32];
+                        tmem_ld32(t_o + c4 * 32, r);
+                        tmem_wait_ld();
+                        reg_fence32(r);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * a);
+                        tmem_st32(t_o + c4 * 32, r);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(b_p);
+            }
+            if (!ok) break;
+
+            // ------------------------------------------------------ epilogue
+            bool got = wait_bounded(b_of, local & 1, abort_flag, p.wait_ns);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float inv_l = 1.f / l;
+            const bool store = row < p.N;
+            uint16_t* orow = out_o + (static_cast<size_t>(w.bh) * p.N + (store ? row : 0)) * D;
+#pragma unroll
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+                uint32_t r[32];
+                tmem_ld32(t_o + c4 * 32, r);
+                tmem_wait_ld();
+                reg_fence32(r);
+                if (c4 == D / 32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(b_oe);  // O_t may now be overwritten by the next unit
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
+                if (store) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                }
+            }
+            if (store) out_lse[static_cast<size_t>(w.bh) * p.N + row] = (m + __log2f(l)) * kLn2;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// A kernel that waits on a barrier nobody arrives at, to exercise the bounded
+// wait: it must give up after limit_ns, record the timeout and return.
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t b;
+    const uint32_t bar = smem_addr(&b);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) wait_bounded(bar, 0, nullptr, limit_ns);
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+typedef CUresult (*AddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+struct DriverFns {
+    EncodeTiledFn encode = nullptr;
+    AddressRangeFn range = nullptr;
+    bool ok = false;
+};
+
+DriverFns& driver_fns() {
+    static DriverFns fns;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q1, q2;
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuMemGetAddressRange", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+            q2 == cudaDriverEntryPointSuccess) {
+            fns.encode = reinterpret_cast<EncodeTiledFn>(f1);
+            fns.range = reinterpret_cast<AddressRangeFn>(f2);
+            fns.ok = true;
+        }
+    });
+    return fns;
+}
+
+// [B*H, N, d] bf16 viewed as a 3-D tensor; box = 64 columns x 128 rows x 1 head, 128-byte swizzle.
+bool encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBlockN), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return driver_fns().encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The pointer must be device memory of `device` and its allocation must hold `bytes` from it.
+bool device_span_ok(const void* ptr, size_t bytes, int device) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return false;
+    if (a.device != device) return false;
+    CUdeviceptr lo = 0;
+    size_t size = 0;
+    if (driver_fns().range(&lo, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return false;
+    const uintptr_t p = reinterpret_cast<uintptr_t>(ptr);
+    return p >= lo && bytes <= size && p - lo <= size - bytes;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+template <int D, bool CAUSAL>
+int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
+           const Params& p, int grid, cudaStream_t stream) {
+    auto kernel = attn_fwd_kernel<D, CAUSAL>;
+    const int smem = Cfg<D>::kSmemBytes;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    kernel<<<grid, kThreads, smem, stream>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_version(void) { return 100; }
+
+const char* attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported head size (d must be 64 or 128)";
+        case ATTN_ERR_CUDA: return "CUDA call failed";
+        case ATTN_ERR_TIMEOUT: return "a bounded device wait ran out";
+        default: return "unknown status";
+    }
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+             float scale, int causal, attn_stream_t stream) {
+    // ---- host-side validation: nothing touches the GPU until all of it passes
+    if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    // scale must be a positive, finite fp32: masked keys are -inf scores and the
+    // row maximum is taken before scaling.
+    if (!isfinite(scale) || !(scale >= 1e-30f)) return ATTN_ERR_INVALID_ARG;
+    const long long BH = static_cast<long long>(B) * H;
+    if (BH > 0x7fffffffLL || N > 0x7fffffff - kUnitRows) return ATTN_ERR_INVALID_ARG;
+    auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
+    if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) || misaligned(lse, 4))
+        return ATTN_ERR_INVALID_ARG;
+    const size_t elems = static_cast<size_t>(BH) * N * d;
+    const size_t tbytes = elems * 2, lbytes = static_cast<size_t>(BH) * N * 4;
+    if (overlaps(o, tbytes, q, tbytes) || overlaps(o, tbytes, k, tbytes) || overlaps(o, tbytes, v, tbytes) ||
+        overlaps(lse, lbytes, q, tbytes) || overlaps(lse, lbytes, k, tbytes) || overlaps(lse, lbytes, v, tbytes) ||
+        overlaps(lse, lbytes, o, tbytes))
+        return ATTN_ERR_INVALID_ARG;
+
+    if (!driver_fns().ok) return ATTN_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (!device_span_ok(q, tbytes, dev) || !device_span_ok(k, tbytes, dev) || !device_span_ok(v, tbytes, dev) ||
+        !device_span_ok(o, tbytes, dev) || !device_span_ok(lse, lbytes, dev))
+        return ATTN_ERR_INVALID_ARG;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return ATTN_ERR_CUDA;
+
+    alignas(64) CUtensorMap mq, mk, mv;
+    if (!encode_qkv_map(&mq, q, static_cast<int>(BH), N, d) || !encode_qkv_map(&mk, k, static_cast<int>(BH), N, d) ||
+        !encode_qkv_map(&mv, v, static_cast<int>(BH), N, d))
+        return ATTN_ERR_CUDA;
+
+    Params p;
+    p.BH = static_cast<int>(BH);
+    p.N = N;
+    p.n_pairs = (N + kUnitRows - 1) / kUnitRows;
+    p.n_kv_all = (N + kBlockN - 1) / kBlockN;
+    const long long units = BH * p.n_pairs;
+    if (units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    p.total_units = static_cast<int>(units);
+    p.scale_log2 = scale * kLog2e;
+    p.wait_ns = kDefaultWaitNs;
+    const int grid = static_cast<int>(units < sms ? units : sms);
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 64) {
+        return causal ? launch<64, true>(mq, mk, mv, o, lse, p, grid, s) : launch<64, false>(mq, mk, mv, o, lse, p, grid, s);
+    }
+    return causal ? launch<128, true>(mq, mk, mv, o, lse, p, grid, s) : launch<128, false>(mq, mk, mv, o, lse, p, grid, s);
+}
+
+int attn_check_device_status(attn_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+    int status = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&status, g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return status == 0 ? ATTN_OK : status;
+}
+
+int attn_selftest_wait_timeout(unsigned long long limit_ns, attn_stream_t stream) {
+    if (limit_ns < 1000ull || limit_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
+    wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

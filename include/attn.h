@@ -1,0 +1,91 @@
+/*
+ * attn.h -- C ABI of the exact, IO-aware attention forward library (libattn.so).
+ *
+ * The operation (FlashAttention: Fast and Memory-Efficient Exact Attention
+ * with IO-Awareness, wiki notes, sections "Problem setting", "Tiling",
+ * "Recomputation" and "Kernel fusion"): for every batch b and head h,
+ *
+ *     O[b,h] = softmax(scale * Q[b,h] K[b,h]^T) V[b,h]
+ *     LSE[b,h,i] = ln sum_j exp(scale * q_i . k_j)        (natural log)
+ *
+ * computed tile by tile in one kernel with a running row maximum m and a
+ * running row sum l, so the N x N score and probability matrices never reach
+ * device memory; the softmax statistics are kept as one fp32 log-sum-exp per
+ * query row (the notes' "keep only O and the softmax statistics (m, l)").
+ * With causal != 0, key j is visible to query i iff j <= i (square, top-left
+ * aligned); tiles entirely above the diagonal are never computed.
+ *
+ * Every pointer is a DEVICE pointer on the current CUDA device.  The caller
+ * owns every buffer; the library allocates no device memory and keeps no
+ * pointer after a call returns.  Calls are asynchronous on `stream` and never
+ * synchronise the host.
+ */
+#ifndef EXACT_ATTN_H
+#define EXACT_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; 0 is the legacy default stream. */
+typedef struct CUstream_st* attn_stream_t;
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or scale          */
+    ATTN_ERR_UNSUPPORTED = 2,  /* head size other than 64 or 128                  */
+    ATTN_ERR_CUDA = 3,         /* a CUDA runtime or driver call failed            */
+    ATTN_ERR_TIMEOUT = 4       /* a bounded wait inside a kernel ran out (device) */
+} attn_status;
+
+/*
+ * attn_fwd -- exact attention forward.
+ *
+ *   q, k, v : bf16 [B, H, N, d], contiguous, 16-byte aligned, read only.
+ *   o       : bf16 [B, H, N, d], contiguous, 16-byte aligned, written.
+ *   lse     : fp32 [B, H, N], contiguous, 4-byte aligned, written: natural-log
+ *             log-sum-exp of the scaled scores of each query row.
+ *   B, H, N : >= 1;  B*H <= 2^31-1;  N <= 2^31-1 - 256.
+ *   d       : 64 or 128 (other values return ATTN_ERR_UNSUPPORTED).
+ *   scale   : finite and >= 1e-30 (positive); the usual choice is 1/sqrt(d).
+ *             Scores scale * q.k must be finite in fp32.
+ *   causal  : 0 = every key visible; nonzero = key j visible to query i iff j <= i.
+ *   stream  : CUDA stream the kernel is queued on.
+ *
+ * Each pointer must lie in device memory of the current device, and the
+ * allocation that holds it must cover the whole tensor (checked on the host,
+ * before anything is launched: violations return ATTN_ERR_INVALID_ARG and
+ * nothing is written).  o and lse must not overlap q, k or v.
+ * Returns ATTN_OK once the kernel is queued.  A device-side failure (a wait
+ * that ran out) is reported later by attn_check_device_status().
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
+
+/* Human-readable name of an attn_status value (static string, never NULL). */
+const char* attn_status_string(int status);
+
+/*
+ * attn_check_device_status -- synchronise `stream`, then read and clear the
+ * library's device status word on the current device.  Returns ATTN_OK,
+ * ATTN_ERR_TIMEOUT if any kernel of this library gave up on a bounded wait
+ * since the last check (its outputs are then undefined), or ATTN_ERR_CUDA.
+ */
+int attn_check_device_status(attn_stream_t stream);
+
+/*
+ * attn_selftest_wait_timeout -- exercise the bounded-wait path without any
+ * fault: queue on `stream` one tiny kernel that waits on a barrier nobody
+ * arrives at, with a limit of `limit_ns` nanoseconds (1e3 .. 1e10).  The wait
+ * gives up, records ATTN_ERR_TIMEOUT in the device status word and the kernel
+ * returns normally; attn_check_device_status() then reports it.
+ */
+int attn_selftest_wait_timeout(unsigned long long limit_ns, attn_stream_t stream);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EXACT_ATTN_H */

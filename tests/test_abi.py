@@ -1,0 +1,117 @@
+"""The C ABI library: it loads, exports every declared entry point, and rejects
+bad arguments on the host before touching a GPU (these run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_io_aware_102_b200 as pkg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(attn_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(pkg.LIB_PATH):
+        from exact_io_aware_102_b200 import build
+        build.build()
+    return pkg.library()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert {"attn_fwd", "attn_status_string", "attn_check_device_status",
+            "attn_selftest_wait_timeout", "attn_version"} <= set(names)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(pkg.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+
+
+def test_status_strings(lib):
+    assert pkg.attn_status_string(pkg.ATTN_OK) == "ok"
+    for s in range(1, 5):
+        assert pkg.attn_status_string(s) not in ("", "unknown status")
+    assert pkg.attn_status_string(99) == "unknown status"
+    assert pkg.attn_version() >= 100
+
+
+FAKE = 0x10000  # an aligned address: never dereferenced, validation fails first
+
+
+@pytest.mark.parametrize("B,H,N,d,scale,expect", [
+    (1, 1, 128, 96, 0.125, pkg.ATTN_ERR_UNSUPPORTED),
+    (1, 1, 128, 32, 0.125, pkg.ATTN_ERR_UNSUPPORTED),
+    (0, 1, 128, 64, 0.125, pkg.ATTN_ERR_INVALID_ARG),
+    (1, 0, 128, 64, 0.125, pkg.ATTN_ERR_INVALID_ARG),
+    (1, 1, 0, 64, 0.125, pkg.ATTN_ERR_INVALID_ARG),
+    (1, 1, -5, 64, 0.125, pkg.ATTN_ERR_INVALID_ARG),
+    (1, 1, 128, 64, float("nan"), pkg.ATTN_ERR_INVALID_ARG),
+    (1, 1, 128, 64, float("inf"), pkg.ATTN_ERR_INVALID_ARG),
+    (1, 1, 128, 64, 0.0, pkg.ATTN_ERR_INVALID_ARG),
+    (1, 1, 128, 64, -0.125, pkg.ATTN_ERR_INVALID_ARG),
+    (65536, 65536, 128, 64, 0.125, pkg.ATTN_ERR_INVALID_ARG),
+    (1, 1, 2**31 - 100, 64, 0.125, pkg.ATTN_ERR_INVALID_ARG),
+])
+def test_bad_sizes_rejected_on_host(lib, B, H, N, d, scale, expect):
+    assert pkg.attn_fwd(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5, B, H, N, d, scale, 0, None) == expect
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    ok = [FAKE, FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5]
+    for i in range(5):
+        ptrs = list(ok)
+        ptrs[i] = None
+        assert pkg.attn_fwd(*ptrs, 1, 1, 64, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    for i in range(4):  # q, k, v, o need 16-byte alignment
+        ptrs = list(ok)
+        ptrs[i] += 8
+        assert pkg.attn_fwd(*ptrs, 1, 1, 64, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    ptrs = list(ok)
+    ptrs[4] += 2  # lse needs 4-byte alignment
+    assert pkg.attn_fwd(*ptrs, 1, 1, 64, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+
+
+def test_overlapping_outputs_rejected(lib):
+    base = 1 << 20
+    n_bytes = 1 * 2 * 64 * 64 * 2
+    # o overlapping q
+    assert pkg.attn_fwd(base, base + 2 * n_bytes, base + 4 * n_bytes, base + 16, base + 8 * n_bytes,
+                        1, 2, 64, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    # lse overlapping o
+    assert pkg.attn_fwd(base, base + 2 * n_bytes, base + 4 * n_bytes, base + 6 * n_bytes,
+                        base + 6 * n_bytes + 64, 1, 2, 64, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+
+
+def test_selftest_limit_validated(lib):
+    assert pkg.attn_selftest_wait_timeout(10, 0) == pkg.ATTN_ERR_INVALID_ARG
+    assert pkg.attn_selftest_wait_timeout(10**11, 0) == pkg.ATTN_ERR_INVALID_ARG
+
+
+def test_forward_rejects_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        pkg.forward(q, q, q)
+    with pytest.raises(ValueError):
+        pkg.forward(q.float(), q.float(), q.float())
+
+
+def test_product_path_does_not_import_the_oracle():
+    # The package and its sources never reference the oracle.
+    pkg_dir = os.path.join(ROOT, "exact_io_aware_102_b200")
+    for dirpath, _, files in os.walk(pkg_dir):
+        for f in files:
+            if f.endswith((".py", ".cu", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "attn_oracle" not in text, f
