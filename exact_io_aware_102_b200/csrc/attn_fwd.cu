@@ -44,9 +44,17 @@ namespace {
 constexpr int kBlockM = 128;           // query rows per Q tile (= TMEM lanes)
 constexpr int kBlockN = 128;           // keys per K / V tile
 constexpr int kUnitRows = 2 * kBlockM;  // query rows per work unit
-constexpr int kThreads = 320;          // 2 softmax warpgroups + load warp + MMA warp
+constexpr int kThreads = 384;          // softmax WG 0, softmax WG 1, WG 2 = {load, MMA, 2 idle}
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
+// Register split (setmaxnreg): the block launches with 384 x 168 registers;
+// the two softmax warpgroups take 192 each, warpgroup 2 keeps 120
+// (256 x 192 + 128 x 120 = 384 x 168).
+constexpr int kSoftmaxRegs = 192;
+constexpr int kOtherRegs = 120;
+// The reference maximum of a row moves only when the row maximum exceeds it
+// by more than this many powers of two; O and l always share the reference.
+constexpr float kLazyRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -117,7 +125,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Gives up after `limit_ns` (then raises the CTA abort flag and the device
 // status word) or as soon as another thread of the CTA has raised the abort
 // flag.  Returns false when it gave up.
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
                                        unsigned long long limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     uint32_t n = 0;
@@ -255,6 +263,43 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
+template <int R>
+__device__ __forceinline__ void regs_increase() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R>
+__device__ __forceinline__ void regs_decrease() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for x <= 8 on the FMA/ALU pipes (no MUFU), two lanes at a time:
+// x = j + f with j = round(x) and f in [-1/2, 1/2]; 2^f from a degree-3
+// polynomial fitted for minimal relative error on [-1/2, 1/2]
+// (fit_exp2_poly.py; max relative error 7.6e-5, far below the bf16 rounding
+// that P gets); 2^j by adding j to the exponent field.  x is clamped at -126
+// so the exponent never wraps (2^-126 stands in for 0).
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
+    constexpr float kC0 = 0.99992824f, kC1 = 0.6932636f, kC2 = 0.2426099f, kC3 = 0.05515746f;
+    x.x = fmaxf(x.x, -126.0f);
+    x.y = fmaxf(x.y, -126.0f);
+    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+    const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
+    const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+    float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+    q = __ffma2_rn(q, f, make_float2(kC1, kC1));
+    q = __ffma2_rn(q, f, make_float2(kC0, kC0));
+    // the low mantissa bits of t hold j (two's complement); shifting by 23 moves them to the exponent
+    const uint32_t rx = __float_as_uint(q.x) + (__float_as_uint(t.x) << 23);
+    const uint32_t ry = __float_as_uint(q.y) + (__float_as_uint(t.y) << 23);
+    return make_float2(__uint_as_float(rx), __uint_as_float(ry));
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: version
 // field 1 at bit 46, layout type 2 = SWIZZLE_128B at bits 61..63).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
@@ -363,7 +408,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kLoadWarp) {
+    if (warp >= kLoadWarp) {
+      regs_decrease<kOtherRegs>();
+      if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             uint32_t kv_i = 0;
@@ -415,7 +462,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
+      } else if (warp == kMmaWarp) {
         // ----------------------------------------------------------- MMA issue
         if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN, false);
@@ -513,7 +560,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         __syncwarp();
+      }
     } else {
+        regs_increase<kSoftmaxRegs>();
         // -------------------------------------------------- softmax warpgroups
         const int t = warp >> 2;                  // Q tile of this warpgroup
         const int quarter = warp & 3;             // TMEM lane quarter of this warp
@@ -536,8 +585,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int n_kv = (t == 0) ? w.n0 : w.n1;
             // last visible key of this row (the row itself when causal)
             const int last_key = CAUSAL ? min(row, p.N - 1) : p.N - 1;
-            float m = -INFINITY;  // running max of scale*log2(e)*s, log2 units
-            float l = 0.f;        // running sum of exp2(...- m)
+            float m = -INFINITY;  // reference max of scale*log2(e)*s (log2 units), shared by O and l
+            float l = 0.f;        // sum of exp2(scale*log2(e)*s - m) over the keys seen so far
 
             for (int j = 0; j < n_kv; ++j) {
                 bool got = wait_bounded(b_s, s_phase, abort_flag, p.wait_ns);
@@ -569,42 +618,58 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int c = 0; c < kBlockN; ++c)
                         if (c > lim) s[c] = -INFINITY;
                 }
-                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+                // row maximum (scale > 0, so it is taken on the raw scores)
+                float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-                for (int c = 4; c < kBlockN; c += 4) {
-                    mx0 = fmaxf(mx0, s[c]);
-                    mx1 = fmaxf(mx1, s[c + 1]);
-                    mx2 = fmaxf(mx2, s[c + 2]);
-                    mx3 = fmaxf(mx3, s[c + 3]);
+                for (int c = 4; c < kBlockN; c += 8) {
+                    mx[0] = fmax3(mx[0], s[c], s[c + 1]);
+                    mx[1] = fmax3(mx[1], s[c + 2], s[c + 3]);
+                    if (c + 4 < kBlockN) {
+                        mx[2] = fmax3(mx[2], s[c + 4], s[c + 5]);
+                        mx[3] = fmax3(mx[3], s[c + 6], s[c + 7]);
+                    }
                 }
-                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-                const float m_new = fmaxf(m, mx);
-                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-                const float alpha = ex2(m - m_use);  // 0 on the first tile
-                const bool grow = (j > 0) && (m_new > m);
+                const float row_max = fmax3(fmax3(mx[0], mx[1], mx[2]), mx[3], -INFINITY) * sl2;
+                // lazy rescaling: move the reference only when the row maximum
+                // exceeds it by more than 2^8 (always on the first tile)
+                const bool move = row_max > m + kLazyRescaleLog2;
+                float alpha = 1.f;
+                if (move) {
+                    alpha = ex2(m - row_max);  // 0 when m was -inf
+                    m = row_max;
+                }
                 l *= alpha;
-                m = m_new;
-                const float neg_m = -m_use;
-                // P = exp2(scale*log2(e)*s - m), written as bf16 pairs over the S columns
-                float sum0 = 0.f, sum1 = 0.f;
+                const float m_use = (m == -INFINITY) ? 0.f : m;
+                const float2 sl2x2 = make_float2(sl2, sl2);
+                const float2 negm = make_float2(-m_use, -m_use);
+
+                // P = exp2(scale*log2(e)*s - m) as bf16 pairs over the S columns;
+                // 3 of every 8 pairs use the FMA-pipe exponential, the rest MUFU.
+                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c2 = 0; c2 < 2; ++c2) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const float e0 = ex2(fmaf(s[c2 * 64 + 2 * c], sl2, neg_m));
-                        const float e1 = ex2(fmaf(s[c2 * 64 + 2 * c + 1], sl2, neg_m));
-                        sum0 += e0;
-                        sum1 += e1;
-                        pk[c] = pack_bf16x2(e0, e1);
+                        const int e = c2 * 64 + 2 * c;
+                        float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sl2x2, negm);
+                        if ((c & 7) >= 5) {
+                            x = ex2_poly2(x);
+                        } else {
+                            x.x = ex2(x.x);
+                            x.y = ex2(x.y);
+                        }
+                        acc = __fadd2_rn(acc, x);
+                        pk[c] = pack_bf16x2(x.x, x.y);
                     }
                     tmem_st32(t_s + c2 * 32, pk);
                 }
-                l += sum0 + sum1;
-                // O holds sum over earlier tiles of exp2(.. - m_old) v: bring it to m_new
-                // before the next P V accumulates into it.
-                if (__any_sync(0xffffffffu, grow)) {
-                    const float a = grow ? alpha : 1.f;
+                l += acc.x + acc.y;
+                // O holds the sum over earlier tiles at the old reference:
+                // bring it to the new one before the next P V accumulates.
+                const bool rescale = move && j > 0;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    const float a = rescale ? alpha : 1.f;
 #pragma unroll
                     for (int c4 = 0; c4 < D / 32; ++c4) {
                         uint32_t r[32];
