@@ -12,15 +12,19 @@
 //
 // How it maps to sm_100a (the page's A100 design is prior art, not followed):
 //   * persistent grid, one CTA per SM, each CTA walks work units
-//     (b, h, 256 query rows = two 128-row Q tiles);
-//   * warp 8 (one lane) issues TMA loads: the two Q tiles once per unit and a
-//     ring of K / V tiles (128 keys each) guarded by full/empty mbarriers;
-//   * warp 9 (one lane) issues tcgen05.mma: S_t = Q_t K_j^T into TMEM
-//     (fp32, 128 x 128), then O_t += P_t V_j with P_t read from TMEM;
+//     (b, h, 256 query rows = two 128-row Q tiles), 12 warps;
+//   * warp 8 (one lane) issues TMA loads: the two Q tiles once per unit and
+//     K / V tiles of 128 keys into shared-memory rings guarded by full/empty
+//     mbarriers;
+//   * tcgen05.mma computes S_t = Q_t K_j^T into TMEM (fp32, 128 x 128) and
+//     O_t += P_t V_j with P_t read from TMEM.  At d = 64, P_t has TMEM columns
+//     of its own, so the S stream (warp 9) and the P V stream (warp 10) are
+//     issued by two threads and neither waits behind the other; at d = 128,
+//     P_t overlays S_t and warp 9 issues both in one ordered stream;
 //   * warps 0-3 and 4-7 are the softmax warpgroups of Q tiles 0 and 1: one
 //     thread per query row reads its S row from TMEM, masks, updates m and l,
-//     rescales its O row in TMEM when m grows, writes P (bf16) back over S,
-//     and at the end normalises O by l and stores O and LSE;
+//     writes P (bf16), rescales its O row in TMEM when m moves, and at the
+//     end normalises O by l and stores O and LSE;
 //   * every mbarrier wait is bounded; on timeout a status word is set, the
 //     CTA drains its in-flight copies and MMAs, frees TMEM and returns.
 //
@@ -28,7 +32,8 @@
 // Shared memory tiles use the 128-byte swizzle (TMA writes them, the tensor
 // cores read them through matrix descriptors); d = 128 tiles are stored as two
 // 64-column halves.  TMEM: S0 cols [0,128), S1 [128,256), O0 [256,256+d),
-// O1 [256+d, 256+2d); P_t overlays the first 64 columns of S_t.
+// O1 [256+d, 256+2d); P0, P1 at [384,448), [448,512) for d = 64, over the
+// first 64 columns of S0, S1 for d = 128.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -44,9 +49,10 @@ namespace {
 constexpr int kBlockM = 128;           // query rows per Q tile (= TMEM lanes)
 constexpr int kBlockN = 128;           // keys per K / V tile
 constexpr int kUnitRows = 2 * kBlockM;  // query rows per work unit
-constexpr int kThreads = 384;          // softmax WG 0, softmax WG 1, WG 2 = {load, MMA, 2 idle}
+constexpr int kThreads = 384;          // softmax WG 0, softmax WG 1, WG 2 = {load, MMA S, MMA PV, idle}
 constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;            // S stream (and, at d = 128, the P V stream too)
+constexpr int kMmaPvWarp = 10;         // P V stream at d = 64
 // Register split (setmaxnreg): the block launches with 384 x 168 registers;
 // the two softmax warpgroups take 192 each, warpgroup 2 keeps 120
 // (256 x 192 + 128 x 120 = 384 x 168).
@@ -55,37 +61,59 @@ constexpr int kOtherRegs = 120;
 // The reference maximum of a row moves only when the row maximum exceeds it
 // by more than this many powers of two; O and l always share the reference.
 constexpr float kLazyRescaleLog2 = 8.0f;
+// Of every 8 exponential pairs, this many run on the FMA-pipe polynomial and
+// the rest on MUFU (ex2.approx).
+#ifndef ATTN_POLY_PAIRS_PER_8
+#define ATTN_POLY_PAIRS_PER_8 2
+#endif
+constexpr int kPolyPairsPer8 = ATTN_POLY_PAIRS_PER_8;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s per wait
+constexpr unsigned long long kDrainWaitNs = 100000000ull;     // 0.1 s per drain wait
 
 template <int D>
 struct Cfg {
     static constexpr int kHalfBytes = kBlockN * 64 * 2;       // one 128 x 64 bf16 swizzled half
     static constexpr int kTileBytes = kBlockN * D * 2;        // one Q, K or V tile
-    static constexpr int kSlots = (D == 64) ? 8 : 4;          // K/V ring depth
+    // d = 64: P_t has its own 64 TMEM columns after O, so S_t can be refilled
+    // as soon as the softmax has loaded it, and the S and P V streams are
+    // independent (two issuing threads, a K ring and a V ring).  d = 128: no
+    // TMEM room; P_t overlays S_t and one thread issues P_t V before S_t.
+    static constexpr bool kSplit = (D == 64);
+    static constexpr int kKSlots = kSplit ? 4 : 4;            // split: K ring; else the shared K/V ring
+    static constexpr int kVSlots = kSplit ? 4 : 0;            // split: V ring
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = 2 * kTileBytes;
-    static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+    static constexpr int kVRingOff = kRingOff + kKSlots * kTileBytes;
+    static constexpr int kBarOff = kVRingOff + kVSlots * kTileBytes;
     static constexpr int kSmemBytes = kBarOff + 512 + 1024;   // barriers + 1 KB alignment slack
     static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
-    static_assert(256 + 2 * D <= (int)kTmemCols, "TMEM budget");
+    static constexpr uint32_t kColP0 = kSplit ? 256 + 2 * D : kColS0;
+    static constexpr uint32_t kColP1 = kSplit ? 256 + 2 * D + 64 : kColS1;
+    static_assert(256 + 2 * D + (kSplit ? 128 : 0) <= (int)kTmemCols, "TMEM budget");
+    static_assert(kKSlots <= 8 && kVSlots <= 8, "barrier block holds 8 + 8 ring slots");
 };
 
-// Barrier block (offsets in bytes from the barrier area).
+// Barrier block (offsets in bytes from the barrier area).  No barrier can
+// complete twice before its consumer has waited on it.
 struct Bars {
-    static constexpr int kQFull = 0;                 // [2]
-    static constexpr int kQEmpty = 16;               // [1]
-    static constexpr int kSFull = 24;                // [2]
-    static constexpr int kPFull = 40;                // [2]
-    static constexpr int kOFull = 56;                // [2]
-    static constexpr int kOEmpty = 72;               // [2]
-    static constexpr int kDrain = 88;                // [1]
-    static constexpr int kTmemSlot = 96;             // u32: TMEM base address
-    static constexpr int kAbort = 100;               // u32: abort flag
-    static constexpr int kKvFull = 128;              // [slots]
-    static constexpr int kKvEmpty = 128 + 8 * 8;     // [slots]
+    static constexpr int kQFull = 0;       // [2] TMA -> MMA: Q tile t landed
+    static constexpr int kQEmpty = 16;     // [1] MMA -> TMA: the unit's last S MMA retired
+    static constexpr int kSFull = 24;      // [2] MMA -> softmax t: S_t computed
+    static constexpr int kPFull = 40;      // [2] softmax t -> MMA: P_t written (and O_t rescaled)
+    static constexpr int kOFull = 56;      // [2] MMA -> softmax t: O_t of the unit complete
+    static constexpr int kOEmpty = 72;     // [2] softmax t -> MMA: O_t read out
+    static constexpr int kDrain = 88;      // [2] one per MMA-issuing thread
+    static constexpr int kSFree = 104;     // [2] softmax t -> MMA: S_t loaded (split layout)
+    static constexpr int kPFree = 120;     // [2] MMA -> softmax t: P_t V retired (split layout)
+    static constexpr int kTmemSlot = 136;  // u32: TMEM base address
+    static constexpr int kAbort = 140;     // u32: abort flag
+    static constexpr int kKFull = 144;     // [8] TMA -> MMA: K (or K/V) ring slot landed
+    static constexpr int kKEmpty = 208;    // [8] MMA -> TMA: K (or K/V) ring slot free
+    static constexpr int kVFull = 272;     // [8] V ring (split layout)
+    static constexpr int kVEmpty = 336;    // [8]
 };
 
 __device__ int g_attn_status = 0;   // 0 = fine; ATTN_ERR_TIMEOUT after a wait ran out
@@ -190,24 +218,28 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                      bar)
                  : "memory");
 }
-// D[tmem] (+)= A[smem desc] * B[smem desc]
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
+// The same two MMAs with the shared-memory descriptors passed as 32-bit
+// halves: the high word is a per-operand constant and the low word is
+// (address >> 4) | (LBO >> 4) << 16, so stepping an operand is one add.
+__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                          uint32_t idesc, uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 da, {%1, %3};\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem desc]
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
+__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                          uint32_t idesc, uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -300,16 +332,15 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
     return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: version
-// field 1 at bit 46, layout type 2 = SWIZZLE_128B at bits 61..63).
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-    d |= static_cast<uint64_t>(1) << 46;
-    d |= static_cast<uint64_t>(2) << 61;
-    return d;
+// Shared-memory matrix descriptor for the 128-byte swizzle, as two 32-bit
+// words (tcgen05 format): low = start address >> 4 (bits 0-13) | leading
+// byte offset >> 4 (bits 16-29); high = stride byte offset >> 4 (bits 0-13),
+// version 1 (bit 14), layout type 2 = SWIZZLE_128B (bits 29-31).
+__host__ __device__ constexpr uint32_t sdesc_hi_sw128(uint32_t sbo_bytes) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+    return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
 }
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, A K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool b_mn_major) {
@@ -328,12 +359,14 @@ struct Params {
 };
 
 struct Unit {
-    int bh, q0, n0, n1;  // head, first query row, KV tiles for Q tile 0 / 1
+    int bh, q0, n0, n1;  // head, first query row, key tiles for Q tile 0 / 1
 };
 
 // Work units: (head, pair of Q tiles).  Non-causal: heads-major so the CTAs
 // running at one time share K/V of few heads (L2 reuse).  Causal: the pairs
-// with the most key tiles first, so the short units fill the tail.
+// with the most key tiles first, so the short units fill the tail; a Q tile
+// stops at the key tile holding its last row (tiles above the diagonal are
+// never loaded or multiplied).
 template <bool CAUSAL>
 __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     Unit w;
@@ -347,14 +380,441 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     }
     w.q0 = pair * kUnitRows;
     if (CAUSAL) {
-        const int need1 = (w.q0 + kUnitRows) / kBlockN;  // tiles touching rows < q0 + 256
-        const int need0 = w.q0 / kBlockN + 1;            // tiles touching rows < q0 + 128
-        w.n1 = min(p.n_kv_all, need1);
-        w.n0 = min(w.n1, need0);
+        w.n1 = min(p.n_kv_all, (w.q0 + kUnitRows) / kBlockN);  // tiles touching rows < q0 + 256
+        w.n0 = min(w.n1, w.q0 / kBlockN + 1);                 // tiles touching rows < q0 + 128
     } else {
         w.n0 = w.n1 = p.n_kv_all;
     }
     return w;
+}
+
+// What every role of one CTA shares.
+struct Ctx {
+    uint32_t base;   // shared-memory base (1 KB aligned)
+    uint32_t bar;    // barrier block
+    uint32_t tmem;   // TMEM base address
+    volatile uint32_t* abort_flag;
+    Params p;
+};
+
+// A ring of shared-memory tiles with full/empty barriers, walked in order.
+struct Ring {
+    uint32_t smem, full, empty, slots, i;
+    __device__ __forceinline__ uint32_t slot() const { return i % slots; }
+    __device__ __forceinline__ uint32_t phase() const { return (i / slots) & 1u; }
+};
+
+// ------------------------------------------------------------ TMA producer
+// Per unit: Q0, Q1 once; then the key tiles in the order the MMA warps use
+// them (split: K_j into the K ring and V_j into the V ring; shared ring:
+// K_j then V_j).
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void role_producer(const Ctx& c, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                              const CUtensorMap* tm_v) {
+    using C = Cfg<D>;
+    Ring rk{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
+    Ring rv{c.base + C::kVRingOff, c.bar + Bars::kVFull, c.bar + Bars::kVEmpty, (uint32_t)C::kVSlots, 0};
+    uint32_t q_issued = 0;
+    bool ok = true;
+    auto load = [&](Ring& r, const CUtensorMap* map, int key0, int bh) {
+        const uint32_t s = r.slot();
+        if (!wait_bounded(r.empty + 8 * s, r.phase() ^ 1u, c.abort_flag, c.p.wait_ns)) return false;
+        const uint32_t fb = r.full + 8 * s;
+        const uint32_t dst = r.smem + s * C::kTileBytes;
+        mbar_expect_tx(fb, C::kTileBytes);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) tma_load_3d(dst + h * C::kHalfBytes, map, fb, h * 64, key0, bh);
+        ++r.i;
+        return true;
+    };
+    int local = 0;
+    for (int u = blockIdx.x; ok && u < c.p.total_units; u += gridDim.x, ++local) {
+        const Unit w = decode_unit<CAUSAL>(u, c.p);
+        if (!wait_bounded(c.bar + Bars::kQEmpty, (local & 1) ^ 1, c.abort_flag, c.p.wait_ns)) {
+            ok = false;
+            break;
+        }
+        for (int t = 0; t < 2; ++t) {
+            const uint32_t qb = c.bar + Bars::kQFull + 8 * t;
+            const uint32_t dst = c.base + C::kQOff + t * C::kTileBytes;
+            mbar_expect_tx(qb, C::kTileBytes);
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+                tma_load_3d(dst + h * C::kHalfBytes, tm_q, qb, h * 64, w.q0 + t * kBlockM, w.bh);
+        }
+        q_issued = local + 1;
+        for (int j = 0; ok && j < w.n1; ++j) {
+            ok = load(rk, tm_k, j * kBlockN, w.bh);
+            if (ok) ok = load(C::kSplit ? rv : rk, tm_v, j * kBlockN, w.bh);
+        }
+    }
+    if (!ok) {
+        // Drain: every issued copy lands before the CTA may exit.
+        for (Ring* r : {&rk, &rv})
+            for (uint32_t i = (r->i > r->slots ? r->i - r->slots : 0); i < r->i; ++i)
+                wait_bounded(r->full + 8 * (i % r->slots), (i / r->slots) & 1, nullptr, kDrainWaitNs);
+        if (q_issued > 0)
+            for (int t = 0; t < 2; ++t)
+                wait_bounded(c.bar + Bars::kQFull + 8 * t, (q_issued - 1) & 1, nullptr, kDrainWaitNs);
+    }
+}
+
+// ---------------------------------------------------------- MMA issuing
+template <int D>
+struct Mma {
+    static constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN, false);
+    static constexpr uint32_t kIdescO = idesc_bf16_f32(kBlockM, D, true);
+    static constexpr uint32_t kHi = sdesc_hi_sw128(1024);
+    using C = Cfg<D>;
+    // S_t = Q_t K^T: K-major A (Q tile) and B (K tile), 16 columns of d per instruction
+    __device__ __forceinline__ static void qk(const Ctx& c, int t, uint32_t k_smem) {
+        const uint32_t a0 = sdesc_lo(c.base + C::kQOff + t * C::kTileBytes, 16);
+        const uint32_t b0 = sdesc_lo(k_smem, 16);
+        const uint32_t d = c.tmem + (t == 0 ? C::kColS0 : C::kColS1);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * C::kHalfBytes + (kk % 4) * 32) >> 4;
+            mma_ss_lo(d, a0 + off, b0 + off, kHi, kIdescS, kk > 0 ? 1u : 0u);
+        }
+    }
+    // O_t (+)= P_t V: P from TMEM, V tile MN-major (LBO = one 64-column half), 16 keys per instruction
+    __device__ __forceinline__ static void pv(const Ctx& c, int t, uint32_t v_smem, bool accumulate) {
+        const uint32_t b0 = sdesc_lo(v_smem, C::kHalfBytes);
+        const uint32_t d = c.tmem + (t == 0 ? C::kColO0 : C::kColO1);
+        const uint32_t a = c.tmem + (t == 0 ? C::kColP0 : C::kColP1);
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk)
+            mma_ts_lo(d, a + kk * 8, b0 + ((kk * 16 * 128) >> 4), kHi, kIdescO, (accumulate || kk > 0) ? 1u : 0u);
+    }
+};
+
+// Bounded wait for the MMA-issuing threads: false once anything gave up.
+struct Waiter {
+    const Ctx& c;
+    bool ok;
+    __device__ __forceinline__ bool operator()(uint32_t b, uint32_t parity) {
+        if (ok && !wait_bounded(b, parity, c.abort_flag, c.p.wait_ns)) ok = false;
+        return ok;
+    }
+    __device__ __forceinline__ bool take(Ring& r, uint32_t& slot) {
+        slot = r.slot();
+        const bool got = (*this)(r.full + 8 * slot, r.phase());
+        ++r.i;
+        return got;
+    }
+};
+
+__device__ __forceinline__ void mma_drain(const Ctx& c, int which) {
+    tc_commit(c.bar + Bars::kDrain + 8 * which);
+    wait_bounded(c.bar + Bars::kDrain + 8 * which, 0, nullptr, kDrainWaitNs);
+}
+
+// Split layout, S stream: S_t(j) once the softmax has loaded S_t(j-1).
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void role_mma_s(const Ctx& c) {
+    using C = Cfg<D>;
+    Ring rk{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
+    Waiter wait{c, true};
+    uint32_t s_issued[2] = {0u, 0u};
+    int local = 0;
+    for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
+        const Unit w = decode_unit<CAUSAL>(u, c.p);
+        if (!wait(c.bar + Bars::kQFull + 0, local & 1) || !wait(c.bar + Bars::kQFull + 8, local & 1)) break;
+        for (int j = 0; j < w.n1; ++j) {
+            uint32_t ks;
+            if (!wait.take(rk, ks)) break;
+            for (int t = 0; t < 2; ++t) {
+                if (t == 0 && j >= w.n0) continue;
+                if (s_issued[t] > 0 && !wait(c.bar + Bars::kSFree + 8 * t, (s_issued[t] - 1) & 1)) break;
+                tc_fence_after();
+                Mma<D>::qk(c, t, rk.smem + ks * C::kTileBytes);
+                tc_commit(c.bar + Bars::kSFull + 8 * t);
+                ++s_issued[t];
+            }
+            if (!wait.ok) break;
+            if (j + 1 == w.n1) tc_commit(c.bar + Bars::kQEmpty);
+            tc_commit(rk.empty + 8 * ks);
+        }
+    }
+    if (!wait.ok) mma_drain(c, 0);
+}
+
+// Split layout, P V stream: O_t += P_t(j) V_j once the softmax has written P_t(j).
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void role_mma_pv(const Ctx& c) {
+    using C = Cfg<D>;
+    Ring rv{c.base + C::kVRingOff, c.bar + Bars::kVFull, c.bar + Bars::kVEmpty, (uint32_t)C::kVSlots, 0};
+    Waiter wait{c, true};
+    uint32_t p_phase[2] = {0u, 0u};
+    int local = 0;
+    for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
+        const Unit w = decode_unit<CAUSAL>(u, c.p);
+        for (int j = 0; j < w.n1; ++j) {
+            uint32_t vs;
+            if (!wait.take(rv, vs)) break;
+            for (int t = 0; t < 2; ++t) {
+                const int n = t == 0 ? w.n0 : w.n1;
+                if (j >= n) continue;
+                if (!wait(c.bar + Bars::kPFull + 8 * t, p_phase[t])) break;
+                p_phase[t] ^= 1u;
+                if (j == 0 && !wait(c.bar + Bars::kOEmpty + 8 * t, (local & 1) ^ 1)) break;
+                tc_fence_after();
+                Mma<D>::pv(c, t, rv.smem + vs * C::kTileBytes, j > 0);
+                tc_commit(c.bar + Bars::kPFree + 8 * t);
+                if (j + 1 == n) tc_commit(c.bar + Bars::kOFull + 8 * t);
+            }
+            if (!wait.ok) break;
+            tc_commit(rv.empty + 8 * vs);
+        }
+    }
+    if (!wait.ok) mma_drain(c, 1);
+}
+
+// Shared layout (P over S): one ordered stream per key tile j:
+// P_0 V_j, S_0(j+1), P_1 V_j, S_1(j+1) -- S_t(j+1) overwrites P_t(j) after
+// the product that reads it, by issue order.
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void role_mma_ordered(const Ctx& c) {
+    using C = Cfg<D>;
+    Ring r{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
+    Waiter wait{c, true};
+    uint32_t p_phase[2] = {0u, 0u};
+    int local = 0;
+    auto smem = [&](uint32_t slot) { return r.smem + slot * C::kTileBytes; };
+    for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
+        const Unit w = decode_unit<CAUSAL>(u, c.p);
+        if (!wait(c.bar + Bars::kQFull + 0, local & 1) || !wait(c.bar + Bars::kQFull + 8, local & 1)) break;
+        uint32_t ks;
+        if (!wait.take(r, ks)) break;
+        tc_fence_after();
+        Mma<D>::qk(c, 0, smem(ks));
+        tc_commit(c.bar + Bars::kSFull + 0);
+        Mma<D>::qk(c, 1, smem(ks));
+        tc_commit(c.bar + Bars::kSFull + 8);
+        if (w.n1 == 1) tc_commit(c.bar + Bars::kQEmpty);
+        tc_commit(r.empty + 8 * ks);
+        for (int j = 0; j < w.n1; ++j) {
+            uint32_t vs, ks2 = 0;
+            const bool has_next = j + 1 < w.n1;
+            if (!wait.take(r, vs)) break;
+            if (has_next && !wait.take(r, ks2)) break;
+            if (j < w.n0) {
+                if (!wait(c.bar + Bars::kPFull + 0, p_phase[0])) break;
+                p_phase[0] ^= 1u;
+                if (j == 0 && !wait(c.bar + Bars::kOEmpty + 0, (local & 1) ^ 1)) break;
+                tc_fence_after();
+                Mma<D>::pv(c, 0, smem(vs), j > 0);
+                if (j + 1 < w.n0) {
+                    Mma<D>::qk(c, 0, smem(ks2));
+                    tc_commit(c.bar + Bars::kSFull + 0);
+                } else {
+                    tc_commit(c.bar + Bars::kOFull + 0);
+                }
+            }
+            if (!wait(c.bar + Bars::kPFull + 8, p_phase[1])) break;
+            p_phase[1] ^= 1u;
+            if (j == 0 && !wait(c.bar + Bars::kOEmpty + 8, (local & 1) ^ 1)) break;
+            tc_fence_after();
+            Mma<D>::pv(c, 1, smem(vs), j > 0);
+            tc_commit(r.empty + 8 * vs);
+            if (has_next) {
+                Mma<D>::qk(c, 1, smem(ks2));
+                tc_commit(c.bar + Bars::kSFull + 8);
+                if (j + 2 == w.n1) tc_commit(c.bar + Bars::kQEmpty);
+                tc_commit(r.empty + 8 * ks2);
+            } else {
+                tc_commit(c.bar + Bars::kOFull + 8);
+            }
+        }
+    }
+    if (!wait.ok) mma_drain(c, 0);
+}
+
+// ------------------------------------------------------- softmax + epilogue
+// Warpgroup t owns Q tile t; thread = one query row = one TMEM lane.
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, uint16_t* __restrict__ out_o,
+                                             float* __restrict__ out_lse) {
+    using C = Cfg<D>;
+    const Params& p = c.p;
+    const int t = warp >> 2;                  // Q tile of this warpgroup
+    const int quarter = warp & 3;             // TMEM lane quarter of this warp
+    const int r_in_tile = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_s = c.tmem + lane_off + (t == 0 ? C::kColS0 : C::kColS1);
+    const uint32_t t_o = c.tmem + lane_off + (t == 0 ? C::kColO0 : C::kColO1);
+    const uint32_t t_p = c.tmem + lane_off + (t == 0 ? C::kColP0 : C::kColP1);
+    const uint32_t b_s = c.bar + Bars::kSFull + 8 * t;
+    const uint32_t b_p = c.bar + Bars::kPFull + 8 * t;
+    const uint32_t b_of = c.bar + Bars::kOFull + 8 * t;
+    const uint32_t b_oe = c.bar + Bars::kOEmpty + 8 * t;
+    const uint32_t b_sfree = c.bar + Bars::kSFree + 8 * t;
+    const uint32_t b_pfree = c.bar + Bars::kPFree + 8 * t;
+    const float sl2 = p.scale_log2;
+    uint32_t s_phase = 0;
+    uint32_t pv_count = 0;  // P_t V products issued before the current step (split layout)
+    bool ok = true;
+    int local = 0;
+
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++local) {
+        const Unit w = decode_unit<CAUSAL>(u, p);
+        const int row = w.q0 + t * kBlockM + r_in_tile;
+        const int n_kv = (t == 0) ? w.n0 : w.n1;
+        // last visible key of this row (the row itself when causal)
+        const int last_key = CAUSAL ? min(row, p.N - 1) : p.N - 1;
+        float m = -INFINITY;  // reference max of scale*log2(e)*s (log2 units), shared by O and l
+        float l = 0.f;        // sum of exp2(scale*log2(e)*s - m) over the keys seen so far
+
+        for (int j = 0; j < n_kv; ++j) {
+            bool got = wait_bounded(b_s, s_phase, c.abort_flag, p.wait_ns);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) {
+                ok = false;
+                break;
+            }
+            s_phase ^= 1u;
+            tc_fence_after();
+
+            float s[kBlockN];
+            {
+                uint32_t r[4][32];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(t_s + c4 * 32, r[c4]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    reg_fence32(r[c4]);
+#pragma unroll
+                    for (int cc = 0; cc < 32; ++cc) s[c4 * 32 + cc] = __uint_as_float(r[c4][cc]);
+                }
+            }
+            if (C::kSplit) {
+                // S_t is in registers: the S stream may refill it with the next key tile
+                tc_fence_before();
+                mbar_arrive(b_sfree);
+            }
+            // key-tail and causal mask: keys past last_key get -inf
+            const int lim = last_key - j * kBlockN;
+            if (lim < kBlockN - 1) {
+#pragma unroll
+                for (int cc = 0; cc < kBlockN; ++cc)
+                    if (cc > lim) s[cc] = -INFINITY;
+            }
+            // row maximum (scale > 0, so it is taken on the raw scores)
+            float mx[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+            for (int cc = 4; cc < kBlockN; cc += 8) {
+                mx[0] = fmax3(mx[0], s[cc], s[cc + 1]);
+                mx[1] = fmax3(mx[1], s[cc + 2], s[cc + 3]);
+                if (cc + 4 < kBlockN) {
+                    mx[2] = fmax3(mx[2], s[cc + 4], s[cc + 5]);
+                    mx[3] = fmax3(mx[3], s[cc + 6], s[cc + 7]);
+                }
+            }
+            const float row_max = fmax3(fmax3(mx[0], mx[1], mx[2]), mx[3], -INFINITY) * sl2;
+            // lazy rescaling: move the reference only when the row maximum
+            // exceeds it by more than 2^8 (always on the first tile)
+            const bool move = row_max > m + kLazyRescaleLog2;
+            float alpha = 1.f;
+            if (move) {
+                alpha = ex2(m - row_max);  // 0 when m was -inf
+                m = row_max;
+            }
+            l *= alpha;
+            const float m_use = (m == -INFINITY) ? 0.f : m;
+            const float2 sl2x2 = make_float2(sl2, sl2);
+            const float2 negm = make_float2(-m_use, -m_use);
+
+            // P = exp2(scale*log2(e)*s - m) as bf16 pairs; kPolyPairsPer8 of
+            // every 8 pairs use the FMA-pipe exponential, the rest MUFU.
+            float2 acc = make_float2(0.f, 0.f);
+            uint32_t pk[kBlockN / 2];
+#pragma unroll
+            for (int cc = 0; cc < kBlockN / 2; ++cc) {
+                float2 x = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), sl2x2, negm);
+                if ((cc & 7) >= 8 - kPolyPairsPer8) {
+                    x = ex2_poly2(x);
+                } else {
+                    x.x = ex2(x.x);
+                    x.y = ex2(x.y);
+                }
+                acc = __fadd2_rn(acc, x);
+                pk[cc] = pack_bf16x2(x.x, x.y);
+            }
+            l += acc.x + acc.y;
+            const bool rescale = move && j > 0;
+            if (C::kSplit) {
+                // P_t and O_t belong to the previous P V until it retires
+                if (pv_count > 0) {
+                    bool done = wait_bounded(b_pfree, (pv_count - 1) & 1, c.abort_flag, p.wait_ns);
+                    done = __all_sync(0xffffffffu, done);
+                    if (!done) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                ++pv_count;
+            }
+            tmem_st32(t_p, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_st32(t_p + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+            // O holds the sum over earlier tiles at the old reference: bring it
+            // to the new one before the next P V accumulates into it (the
+            // previous P V has retired: waited for above in the split layout,
+            // implied by S_t in the shared one)
+            if (__any_sync(0xffffffffu, rescale)) {
+                const float a = rescale ? alpha : 1.f;
+#pragma unroll
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    uint32_t r[32];
+                    tmem_ld32(t_o + c4 * 32, r);
+                    tmem_wait_ld();
+                    reg_fence32(r);
+#pragma unroll
+                    for (int cc = 0; cc < 32; ++cc) r[cc] = __float_as_uint(__uint_as_float(r[cc]) * a);
+                    tmem_st32(t_o + c4 * 32, r);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(b_p);
+        }
+        if (!ok) break;
+
+        // ---------------------------------------------------------- epilogue
+        bool got = wait_bounded(b_of, local & 1, c.abort_flag, p.wait_ns);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const bool store = row < p.N;
+        uint16_t* orow = out_o + (static_cast<size_t>(w.bh) * p.N + (store ? row : 0)) * D;
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t r[32];
+            tmem_ld32(t_o + c4 * 32, r);
+            tmem_wait_ld();
+            reg_fence32(r);
+            if (c4 == D / 32 - 1) {
+                tc_fence_before();
+                mbar_arrive(b_oe);  // O_t may now be overwritten by the next unit
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc)
+                pk[cc] = pack_bf16x2(__uint_as_float(r[2 * cc]) * inv_l, __uint_as_float(r[2 * cc + 1]) * inv_l);
+            if (store) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                    dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            }
+        }
+        if (store) out_lse[static_cast<size_t>(w.bh) * p.N + row] = (m + __log2f(l)) * kLn2;
+    }
 }
 
 // ----------------------------------------------------------------- the kernel
@@ -376,19 +836,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar + Bars::kQFull + 0, 1);
-        mbar_init(bar + Bars::kQFull + 8, 1);
-        mbar_init(bar + Bars::kQEmpty, 1);
         for (int t = 0; t < 2; ++t) {
+            mbar_init(bar + Bars::kQFull + 8 * t, 1);
             mbar_init(bar + Bars::kSFull + 8 * t, 1);
             mbar_init(bar + Bars::kPFull + 8 * t, kBlockM);
             mbar_init(bar + Bars::kOFull + 8 * t, 1);
             mbar_init(bar + Bars::kOEmpty + 8 * t, kBlockM);
+            mbar_init(bar + Bars::kDrain + 8 * t, 1);
+            mbar_init(bar + Bars::kSFree + 8 * t, kBlockM);
+            mbar_init(bar + Bars::kPFree + 8 * t, 1);
         }
-        mbar_init(bar + Bars::kDrain, 1);
-        for (int s = 0; s < C::kSlots; ++s) {
-            mbar_init(bar + Bars::kKvFull + 8 * s, 1);
-            mbar_init(bar + Bars::kKvEmpty + 8 * s, 1);
+        mbar_init(bar + Bars::kQEmpty, 1);
+        for (int s = 0; s < 8; ++s) {
+            mbar_init(bar + Bars::kKFull + 8 * s, 1);
+            mbar_init(bar + Bars::kKEmpty + 8 * s, 1);
+            mbar_init(bar + Bars::kVFull + 8 * s, 1);
+            mbar_init(bar + Bars::kVEmpty + 8 * s, 1);
         }
         *abort_flag = 0u;
         fence_barrier_init();
@@ -406,328 +869,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const Ctx ctx{base, bar, *tmem_slot, abort_flag, p};
 
     if (warp >= kLoadWarp) {
-      regs_decrease<kOtherRegs>();
-      if (warp == kLoadWarp) {
-        // ------------------------------------------------------------ producer
+        regs_decrease<kOtherRegs>();
         if (lane == 0) {
-            uint32_t kv_i = 0;
-            uint32_t q_issued = 0;
-            bool ok = true;
-            int local = 0;
-            for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++local) {
-                const Unit w = decode_unit<CAUSAL>(u, p);
-                if (!wait_bounded(bar + Bars::kQEmpty, (local & 1) ^ 1, abort_flag, p.wait_ns)) {
-                    ok = false;
-                    break;
-                }
-                for (int t = 0; t < 2; ++t) {
-                    const uint32_t qb = bar + Bars::kQFull + 8 * t;
-                    const uint32_t dst = base + C::kQOff + t * C::kTileBytes;
-                    mbar_expect_tx(qb, C::kTileBytes);
-                    for (int h = 0; h < D / 64; ++h)
-                        tma_load_3d(dst + h * C::kHalfBytes, &tm_q, qb, h * 64, w.q0 + t * kBlockM, w.bh);
-                }
-                q_issued = local + 1;
-                for (int j = 0; ok && j < w.n1; ++j) {
-                    for (int kv = 0; kv < 2; ++kv) {
-                        const uint32_t slot = kv_i % C::kSlots;
-                        const uint32_t round = kv_i / C::kSlots;
-                        if (!wait_bounded(bar + Bars::kKvEmpty + 8 * slot, (round & 1) ^ 1, abort_flag,
-                                          p.wait_ns)) {
-                            ok = false;
-                            break;
-                        }
-                        const uint32_t fb = bar + Bars::kKvFull + 8 * slot;
-                        const uint32_t dst = base + C::kRingOff + slot * C::kTileBytes;
-                        mbar_expect_tx(fb, C::kTileBytes);
-                        for (int h = 0; h < D / 64; ++h)
-                            tma_load_3d(dst + h * C::kHalfBytes, kv == 0 ? &tm_k : &tm_v, fb, h * 64,
-                                        j * kBlockN, w.bh);
-                        ++kv_i;
-                    }
-                }
-            }
-            if (!ok) {
-                // Drain: every issued copy lands before the CTA may exit.
-                const unsigned long long drain_ns = 100000000ull;
-                for (uint32_t i = (kv_i > (uint32_t)C::kSlots ? kv_i - C::kSlots : 0); i < kv_i; ++i)
-                    wait_bounded(bar + Bars::kKvFull + 8 * (i % C::kSlots), (i / C::kSlots) & 1, nullptr,
-                                 drain_ns);
-                if (q_issued > 0)
-                    for (int t = 0; t < 2; ++t)
-                        wait_bounded(bar + Bars::kQFull + 8 * t, (q_issued - 1) & 1, nullptr, drain_ns);
+            if (warp == kLoadWarp) {
+                role_producer<D, CAUSAL>(ctx, &tm_q, &tm_k, &tm_v);
+            } else if (warp == kMmaWarp) {
+                if (C::kSplit) role_mma_s<D, CAUSAL>(ctx);
+                else role_mma_ordered<D, CAUSAL>(ctx);
+            } else if (warp == kMmaPvWarp && C::kSplit) {
+                role_mma_pv<D, CAUSAL>(ctx);
             }
         }
         __syncwarp();
-      } else if (warp == kMmaWarp) {
-        // ----------------------------------------------------------- MMA issue
-        if (lane == 0) {
-            constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN, false);
-            constexpr uint32_t kIdescO = idesc_bf16_f32(kBlockM, D, true);
-            const uint32_t q_smem[2] = {base + C::kQOff, base + C::kQOff + C::kTileBytes};
-            const uint32_t s_col[2] = {C::kColS0, C::kColS1};
-            const uint32_t o_col[2] = {C::kColO0, C::kColO1};
-            uint32_t kv_i = 0;
-            uint32_t p_phase[2] = {0u, 0u};
-            bool ok = true;
-            int local = 0;
-
-            auto wait = [&](uint32_t b, uint32_t parity) {
-                if (ok && !wait_bounded(b, parity, abort_flag, p.wait_ns)) ok = false;
-                return ok;
-            };
-            // S_t = Q_t K^T  (K-major A and B, 16 columns of d per instruction)
-            auto issue_qk = [&](int t, uint32_t k_smem) {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk / 4) * C::kHalfBytes + (kk % 4) * 32;
-                    mma_ss(tmem + s_col[t], sdesc_sw128(q_smem[t] + off, 16, 1024),
-                           sdesc_sw128(k_smem + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-                }
-            };
-            // O_t (+)= P_t V  (P from TMEM, V MN-major: 16 keys per instruction)
-            auto issue_pv = [&](int t, uint32_t v_smem, bool accumulate) {
-#pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    mma_ts(tmem + o_col[t], tmem + s_col[t] + kk * 8,
-                           sdesc_sw128(v_smem + kk * 16 * 128, C::kHalfBytes, 1024), kIdescO,
-                           (accumulate || kk > 0) ? 1u : 0u);
-                }
-            };
-            auto ring_take = [&](uint32_t& slot) {
-                slot = kv_i % C::kSlots;
-                const bool r = wait(bar + Bars::kKvFull + 8 * slot, (kv_i / C::kSlots) & 1);
-                ++kv_i;
-                return r;
-            };
-            auto ring_smem = [&](uint32_t slot) { return base + C::kRingOff + slot * C::kTileBytes; };
-
-            for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++local) {
-                const Unit w = decode_unit<CAUSAL>(u, p);
-                if (!wait(bar + Bars::kQFull + 0, local & 1) || !wait(bar + Bars::kQFull + 8, local & 1))
-                    break;
-                uint32_t ks;
-                if (!ring_take(ks)) break;
-                tc_fence_after();
-                issue_qk(0, ring_smem(ks));
-                tc_commit(bar + Bars::kSFull + 0);
-                issue_qk(1, ring_smem(ks));
-                tc_commit(bar + Bars::kSFull + 8);
-                if (w.n1 == 1) tc_commit(bar + Bars::kQEmpty);
-                tc_commit(bar + Bars::kKvEmpty + 8 * ks);
-
-                for (int j = 0; j < w.n1; ++j) {
-                    uint32_t vs, ks2 = 0;
-                    const bool has_next = j + 1 < w.n1;
-                    if (!ring_take(vs)) break;
-                    if (has_next && !ring_take(ks2)) break;
-                    if (j < w.n0) {
-                        if (!wait(bar + Bars::kPFull + 0, p_phase[0])) break;
-                        p_phase[0] ^= 1u;
-                        if (j == 0 && !wait(bar + Bars::kOEmpty + 0, (local & 1) ^ 1)) break;
-                        tc_fence_after();
-                        issue_pv(0, ring_smem(vs), j > 0);
-                        if (j + 1 < w.n0) {
-                            issue_qk(0, ring_smem(ks2));
-                            tc_commit(bar + Bars::kSFull + 0);
-                        } else {
-                            tc_commit(bar + Bars::kOFull + 0);
-                        }
-                    }
-                    if (!wait(bar + Bars::kPFull + 8, p_phase[1])) break;
-                    p_phase[1] ^= 1u;
-                    if (j == 0 && !wait(bar + Bars::kOEmpty + 8, (local & 1) ^ 1)) break;
-                    tc_fence_after();
-                    issue_pv(1, ring_smem(vs), j > 0);
-                    tc_commit(bar + Bars::kKvEmpty + 8 * vs);
-                    if (has_next) {
-                        issue_qk(1, ring_smem(ks2));
-                        tc_commit(bar + Bars::kSFull + 8);
-                        if (j + 2 == w.n1) tc_commit(bar + Bars::kQEmpty);
-                        tc_commit(bar + Bars::kKvEmpty + 8 * ks2);
-                    } else {
-                        tc_commit(bar + Bars::kOFull + 8);
-                    }
-                }
-            }
-            if (!ok) {
-                // Drain: all issued MMAs retire before TMEM is released.
-                tc_commit(bar + Bars::kDrain);
-                wait_bounded(bar + Bars::kDrain, 0, nullptr, 100000000ull);
-            }
-        }
-        __syncwarp();
-      }
     } else {
         regs_increase<kSoftmaxRegs>();
-        // -------------------------------------------------- softmax warpgroups
-        const int t = warp >> 2;                  // Q tile of this warpgroup
-        const int quarter = warp & 3;             // TMEM lane quarter of this warp
-        const int r_in_tile = quarter * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t t_s = tmem + lane_off + (t == 0 ? C::kColS0 : C::kColS1);
-        const uint32_t t_o = tmem + lane_off + (t == 0 ? C::kColO0 : C::kColO1);
-        const uint32_t b_s = bar + Bars::kSFull + 8 * t;
-        const uint32_t b_p = bar + Bars::kPFull + 8 * t;
-        const uint32_t b_of = bar + Bars::kOFull + 8 * t;
-        const uint32_t b_oe = bar + Bars::kOEmpty + 8 * t;
-        const float sl2 = p.scale_log2;
-        uint32_t s_phase = 0;
-        bool ok = true;
-        int local = 0;
-
-        for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++local) {
-            const Unit w = decode_unit<CAUSAL>(u, p);
-            const int row = w.q0 + t * kBlockM + r_in_tile;
-            const int n_kv = (t == 0) ? w.n0 : w.n1;
-            // last visible key of this row (the row itself when causal)
-            const int last_key = CAUSAL ? min(row, p.N - 1) : p.N - 1;
-            float m = -INFINITY;  // reference max of scale*log2(e)*s (log2 units), shared by O and l
-            float l = 0.f;        // sum of exp2(scale*log2(e)*s - m) over the keys seen so far
-
-            for (int j = 0; j < n_kv; ++j) {
-                bool got = wait_bounded(b_s, s_phase, abort_flag, p.wait_ns);
-                got = __all_sync(0xffffffffu, got);
-                if (!got) {
-                    ok = false;
-                    break;
-                }
-                s_phase ^= 1u;
-                tc_fence_after();
-
-                float s[kBlockN];
-                {
-                    uint32_t r[4][32];
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(t_s + c4 * 32, r[c4]);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        reg_fence32(r[c4]);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) s[c4 * 32 + c] = __uint_as_float(r[c4][c]);
-                    }
-                }
-                // key-tail and causal mask: keys past last_key get -inf
-                const int lim = last_key - j * kBlockN;
-                if (lim < kBlockN - 1) {
-#pragma unroll
-                    for (int c = 0; c < kBlockN; ++c)
-                        if (c > lim) s[c] = -INFINITY;
-                }
-                // row maximum (scale > 0, so it is taken on the raw scores)
-                float mx[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-                for (int c = 4; c < kBlockN; c += 8) {
-                    mx[0] = fmax3(mx[0], s[c], s[c + 1]);
-                    mx[1] = fmax3(mx[1], s[c + 2], s[c + 3]);
-                    if (c + 4 < kBlockN) {
-                        mx[2] = fmax3(mx[2], s[c + 4], s[c + 5]);
-                        mx[3] = fmax3(mx[3], s[c + 6], s[c + 7]);
-                    }
-                }
-                const float row_max = fmax3(fmax3(mx[0], mx[1], mx[2]), mx[3], -INFINITY) * sl2;
-                // lazy rescaling: move the reference only when the row maximum
-                // exceeds it by more than 2^8 (always on the first tile)
-                const bool move = row_max > m + kLazyRescaleLog2;
-                float alpha = 1.f;
-                if (move) {
-                    alpha = ex2(m - row_max);  // 0 when m was -inf
-                    m = row_max;
-                }
-                l *= alpha;
-                const float m_use = (m == -INFINITY) ? 0.f : m;
-                const float2 sl2x2 = make_float2(sl2, sl2);
-                const float2 negm = make_float2(-m_use, -m_use);
-
-                // P = exp2(scale*log2(e)*s - m) as bf16 pairs over the S columns;
-                // 3 of every 8 pairs use the FMA-pipe exponential, the rest MUFU.
-                float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int e = c2 * 64 + 2 * c;
-                        float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sl2x2, negm);
-                        if ((c & 7) >= 5) {
-                            x = ex2_poly2(x);
-                        } else {
-                            x.x = ex2(x.x);
-                            x.y = ex2(x.y);
-                        }
-                        acc = __fadd2_rn(acc, x);
-                        pk[c] = pack_bf16x2(x.x, x.y);
-                    }
-                    tmem_st32(t_s + c2 * 32, pk);
-                }
-                l += acc.x + acc.y;
-                // O holds the sum over earlier tiles at the old reference:
-                // bring it to the new one before the next P V accumulates.
-                const bool rescale = move && j > 0;
-                if (__any_sync(0xffffffffu, rescale)) {
-                    const float a = rescale ? alpha : 1.f;
-#pragma unroll
-                    for (int c4 = 0; c4 < D / 32; ++c4) {
-                        uint32_t r[32];
-                        tmem_ld32(t_o + c4 * 32, r);
-                        tmem_wait_ld();
-                        reg_fence32(r);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * a);
-                        tmem_st32(t_o + c4 * 32, r);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(b_p);
-            }
-            if (!ok) break;
-
-            // ------------------------------------------------------ epilogue
-            bool got = wait_bounded(b_of, local & 1, abort_flag, p.wait_ns);
-            got = __all_sync(0xffffffffu, got);
-            if (!got) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const float inv_l = 1.f / l;
-            const bool store = row < p.N;
-            uint16_t* orow = out_o + (static_cast<size_t>(w.bh) * p.N + (store ? row : 0)) * D;
-#pragma unroll
-            for (int c4 = 0; c4 < D / 32; ++c4) {
-                uint32_t r[32];
-                tmem_ld32(t_o + c4 * 32, r);
-                tmem_wait_ld();
-                reg_fence32(r);
-                if (c4 == D / 32 - 1) {
-                    tc_fence_before();
-                    mbar_arrive(b_oe);  // O_t may now be overwritten by the next unit
-                }
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    pk[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
-                if (store) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-                }
-            }
-            if (store) out_lse[static_cast<size_t>(w.bh) * p.N + row] = (m + __log2f(l)) * kLn2;
-        }
+        role_softmax<D, CAUSAL>(ctx, warp, lane, out_o, out_lse);
     }
 
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(ctx.tmem, kTmemCols);
     }
 }
 
