@@ -64,9 +64,16 @@ constexpr float kLazyRescaleLog2 = 8.0f;
 // Of every 8 exponential pairs, this many run on the FMA-pipe polynomial and
 // the rest on MUFU (ex2.approx).
 #ifndef ATTN_POLY_PAIRS_PER_8
-#define ATTN_POLY_PAIRS_PER_8 2
+#define ATTN_POLY_PAIRS_PER_8 3
 #endif
 constexpr int kPolyPairsPer8 = ATTN_POLY_PAIRS_PER_8;
+// Which pairs of each group of 8 take the polynomial (best measured patterns).
+constexpr uint32_t kPolyMask8 = kPolyPairsPer8 <= 0 ? 0x00u
+                              : kPolyPairsPer8 == 1 ? 0x80u
+                              : kPolyPairsPer8 == 2 ? 0xC0u
+                              : kPolyPairsPer8 == 3 ? 0x70u
+                              : kPolyPairsPer8 == 4 ? 0xAAu
+                              : 0xFFu;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -148,6 +155,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// The same test, but a thread whose phase is not complete is suspended (it
+// resumes as soon as the phase completes, or after at most hint_ns) instead
+// of spinning on the issue slots of its sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+constexpr uint32_t kWaitSleepNs = 20000;
 
 // Wait until the phase with parity `parity` of barrier `bar` has completed.
 // Gives up after `limit_ns` (then raises the CTA abort flag and the device
@@ -157,8 +179,8 @@ __device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatil
                                        unsigned long long limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     uint32_t n = 0;
-    while (!mbar_try_wait(bar, parity)) {
-        if ((++n & 31u) == 0) {
+    while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
+        if ((++n & 3u) == 0) {
             if (abort_flag != nullptr && *abort_flag) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 if (abort_flag != nullptr) *abort_flag = 1u;
@@ -326,9 +348,11 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
     float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
     q = __ffma2_rn(q, f, make_float2(kC1, kC1));
     q = __ffma2_rn(q, f, make_float2(kC0, kC0));
-    // the low mantissa bits of t hold j (two's complement); shifting by 23 moves them to the exponent
-    const uint32_t rx = __float_as_uint(q.x) + (__float_as_uint(t.x) << 23);
-    const uint32_t ry = __float_as_uint(q.y) + (__float_as_uint(t.y) << 23);
+    // the low mantissa bits of t hold j (two's complement); t * 2^23 moves them
+    // to the exponent field, added to q in one integer multiply-add
+    uint32_t rx, ry;
+    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rx) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(q.x)));
+    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(ry) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(q.y)));
     return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
@@ -725,23 +749,23 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
             const float2 sl2x2 = make_float2(sl2, sl2);
             const float2 negm = make_float2(-m_use, -m_use);
 
-            // P = exp2(scale*log2(e)*s - m) as bf16 pairs; kPolyPairsPer8 of
-            // every 8 pairs use the FMA-pipe exponential, the rest MUFU.
-            float2 acc = make_float2(0.f, 0.f);
+            // P = exp2(scale*log2(e)*s - m) as bf16 pairs; the pairs marked in
+            // kPolyMask8 use the FMA-pipe exponential, the rest MUFU.
+            float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
             uint32_t pk[kBlockN / 2];
 #pragma unroll
             for (int cc = 0; cc < kBlockN / 2; ++cc) {
                 float2 x = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), sl2x2, negm);
-                if ((cc & 7) >= 8 - kPolyPairsPer8) {
+                if ((kPolyMask8 >> (cc & 7)) & 1u) {
                     x = ex2_poly2(x);
                 } else {
                     x.x = ex2(x.x);
                     x.y = ex2(x.y);
                 }
-                acc = __fadd2_rn(acc, x);
+                acc[cc & 1] = __fadd2_rn(acc[cc & 1], x);
                 pk[cc] = pack_bf16x2(x.x, x.y);
             }
-            l += acc.x + acc.y;
+            l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
             const bool rescale = move && j > 0;
             if (C::kSplit) {
                 // P_t and O_t belong to the previous P V until it retires
