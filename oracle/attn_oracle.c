@@ -20,10 +20,17 @@
  * the "standard attention" the notes contrast with the tiled method, section
  * "IO complexity analysis"); nothing is blocked, fused or reordered.
  *
+ * Key padding (flash-attnの代役がVRAMを18GB溶かしていたので87%削った話, §3 and
+ * §6): key_pad is NULL or a [B, N] byte mask in which a nonzero byte marks a
+ * padded key, excluded from every row of that batch (the key_padding_mask
+ * convention: nonzero = ignore, the opposite of a boolean "attend" mask).
+ *
  * Readings where the pages are silent:
  *   - scale is an explicit argument (the notes' formula omits it);
  *   - LSE is the natural log of sum_j exp(s_j), in scaled-logit units;
  *   - causal is the square top-left mask: key j is visible to query i iff j <= i;
+ *   - a row with no visible key (every key it may see is padded) has O = 0 and
+ *     LSE = -inf;
  *   - bf16 inputs are widened exactly to fp64 before any arithmetic.
  *
  * Parity status: pinned by the CPU tests (closed forms, invariants, a
@@ -45,23 +52,33 @@ static double widen_bf16(uint16_t bits) {
     return (double)f;
 }
 
-/* One query row against one head's keys and values; s and p are scratch rows of length N. */
+/* One query row against one head's keys and values; s and p are scratch rows
+ * of length N.  Keys 0..visible-1 are candidates; pad (NULL or [N]) removes
+ * the padded ones.  Excluded keys get no score and probability 0. */
 static void one_row(const double* qi, const double* kh, const double* vh, int N, int d,
-                    double scale, int visible, double* s, double* p, double* oi, double* lse) {
+                    double scale, int visible, const unsigned char* pad, double* s, double* p,
+                    double* oi, double* lse) {
     double m = -INFINITY;
+    int any = 0;
     for (int j = 0; j < visible; ++j) {
+        if (pad && pad[j]) continue;
         double acc = 0.0;
         for (int t = 0; t < d; ++t) acc += qi[t] * kh[(size_t)j * d + t];
         s[j] = scale * acc;
-        if (s[j] > m) m = s[j];
+        if (!any || s[j] > m) m = s[j];
+        any = 1;
+    }
+    for (int t = 0; t < d; ++t) oi[t] = 0.0;
+    if (!any) {
+        *lse = -INFINITY;
+        return;
     }
     double sum = 0.0;
     for (int j = 0; j < visible; ++j) {
-        p[j] = exp(s[j] - m);
+        p[j] = (pad && pad[j]) ? 0.0 : exp(s[j] - m);
         sum += p[j];
     }
     for (int j = 0; j < visible; ++j) p[j] /= sum;
-    for (int t = 0; t < d; ++t) oi[t] = 0.0;
     for (int j = 0; j < visible; ++j) {
         const double* vj = vh + (size_t)j * d;
         for (int t = 0; t < d; ++t) oi[t] += p[j] * vj[t];
@@ -72,8 +89,8 @@ static void one_row(const double* qi, const double* kh, const double* vh, int N,
 
 /* All selected rows of one head.  rows == NULL means every row 0..N-1. */
 static void one_head(const double* qh, const double* kh, const double* vh, int N, int d,
-                     double scale, int causal, const int32_t* rows, int n_rows,
-                     double* o, double* lse, int n_threads) {
+                     double scale, int causal, const unsigned char* pad, const int32_t* rows,
+                     int n_rows, double* o, double* lse, int n_threads) {
 #ifdef _OPENMP
 #pragma omp parallel num_threads(n_threads > 0 ? n_threads : omp_get_max_threads())
 #endif
@@ -86,7 +103,7 @@ static void one_head(const double* qh, const double* kh, const double* vh, int N
         for (int r = 0; r < n_rows; ++r) {
             int i = rows ? rows[r] : r;
             int visible = causal ? i + 1 : N;
-            one_row(qh + (size_t)i * d, kh, vh, N, d, scale, visible, s, p,
+            one_row(qh + (size_t)i * d, kh, vh, N, d, scale, visible, pad, s, p,
                     o + (size_t)r * d, lse + r);
         }
         free(s);
@@ -108,17 +125,19 @@ static int args_ok(int B, int H, int N, int d, const int32_t* rows, int n_rows) 
 
 /*
  * fp64 inputs, layout [B, H, N, d] contiguous.
+ * key_pad: NULL or [B, N] bytes, nonzero = padded key.
  * rows: NULL (all rows, n_rows must equal N) or int32 [B*H, n_rows], the
  * query rows to evaluate for each head.  o: fp64 [B*H, n_rows, d];
  * lse: fp64 [B*H, n_rows].  Returns 0 on success, -1 on bad arguments.
  */
 int attn_oracle_f64(const double* q, const double* k, const double* v, int B, int H, int N,
-                    int d, double scale, int causal, const int32_t* rows, int n_rows,
-                    double* o, double* lse, int n_threads) {
+                    int d, double scale, int causal, const unsigned char* key_pad,
+                    const int32_t* rows, int n_rows, double* o, double* lse, int n_threads) {
     if (!args_ok(B, H, N, d, rows, n_rows)) return -1;
     size_t head = (size_t)N * d;
     for (long bh = 0; bh < (long)B * H; ++bh) {
-        one_head(q + bh * head, k + bh * head, v + bh * head, N, d, scale, causal,
+        const unsigned char* pad = key_pad ? key_pad + (size_t)(bh / H) * N : NULL;
+        one_head(q + bh * head, k + bh * head, v + bh * head, N, d, scale, causal, pad,
                  rows ? rows + bh * n_rows : NULL, n_rows, o + (size_t)bh * n_rows * d,
                  lse + (size_t)bh * n_rows, n_threads);
     }
@@ -131,8 +150,8 @@ int attn_oracle_f64(const double* q, const double* k, const double* v, int B, in
  * arguments and outputs as attn_oracle_f64.
  */
 int attn_oracle_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
-                     int N, int d, double scale, int causal, const int32_t* rows, int n_rows,
-                     double* o, double* lse, int n_threads) {
+                     int N, int d, double scale, int causal, const unsigned char* key_pad,
+                     const int32_t* rows, int n_rows, double* o, double* lse, int n_threads) {
     if (!args_ok(B, H, N, d, rows, n_rows)) return -1;
     size_t head = (size_t)N * d;
     double* qh = (double*)malloc(sizeof(double) * head);
@@ -148,7 +167,8 @@ int attn_oracle_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
             kh[e] = widen_bf16(k[bh * head + e]);
             vh[e] = widen_bf16(v[bh * head + e]);
         }
-        one_head(qh, kh, vh, N, d, scale, causal, rows ? rows + bh * n_rows : NULL, n_rows,
+        const unsigned char* pad = key_pad ? key_pad + (size_t)(bh / H) * N : NULL;
+        one_head(qh, kh, vh, N, d, scale, causal, pad, rows ? rows + bh * n_rows : NULL, n_rows,
                  o + (size_t)bh * n_rows * d, lse + (size_t)bh * n_rows, n_threads);
     }
     free(qh); free(kh); free(vh);

@@ -10,22 +10,30 @@ j <= i.
 import numpy as np
 
 
-def attention_full(q, k, v, scale, causal=False, return_probs=False):
-    """q, k, v: float64 arrays [B, H, N, d].  Returns (O [B,H,N,d], LSE [B,H,N]) and optionally P."""
+def attention_full(q, k, v, scale, causal=False, return_probs=False, key_pad=None):
+    """q, k, v: float64 arrays [B, H, N, d]; key_pad: None or [B, N], nonzero =
+    padded key.  Returns (O [B,H,N,d], LSE [B,H,N]) and optionally P; a row
+    with no visible key has O = 0, LSE = -inf and P = 0."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     n = q.shape[-2]
     s = scale * np.matmul(q, np.swapaxes(k, -1, -2))
+    visible = np.ones(s.shape, dtype=bool)
     if causal:
-        visible = np.tril(np.ones((n, n), dtype=bool))
-        s = np.where(visible, s, -np.inf)
+        visible &= np.tril(np.ones((n, n), dtype=bool))
+    if key_pad is not None:
+        visible &= ~np.asarray(key_pad, dtype=bool)[:, None, None, :]
+    s = np.where(visible, s, -np.inf)
     m = s.max(axis=-1, keepdims=True)
-    e = np.exp(s - m)
+    empty = ~visible.any(axis=-1, keepdims=True)
+    m_safe = np.where(empty, 0.0, m)
+    e = np.where(visible, np.exp(s - m_safe), 0.0)
     total = e.sum(axis=-1, keepdims=True)
-    p = e / total
+    p = e / np.where(empty, 1.0, total)
     o = np.matmul(p, v)
-    lse = m[..., 0] + np.log(total[..., 0])
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty[..., 0], -np.inf, m_safe[..., 0] + np.log(np.where(empty, 1.0, total)[..., 0]))
     if return_probs:
         return o, lse, p
     return o, lse

@@ -36,7 +36,7 @@ def _load():
             fn = getattr(lib, name)
             fn.restype = ctypes.c_int
             fn.argtypes = [ptr, ptr, ptr, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                           ctypes.c_double, ctypes.c_int, ptr, ctypes.c_int, ptr, ptr, ctypes.c_int]
+                           ctypes.c_double, ctypes.c_int, ptr, ptr, ctypes.c_int, ptr, ptr, ctypes.c_int]
         lib.attn_oracle_max_threads.restype = ctypes.c_int
         lib.attn_oracle_max_threads.argtypes = []
         _lib = lib
@@ -54,13 +54,14 @@ def _bf16_bits(t):
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def attention_rows(q, k, v, scale, causal=False, rows=None, n_threads=0):
+def attention_rows(q, k, v, scale, causal=False, rows=None, n_threads=0, key_pad=None):
     """Evaluate the oracle on selected query rows.
 
     q, k, v: [B, H, N, d], either bf16 torch tensors (widened exactly) or
     float64 arrays.  rows: None (all rows) or an int array [B*H, R] (or [R],
-    shared by every head) of query indices.  Returns (O [B*H, R, d],
-    LSE [B*H, R]) as float64 numpy arrays.
+    shared by every head) of query indices.  key_pad: None or a [B, N] array,
+    nonzero = padded key.  Returns (O [B*H, R, d], LSE [B*H, R]) as float64
+    numpy arrays; a row with no visible key has O = 0 and LSE = -inf.
     """
     lib = _load()
     try:
@@ -84,10 +85,14 @@ def attention_rows(q, k, v, scale, causal=False, rows=None, n_threads=0):
         rows_a = np.ascontiguousarray(rows_a.reshape(B * H, -1))
         n_rows = rows_a.shape[1]
         rows_p = rows_a.ctypes.data
+    pad_p = None
+    if key_pad is not None:
+        pad_a = np.ascontiguousarray(np.asarray(key_pad).astype(np.uint8).reshape(B, N))
+        pad_p = pad_a.ctypes.data
     o = np.empty((B * H, n_rows, d), dtype=np.float64)
     lse = np.empty((B * H, n_rows), dtype=np.float64)
     rc = fn(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, B, H, N, d, float(scale),
-            int(bool(causal)), rows_p, n_rows, o.ctypes.data, lse.ctypes.data, int(n_threads))
+            int(bool(causal)), pad_p, rows_p, n_rows, o.ctypes.data, lse.ctypes.data, int(n_threads))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (code %d)" % rc)
     return o, lse

@@ -236,3 +236,97 @@ def test_input_recipe_is_deterministic_and_bf16():
     assert torch.equal(q4.float(), a[0].float() * 4)
     # Q, K, V come from one stream in that order: K differs from Q
     assert not torch.equal(a[0], a[1])
+
+
+# ---------------------------------------------------------------- key padding
+GOLDEN_MASK = __import__("os").path.join(__import__("os").path.dirname(__file__), "golden", "mask_polarity.txt")
+
+
+def test_mask_polarity_worked_example_from_the_page():
+    B, H, N, d, padded, printed, digits = [l.split() for l in open(GOLDEN_MASK)
+                                           if l.strip() and not l.startswith("#")][0]
+    B, H, N, d, padded, digits = (int(x) for x in (B, H, N, d, padded, digits))
+    torch.manual_seed(0)
+    q = torch.randn(B, H, N, d).double().numpy()
+    pad = np.zeros((B, N), dtype=np.uint8)
+    pad[:, padded] = 1
+    scale = 1.0 / math.sqrt(d)
+    o_ref, _ = oracle.attention_rows(q, q, q, scale, key_pad=pad)               # the padded key excluded
+    o_flip, _ = oracle.attention_rows(q, q, q, scale, key_pad=1 - pad)          # polarity not inverted
+    o_twice, _ = oracle.attention_rows(q, q, q, scale, key_pad=1 - (1 - pad))  # inverted: same mask
+    assert round(float(np.abs(o_flip - o_ref).max()), digits) == float(printed)
+    assert np.abs(o_twice - o_ref).max() == 0.0
+    # passing the mask with the wrong polarity attends only the padded key
+    np.testing.assert_allclose(o_flip.reshape(B, H, N, d), np.broadcast_to(q[:, :, padded:padded + 1], (B, H, N, d)),
+                               atol=1e-15)
+
+
+def test_padded_keys_have_no_influence():
+    B, H, N, d = 2, 2, 12, 4
+    q = RNG.normal(size=(B, H, N, d))
+    k = RNG.normal(size=(B, H, N, d))
+    v = RNG.normal(size=(B, H, N, d))
+    pad = (RNG.random((B, N)) < 0.4).astype(np.uint8)
+    pad[:, 0] = 0
+    for causal in (False, True):
+        o, lse = oracle.attention_rows(q, k, v, 0.5, causal, key_pad=pad)
+        k2, v2 = k.copy(), v.copy()
+        bsel, nsel = np.nonzero(pad)
+        k2[bsel, :, nsel] += 9.0
+        v2[bsel, :, nsel] -= 7.0
+        o2, lse2 = oracle.attention_rows(q, k2, v2, 0.5, causal, key_pad=pad)
+        np.testing.assert_array_equal(o2, o)
+        np.testing.assert_array_equal(lse2, lse)
+
+
+def test_padding_equals_attention_over_the_kept_keys():
+    # an independent construction: drop the padded keys and values
+    B, H, N, d = 1, 3, 15, 6
+    q = RNG.normal(size=(B, H, N, d))
+    k = RNG.normal(size=(B, H, N, d))
+    v = RNG.normal(size=(B, H, N, d))
+    pad = np.zeros((B, N), dtype=np.uint8)
+    pad[0, [1, 4, 5, 11, 14]] = 1
+    keep = np.nonzero(pad[0] == 0)[0]
+    o, lse = oracle.attention_rows(q, k, v, 0.3, key_pad=pad)
+    # the kept-key problem has fewer keys than queries: evaluate row by row
+    # through the NumPy twin on [1, H, 1, d] queries
+    for i in range(N):
+        o1, l1 = oracle.attention_full(q[:, :, i:i + 1], k[:, :, keep], v[:, :, keep], 0.3)
+        np.testing.assert_allclose(o.reshape(B, H, N, d)[:, :, i], o1[:, :, 0], atol=1e-13)
+        np.testing.assert_allclose(lse.reshape(B, H, N)[:, :, i], l1[:, :, 0], atol=1e-13)
+
+
+def test_rows_without_visible_keys():
+    B, H, N, d = 2, 2, 7, 3
+    q = RNG.normal(size=(B, H, N, d))
+    k = RNG.normal(size=(B, H, N, d))
+    v = RNG.normal(size=(B, H, N, d))
+    pad = np.zeros((B, N), dtype=np.uint8)
+    pad[1, :] = 1                     # batch 1: every key padded
+    o, lse = oracle.attention_rows(q, k, v, 0.7, key_pad=pad)
+    o0, l0 = oracle.attention_rows(q[:1], k[:1], v[:1], 0.7)
+    o, lse = o.reshape(B, H, N, d), lse.reshape(B, H, N)
+    assert (o[1] == 0).all() and np.isneginf(lse[1]).all()
+    np.testing.assert_array_equal(o[0], o0.reshape(1, H, N, d)[0])
+    # causal: with keys 0..2 padded, rows 0..2 see nothing
+    pad2 = np.zeros((B, N), dtype=np.uint8)
+    pad2[:, :3] = 1
+    oc, lc = oracle.attention_rows(q, k, v, 0.7, True, key_pad=pad2)
+    oc, lc = oc.reshape(B, H, N, d), lc.reshape(B, H, N)
+    assert (oc[:, :, :3] == 0).all() and np.isneginf(lc[:, :, :3]).all()
+    assert np.isfinite(lc[:, :, 3:]).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_masked_c_oracle_matches_numpy_twin(causal):
+    q, k, v = make_qkv(2, 2, 41, 16, seed=13)
+    pad = (np.random.default_rng(5).random((2, 41)) < 0.3).astype(np.uint8)
+    pad[1, :] = 1
+    o, lse = oracle.attention_rows(q, k, v, 0.25, causal, key_pad=pad)
+    qd, kd, vd = (x.double().numpy() for x in (q, k, v))
+    o_np, lse_np = oracle.attention_full(qd, kd, vd, 0.25, causal, key_pad=pad)
+    np.testing.assert_allclose(o.reshape(o_np.shape), o_np, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(np.isneginf(lse.reshape(lse_np.shape)), np.isneginf(lse_np))
+    fin = np.isfinite(lse_np)
+    np.testing.assert_allclose(lse.reshape(lse_np.shape)[fin], lse_np[fin], rtol=0, atol=1e-12)
