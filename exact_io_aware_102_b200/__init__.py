@@ -5,7 +5,7 @@ library ``libattn.so`` (built from ``csrc/attn_fwd.cu`` for sm_100a); PyTorch
 supplies device memory and the current stream.  There is no fallback: if the
 library is missing, every entry point raises.
 
-The C entry points keep their names here (``attn_fwd``,
+The C entry points keep their names here (``attn_fwd``, ``attn_fwd_strided``,
 ``attn_status_string``, ``attn_check_device_status``,
 ``attn_selftest_wait_timeout``, ``attn_version``); ``forward`` is the tensor
 convenience wrapper.
@@ -15,7 +15,7 @@ import math
 import os
 
 __all__ = [
-    "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_status_string", "attn_check_device_status",
+    "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_fwd_strided", "attn_status_string", "attn_check_device_status",
     "attn_selftest_wait_timeout", "attn_version", "forward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
 ]
@@ -46,6 +46,10 @@ def library():
         vp, i32 = ctypes.c_void_p, ctypes.c_int
         lib.attn_fwd.restype = i32
         lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, i32, vp]
+        i64 = ctypes.c_longlong
+        lib.attn_fwd_strided.restype = i32
+        lib.attn_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i64, i64, i64, i64, i64,
+                                         ctypes.c_float, i32, vp]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_status_string.argtypes = [i32]
         lib.attn_check_device_status.restype = i32
@@ -62,6 +66,14 @@ def attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream):
     """Raw C call: pointers are ints (device addresses), stream an int handle; returns the status."""
     return library().attn_fwd(q, k, v, o, lse, int(B), int(H), int(N), int(d), float(scale),
                               int(bool(causal)), stream)
+
+
+def attn_fwd_strided(q, k, v, o, lse, B, H, N, d, qkv_strides, o_strides, scale, causal, stream):
+    """Raw C call with (batch, head, row) element strides for Q/K/V and for O."""
+    sb, sh, sn = (int(x) for x in qkv_strides)
+    ob, oh, on = (int(x) for x in o_strides)
+    return library().attn_fwd_strided(q, k, v, o, lse, int(B), int(H), int(N), int(d), sb, sh, sn, ob, oh, on,
+                                      float(scale), int(bool(causal)), stream)
 
 
 def attn_status_string(status):
@@ -93,30 +105,39 @@ def _stream_handle(stream):
 def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None):
     """Exact attention forward on bf16 CUDA tensors [B, H, N, d] (d = 64 or 128).
 
-    Returns (o, lse): o bf16 [B, H, N, d] and lse fp32 [B, H, N] (natural-log
-    log-sum-exp of each row's scaled scores).  ``scale`` defaults to 1/sqrt(d).
-    ``out`` / ``lse`` may be given to write into existing tensors.  The call is
-    asynchronous on ``stream`` (default: the current stream).
+    q, k and v may be strided views (for example of one packed projection
+    output) as long as their head dimension is contiguous and they share one
+    set of strides; ``out`` may be a strided view too (default: a new
+    contiguous tensor).  Returns (o, lse): o bf16 [B, H, N, d] and lse fp32
+    [B, H, N] (natural-log log-sum-exp of each row's scaled scores).
+    ``scale`` defaults to 1/sqrt(d).  The call is asynchronous on ``stream``
+    (default: the current stream).
     """
     import torch
     if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
         raise ValueError("q, k, v must share one shape [B, H, N, d]")
     for name, t in (("q", q), ("k", k), ("v", v)):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("%s must be a contiguous bf16 CUDA tensor" % name)
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.stride(3) != 1:
+            raise ValueError("%s must be a bf16 CUDA tensor with a contiguous last dimension" % name)
+    if k.stride() != q.stride() or v.stride() != q.stride():
+        raise ValueError("q, k, v must share one set of strides")
     B, H, N, d = (int(x) for x in q.shape)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
-        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if out.shape != q.shape or out.dtype != torch.bfloat16 or out.stride(3) != 1:
+        raise ValueError("out must be a bf16 tensor shaped like q with a contiguous last dimension")
     if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 tensor [B, H, N]")
-    status = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                      B, H, N, d, scale, causal, _stream_handle(stream))
+    # the stride of a size-1 dimension is never used: give it the contiguous value
+    def strides(t):
+        dense = (H * N * d, N * d, d)
+        return [st if n > 1 else c for n, st, c in zip(t.shape[:3], t.stride()[:3], dense)]
+    status = attn_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                              B, H, N, d, strides(q), strides(out), scale, causal, _stream_handle(stream))
     if status != ATTN_OK:
-        raise AttnError(status, "attn_fwd")
+        raise AttnError(status, "attn_fwd_strided")
     return out, lse

@@ -207,12 +207,12 @@ __device__ __forceinline__ void fence_proxy_async() {
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x,
-                                            int y, int z) {
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                            int z, int w) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
         : "memory");
 }
 
@@ -377,13 +377,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool b_mn_ma
 
 // ------------------------------------------------------------- the scheduler
 struct Params {
-    int BH, N, n_pairs, n_kv_all, total_units;
+    int BH, H, N, n_pairs, n_kv_all, total_units;
+    long long o_sb, o_sh, o_sn;  // element strides of O over (batch, head, row)
     float scale_log2;  // scale * log2(e)
     unsigned long long wait_ns;
 };
 
 struct Unit {
-    int bh, q0, n0, n1;  // head, first query row, key tiles for Q tile 0 / 1
+    int bh, b, h, q0, n0, n1;  // head (flat, batch, within batch), first query row, key tiles for Q tile 0 / 1
 };
 
 // Work units: (head, pair of Q tiles).  Non-causal: heads-major so the CTAs
@@ -402,6 +403,8 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
         pair = u % p.n_pairs;
         w.bh = u / p.n_pairs;
     }
+    w.b = w.bh / p.H;
+    w.h = w.bh - w.b * p.H;
     w.q0 = pair * kUnitRows;
     if (CAUSAL) {
         w.n1 = min(p.n_kv_all, (w.q0 + kUnitRows) / kBlockN);  // tiles touching rows < q0 + 256
@@ -440,14 +443,14 @@ __device__ __forceinline__ void role_producer(const Ctx& c, const CUtensorMap* t
     Ring rv{c.base + C::kVRingOff, c.bar + Bars::kVFull, c.bar + Bars::kVEmpty, (uint32_t)C::kVSlots, 0};
     uint32_t q_issued = 0;
     bool ok = true;
-    auto load = [&](Ring& r, const CUtensorMap* map, int key0, int bh) {
+    auto load = [&](Ring& r, const CUtensorMap* map, int key0, const Unit& w) {
         const uint32_t s = r.slot();
         if (!wait_bounded(r.empty + 8 * s, r.phase() ^ 1u, c.abort_flag, c.p.wait_ns)) return false;
         const uint32_t fb = r.full + 8 * s;
         const uint32_t dst = r.smem + s * C::kTileBytes;
         mbar_expect_tx(fb, C::kTileBytes);
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h) tma_load_3d(dst + h * C::kHalfBytes, map, fb, h * 64, key0, bh);
+        for (int x = 0; x < D / 64; ++x) tma_load_4d(dst + x * C::kHalfBytes, map, fb, x * 64, key0, w.h, w.b);
         ++r.i;
         return true;
     };
@@ -463,13 +466,13 @@ __device__ __forceinline__ void role_producer(const Ctx& c, const CUtensorMap* t
             const uint32_t dst = c.base + C::kQOff + t * C::kTileBytes;
             mbar_expect_tx(qb, C::kTileBytes);
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h)
-                tma_load_3d(dst + h * C::kHalfBytes, tm_q, qb, h * 64, w.q0 + t * kBlockM, w.bh);
+            for (int x = 0; x < D / 64; ++x)
+                tma_load_4d(dst + x * C::kHalfBytes, tm_q, qb, x * 64, w.q0 + t * kBlockM, w.h, w.b);
         }
         q_issued = local + 1;
         for (int j = 0; ok && j < w.n1; ++j) {
-            ok = load(rk, tm_k, j * kBlockN, w.bh);
-            if (ok) ok = load(C::kSplit ? rv : rk, tm_v, j * kBlockN, w.bh);
+            ok = load(rk, tm_k, j * kBlockN, w);
+            if (ok) ok = load(C::kSplit ? rv : rk, tm_v, j * kBlockN, w);
         }
     }
     if (!ok) {
@@ -815,7 +818,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
         tc_fence_after();
         const float inv_l = 1.f / l;
         const bool store = row < p.N;
-        uint16_t* orow = out_o + (static_cast<size_t>(w.bh) * p.N + (store ? row : 0)) * D;
+        uint16_t* orow = out_o + w.b * p.o_sb + w.h * p.o_sh + (store ? row : 0) * p.o_sn;
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t r[32];
@@ -966,17 +969,30 @@ DriverFns& driver_fns() {
     return fns;
 }
 
-// [B*H, N, d] bf16 viewed as a 3-D tensor; box = 64 columns x 128 rows x 1 head, 128-byte swizzle.
-bool encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                                static_cast<cuuint64_t>(BH)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBlockN), 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return driver_fns().encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+// A bf16 tensor indexed [b, h, n, k] with element strides (sb, sh, sn, 1),
+// viewed as a 4-D tensor (k, n, h, b); box = 64 columns x 128 rows x 1 x 1,
+// 128-byte swizzle.  Rows past N read as zeros.
+bool encode_qkv_map(CUtensorMap* map, const void* ptr, int B, int H, int N, int d, long long sb, long long sh,
+                    long long sn) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(sn) * 2, static_cast<cuuint64_t>(sh) * 2,
+                                   static_cast<cuuint64_t>(sb) * 2};
+    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(kBlockN), 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return driver_fns().encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Largest element offset + 1 of a [B, H, N, d] tensor with the given strides
+// (0 if it would not fit in 2^46 elements).
+size_t span_elems(int B, int H, int N, int d, long long sb, long long sh, long long sn) {
+    const unsigned __int128 e = static_cast<unsigned __int128>(B - 1) * sb +
+                                static_cast<unsigned __int128>(H - 1) * sh +
+                                static_cast<unsigned __int128>(N - 1) * sn + d;
+    return e > (static_cast<unsigned __int128>(1) << 46) ? 0 : static_cast<size_t>(e);
 }
 
 // The pointer must be device memory of `device` and its allocation must hold `bytes` from it.
@@ -1028,8 +1044,9 @@ const char* attn_status_string(int status) {
     }
 }
 
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-             float scale, int causal, attn_stream_t stream) {
+int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                     long long qkv_sb, long long qkv_sh, long long qkv_sn, long long o_sb, long long o_sh,
+                     long long o_sn, float scale, int causal, attn_stream_t stream) {
     // ---- host-side validation: nothing touches the GPU until all of it passes
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
@@ -1038,35 +1055,48 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     // row maximum is taken before scaling.
     if (!isfinite(scale) || !(scale >= 1e-30f)) return ATTN_ERR_INVALID_ARG;
     const long long BH = static_cast<long long>(B) * H;
-    if (BH > 0x7fffffffLL || N > 0x7fffffff - kUnitRows) return ATTN_ERR_INVALID_ARG;
+    if (BH > 0x7fffffffLL || N > 0x7fffffff - 2 * kBlockM) return ATTN_ERR_INVALID_ARG;
+    // strides: positive, 16-byte multiples (TMA and the 16-byte O stores), and
+    // small enough that every offset fits the 40-bit TMA stride range
+    const long long lim = 1LL << 36;
+    for (long long st : {qkv_sb, qkv_sh, qkv_sn, o_sb, o_sh, o_sn})
+        if (st < 8 || st % 8 != 0 || st > lim) return ATTN_ERR_INVALID_ARG;
+    if (qkv_sn < d || o_sn < d) return ATTN_ERR_INVALID_ARG;  // rows must not overlap
     auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
     if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) || misaligned(lse, 4))
         return ATTN_ERR_INVALID_ARG;
-    const size_t elems = static_cast<size_t>(BH) * N * d;
-    const size_t tbytes = elems * 2, lbytes = static_cast<size_t>(BH) * N * 4;
-    if (overlaps(o, tbytes, q, tbytes) || overlaps(o, tbytes, k, tbytes) || overlaps(o, tbytes, v, tbytes) ||
-        overlaps(lse, lbytes, q, tbytes) || overlaps(lse, lbytes, k, tbytes) || overlaps(lse, lbytes, v, tbytes) ||
-        overlaps(lse, lbytes, o, tbytes))
+    const size_t in_bytes = span_elems(B, H, N, d, qkv_sb, qkv_sh, qkv_sn) * 2;
+    const size_t out_bytes = span_elems(B, H, N, d, o_sb, o_sh, o_sn) * 2;
+    const size_t lbytes = static_cast<size_t>(BH) * N * 4;
+    if (in_bytes == 0 || out_bytes == 0) return ATTN_ERR_INVALID_ARG;
+    if (overlaps(o, out_bytes, q, in_bytes) || overlaps(o, out_bytes, k, in_bytes) ||
+        overlaps(o, out_bytes, v, in_bytes) || overlaps(lse, lbytes, q, in_bytes) ||
+        overlaps(lse, lbytes, k, in_bytes) || overlaps(lse, lbytes, v, in_bytes) || overlaps(lse, lbytes, o, out_bytes))
         return ATTN_ERR_INVALID_ARG;
 
     if (!driver_fns().ok) return ATTN_ERR_CUDA;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
-    if (!device_span_ok(q, tbytes, dev) || !device_span_ok(k, tbytes, dev) || !device_span_ok(v, tbytes, dev) ||
-        !device_span_ok(o, tbytes, dev) || !device_span_ok(lse, lbytes, dev))
+    if (!device_span_ok(q, in_bytes, dev) || !device_span_ok(k, in_bytes, dev) || !device_span_ok(v, in_bytes, dev) ||
+        !device_span_ok(o, out_bytes, dev) || !device_span_ok(lse, lbytes, dev))
         return ATTN_ERR_INVALID_ARG;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         return ATTN_ERR_CUDA;
 
     alignas(64) CUtensorMap mq, mk, mv;
-    if (!encode_qkv_map(&mq, q, static_cast<int>(BH), N, d) || !encode_qkv_map(&mk, k, static_cast<int>(BH), N, d) ||
-        !encode_qkv_map(&mv, v, static_cast<int>(BH), N, d))
+    if (!encode_qkv_map(&mq, q, B, H, N, d, qkv_sb, qkv_sh, qkv_sn) ||
+        !encode_qkv_map(&mk, k, B, H, N, d, qkv_sb, qkv_sh, qkv_sn) ||
+        !encode_qkv_map(&mv, v, B, H, N, d, qkv_sb, qkv_sh, qkv_sn))
         return ATTN_ERR_CUDA;
 
     Params p;
     p.BH = static_cast<int>(BH);
+    p.H = H;
     p.N = N;
+    p.o_sb = o_sb;
+    p.o_sh = o_sh;
+    p.o_sn = o_sn;
     p.n_pairs = (N + kUnitRows - 1) / kUnitRows;
     p.n_kv_all = (N + kBlockN - 1) / kBlockN;
     const long long units = BH * p.n_pairs;
@@ -1081,6 +1111,13 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
         return causal ? launch<64, true>(mq, mk, mv, o, lse, p, grid, s) : launch<64, false>(mq, mk, mv, o, lse, p, grid, s);
     }
     return causal ? launch<128, true>(mq, mk, mv, o, lse, p, grid, s) : launch<128, false>(mq, mk, mv, o, lse, p, grid, s);
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+             float scale, int causal, attn_stream_t stream) {
+    // contiguous [B, H, N, d]
+    const long long sn = d, sh = static_cast<long long>(N) * d, sb = static_cast<long long>(H) * N * d;
+    return attn_fwd_strided(q, k, v, o, lse, B, H, N, d, sb, sh, sn, sb, sh, sn, scale, causal, stream);
 }
 
 int attn_check_device_status(attn_stream_t stream) {

@@ -62,6 +62,31 @@ typedef enum {
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
 
+/*
+ * attn_fwd_strided -- attn_fwd on strided tensors, with no copy.
+ *
+ * Element (b, h, n, t) of Q, K and V is at ptr[b*qkv_sb + h*qkv_sh + n*qkv_sn
+ * + t]; element (b, h, n, t) of O at o[b*o_sb + h*o_sh + n*o_sn + t] (strides in
+ * elements; the head dimension t is contiguous).  This covers, for example,
+ * Q, K and V taken as views of one packed projection output [B, N, 3, H, d]
+ * (qkv_sb = 3*N*H*d, qkv_sh = d, qkv_sn = 3*H*d) and O written straight into a
+ * [B, N, H, d] buffer (o_sb = N*H*d, o_sh = d, o_sn = H*d): the physical
+ * layout the pages' patch self-attention module builds before its transpose
+ * (flash-attnの代役がVRAMを18GB溶かしていたので87%削った話, §4).  LSE stays
+ * contiguous fp32 [B, H, N].
+ *
+ * Every stride must be a positive multiple of 8 (16 bytes, for the tensor
+ * memory accelerator and the 16-byte O stores), qkv_sn and o_sn at least d,
+ * and each pointer's allocation must cover its strided span; otherwise
+ * ATTN_ERR_INVALID_ARG and nothing is launched.  Other arguments, ownership
+ * and errors as attn_fwd (which is this call with contiguous strides).
+ */
+int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int N, int d,
+                     long long qkv_sb, long long qkv_sh, long long qkv_sn,
+                     long long o_sb, long long o_sh, long long o_sn,
+                     float scale, int causal, attn_stream_t stream);
+
 /* Human-readable name of an attn_status value (static string, never NULL). */
 const char* attn_status_string(int status);
 

@@ -27,7 +27,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    assert {"attn_fwd", "attn_status_string", "attn_check_device_status",
+    assert {"attn_fwd", "attn_fwd_strided", "attn_status_string", "attn_check_device_status",
             "attn_selftest_wait_timeout", "attn_version"} <= set(names)
 
 
@@ -90,6 +90,27 @@ def test_overlapping_outputs_rejected(lib):
     # lse overlapping o
     assert pkg.attn_fwd(base, base + 2 * n_bytes, base + 4 * n_bytes, base + 6 * n_bytes,
                         base + 6 * n_bytes + 64, 1, 2, 64, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("qkv,o", [
+    ((8192, 64, 0), (8192, 64, 64)),       # zero row stride
+    ((8192, 64, 60), (8192, 64, 64)),      # row stride below d
+    ((8192, 64, 68), (8192, 64, 64)),      # not a multiple of 8 elements (16 bytes)
+    ((8192, 4, 64), (8192, 64, 64)),       # head stride not a multiple of 8
+    ((8192, 64, 64), (-8192, 64, 64)),     # negative stride
+    ((8192, 64, 64), (8192, 64, 1 << 40)),  # beyond the tensor-map stride range
+])
+def test_bad_strides_rejected_on_host(lib, qkv, o):
+    assert pkg.attn_fwd_strided(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5, 1, 2, 64, 64, qkv, o, 0.125, 0,
+                                None) == pkg.ATTN_ERR_INVALID_ARG
+
+
+def test_strided_overlap_uses_the_strided_span(lib):
+    # O's span under its strides reaches into q's allocation range: rejected
+    base = 1 << 24
+    assert pkg.attn_fwd_strided(base, base + (1 << 22), base + (2 << 22), base - 4096, base + (3 << 22),
+                                1, 2, 64, 64, (8192, 64, 128), (8192, 64, 128), 0.125, 0,
+                                None) == pkg.ATTN_ERR_INVALID_ARG
 
 
 def test_selftest_limit_validated(lib):

@@ -143,3 +143,45 @@ def test_permuting_keys_and_values_leaves_output_unchanged():
     o2, l2 = pkg.forward(q.to(dev), k[:, :, perm].contiguous().to(dev), v[:, :, perm].contiguous().to(dev))
     assert (o1.float() - o2.float()).abs().max().item() <= TOL_O
     assert (l1 - l2).abs().max().item() <= TOL_LSE
+
+
+# ---- strided inputs and outputs: the patch self-attention module's layout
+@pytest.mark.parametrize("d,causal", [(64, False), (64, True), (128, False), (128, True)])
+def test_packed_projection_layout_matches_contiguous(d, causal):
+    # Q, K, V as views of one packed projection output [B, N, 3, H, d] and O
+    # written straight into a [B, N, H, d] buffer: no transpose copies.
+    dev = torch.device("cuda:0")
+    B, H, N = 2, 3, 333
+    g = torch.Generator().manual_seed(21)
+    packed = torch.randn(B, N, 3, H, d, generator=g).to(torch.bfloat16).to(dev)
+    q, k, v = (packed[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    assert not q.is_contiguous()
+    o_buf = torch.full((B, N, H, d), 7.0, dtype=torch.bfloat16, device=dev)
+    o_view = o_buf.permute(0, 2, 1, 3)
+    o, lse = pkg.forward(q, k, v, causal=causal, out=o_view)
+    assert o.data_ptr() == o_buf.data_ptr()
+    o_ref, lse_ref = pkg.forward(q.contiguous(), k.contiguous(), v.contiguous(), causal=causal)
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    # the same kernel on the same values: identical results
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+    # and against the oracle on the logical [B, H, N, d] tensors
+    qc, kc, vc = (x.contiguous().cpu() for x in (q, k, v))
+    oo, lo = oracle.attention_rows(qc, kc, vc, 1.0 / math.sqrt(d), causal)
+    assert np.abs(o.float().cpu().numpy().reshape(oo.shape) - oo).max() <= TOL_O
+    assert np.abs(lse.cpu().numpy().reshape(lo.shape) - lo).max() <= TOL_LSE
+
+
+def test_strided_headline_layout_sampled():
+    # the 3 MP workload in the module's packed layout, checked on sampled rows
+    dev = torch.device("cuda:0")
+    B, H, N, d = 1, 16, 11616, 64
+    q0, k0, v0 = make_qkv(B, H, N, d, seed=0)
+    packed = torch.stack([x.permute(0, 2, 1, 3) for x in (q0, k0, v0)], dim=2).to(dev)  # [B, N, 3, H, d]
+    q, k, v = (packed[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    o, lse = pkg.forward(q, k, v)
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    idx = sample_rows(B, H, N, 64).numpy()
+    o_ref, lse_ref = oracle.attention_rows(q0, k0, v0, 1.0 / 8, False, rows=idx)
+    o_gpu = np.take_along_axis(o.float().cpu().numpy().reshape(B * H, N, d), idx[..., None], 1)
+    l_gpu = np.take_along_axis(lse.cpu().numpy().reshape(B * H, N), idx, 1)
+    assert np.abs(o_gpu - o_ref).max() <= TOL_O and np.abs(l_gpu - lse_ref).max() <= TOL_LSE
