@@ -49,7 +49,7 @@ def library():
         i64 = ctypes.c_longlong
         lib.attn_fwd_strided.restype = i32
         lib.attn_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i64, i64, i64, i64, i64,
-                                         ctypes.c_float, i32, vp]
+                                         vp, ctypes.c_float, i32, vp]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_status_string.argtypes = [i32]
         lib.attn_check_device_status.restype = i32
@@ -68,12 +68,14 @@ def attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream):
                               int(bool(causal)), stream)
 
 
-def attn_fwd_strided(q, k, v, o, lse, B, H, N, d, qkv_strides, o_strides, scale, causal, stream):
-    """Raw C call with (batch, head, row) element strides for Q/K/V and for O."""
+def attn_fwd_strided(q, k, v, o, lse, B, H, N, d, qkv_strides, o_strides, scale, causal, stream,
+                     key_padding_mask=None):
+    """Raw C call with (batch, head, row) element strides for Q/K/V and for O,
+    and an optional device address of a [B, N] byte key-padding mask."""
     sb, sh, sn = (int(x) for x in qkv_strides)
     ob, oh, on = (int(x) for x in o_strides)
     return library().attn_fwd_strided(q, k, v, o, lse, int(B), int(H), int(N), int(d), sb, sh, sn, ob, oh, on,
-                                      float(scale), int(bool(causal)), stream)
+                                      key_padding_mask, float(scale), int(bool(causal)), stream)
 
 
 def attn_status_string(status):
@@ -102,7 +104,7 @@ def _stream_handle(stream):
     return stream.cuda_stream
 
 
-def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None):
+def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None, key_padding_mask=None):
     """Exact attention forward on bf16 CUDA tensors [B, H, N, d] (d = 64 or 128).
 
     q, k and v may be strided views (for example of one packed projection
@@ -110,8 +112,10 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None):
     set of strides; ``out`` may be a strided view too (default: a new
     contiguous tensor).  Returns (o, lse): o bf16 [B, H, N, d] and lse fp32
     [B, H, N] (natural-log log-sum-exp of each row's scaled scores).
-    ``scale`` defaults to 1/sqrt(d).  The call is asynchronous on ``stream``
-    (default: the current stream).
+    ``scale`` defaults to 1/sqrt(d).  ``key_padding_mask``: None or a bool /
+    uint8 CUDA tensor [B, N], True (nonzero) = padded key, excluded from every
+    query row of that batch; a row with no visible key gets O = 0 and LSE =
+    -inf.  The call is asynchronous on ``stream`` (default: the current stream).
     """
     import torch
     if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
@@ -132,12 +136,19 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None):
         raise ValueError("out must be a bf16 tensor shaped like q with a contiguous last dimension")
     if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 tensor [B, H, N]")
+    pad_ptr = None
+    if key_padding_mask is not None:
+        if (key_padding_mask.shape != (B, N) or key_padding_mask.dtype not in (torch.bool, torch.uint8)
+                or not key_padding_mask.is_cuda or not key_padding_mask.is_contiguous()):
+            raise ValueError("key_padding_mask must be a contiguous bool/uint8 CUDA tensor [B, N]")
+        pad_ptr = key_padding_mask.data_ptr()
     # the stride of a size-1 dimension is never used: give it the contiguous value
     def strides(t):
         dense = (H * N * d, N * d, d)
         return [st if n > 1 else c for n, st, c in zip(t.shape[:3], t.stride()[:3], dense)]
     status = attn_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                              B, H, N, d, strides(q), strides(out), scale, causal, _stream_handle(stream))
+                              B, H, N, d, strides(q), strides(out), scale, causal, _stream_handle(stream),
+                              key_padding_mask=pad_ptr)
     if status != ATTN_OK:
         raise AttnError(status, "attn_fwd_strided")
     return out, lse

@@ -305,6 +305,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// 16 bytes through the read-only path (every thread of a warpgroup reads the
+// same mask bytes: one broadcast transaction, then L1 hits).
+__device__ __forceinline__ uint4 ldg_nc16(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -379,6 +389,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool b_mn_ma
 struct Params {
     int BH, H, N, n_pairs, n_kv_all, total_units;
     long long o_sb, o_sh, o_sn;  // element strides of O over (batch, head, row)
+    const uint8_t* key_pad;      // [B, N] key-padding mask (nonzero = padded) or null
+    int pad_vec;                 // key_pad rows may be read 16 bytes at a time
     float scale_log2;  // scale * log2(e)
     unsigned long long wait_ns;
 };
@@ -659,7 +671,7 @@ __device__ __forceinline__ void role_mma_ordered(const Ctx& c) {
 
 // ------------------------------------------------------- softmax + epilogue
 // Warpgroup t owns Q tile t; thread = one query row = one TMEM lane.
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool MASK>
 __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, uint16_t* __restrict__ out_o,
                                              float* __restrict__ out_lse) {
     using C = Cfg<D>;
@@ -719,6 +731,33 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
                 // S_t is in registers: the S stream may refill it with the next key tile
                 tc_fence_before();
                 mbar_arrive(b_sfree);
+            }
+            // key padding: the 128 mask bytes of this key tile, 16 at a time;
+            // only 16-key groups that hold a padded key are touched
+            if (MASK) {
+                const int key0 = j * kBlockN;
+                const uint8_t* mrow = p.key_pad + static_cast<size_t>(w.b) * p.N + key0;
+                const bool vec = p.pad_vec && key0 + kBlockN <= p.N;
+#pragma unroll
+                for (int g = 0; g < kBlockN / 16; ++g) {
+                    uint4 x;
+                    if (vec) {
+                        x = ldg_nc16(mrow + 16 * g);
+                    } else {
+                        uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (key0 + 16 * g + e < p.N)
+                                wd[e >> 2] |= static_cast<uint32_t>(mrow[16 * g + e] != 0) << (8 * (e & 3));
+                        x = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                    }
+                    if (x.x | x.y | x.z | x.w) {
+                        const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if ((wv[e >> 2] >> (8 * (e & 3))) & 0xFFu) s[16 * g + e] = -INFINITY;
+                    }
+                }
             }
             // key-tail and causal mask: keys past last_key get -inf
             const int lim = last_key - j * kBlockN;
@@ -816,7 +855,10 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
             break;
         }
         tc_fence_after();
-        const float inv_l = 1.f / l;
+        // a row that saw no visible key (every key it may see is padded) keeps
+        // m = -inf: its O is 0 and its LSE -inf
+        const bool empty = (m == -INFINITY);
+        const float inv_l = empty ? 0.f : 1.f / l;
         const bool store = row < p.N;
         uint16_t* orow = out_o + w.b * p.o_sb + w.h * p.o_sh + (store ? row : 0) * p.o_sn;
 #pragma unroll
@@ -840,12 +882,12 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
                     dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
             }
         }
-        if (store) out_lse[static_cast<size_t>(w.bh) * p.N + row] = (m + __log2f(l)) * kLn2;
+        if (store) out_lse[static_cast<size_t>(w.bh) * p.N + row] = empty ? -INFINITY : (m + __log2f(l)) * kLn2;
     }
 }
 
 // ----------------------------------------------------------------- the kernel
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool MASK>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out_o,
@@ -913,7 +955,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncwarp();
     } else {
         regs_increase<kSoftmaxRegs>();
-        role_softmax<D, CAUSAL>(ctx, warp, lane, out_o, out_lse);
+        role_softmax<D, CAUSAL, MASK>(ctx, warp, lane, out_o, out_lse);
     }
 
     tc_fence_before();
@@ -1016,10 +1058,10 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool MASK>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
            const Params& p, int grid, cudaStream_t stream) {
-    auto kernel = attn_fwd_kernel<D, CAUSAL>;
+    auto kernel = attn_fwd_kernel<D, CAUSAL, MASK>;
     const int smem = Cfg<D>::kSmemBytes;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return ATTN_ERR_CUDA;
@@ -1046,7 +1088,8 @@ const char* attn_status_string(int status) {
 
 int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                      long long qkv_sb, long long qkv_sh, long long qkv_sn, long long o_sb, long long o_sh,
-                     long long o_sn, float scale, int causal, attn_stream_t stream) {
+                     long long o_sn, const unsigned char* key_padding_mask, float scale, int causal,
+                     attn_stream_t stream) {
     // ---- host-side validation: nothing touches the GPU until all of it passes
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
@@ -1073,12 +1116,17 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
         overlaps(o, out_bytes, v, in_bytes) || overlaps(lse, lbytes, q, in_bytes) ||
         overlaps(lse, lbytes, k, in_bytes) || overlaps(lse, lbytes, v, in_bytes) || overlaps(lse, lbytes, o, out_bytes))
         return ATTN_ERR_INVALID_ARG;
+    const size_t pad_bytes = static_cast<size_t>(B) * N;
+    if (key_padding_mask &&
+        (overlaps(o, out_bytes, key_padding_mask, pad_bytes) || overlaps(lse, lbytes, key_padding_mask, pad_bytes)))
+        return ATTN_ERR_INVALID_ARG;
 
     if (!driver_fns().ok) return ATTN_ERR_CUDA;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
     if (!device_span_ok(q, in_bytes, dev) || !device_span_ok(k, in_bytes, dev) || !device_span_ok(v, in_bytes, dev) ||
-        !device_span_ok(o, out_bytes, dev) || !device_span_ok(lse, lbytes, dev))
+        !device_span_ok(o, out_bytes, dev) || !device_span_ok(lse, lbytes, dev) ||
+        (key_padding_mask && !device_span_ok(key_padding_mask, pad_bytes, dev)))
         return ATTN_ERR_INVALID_ARG;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
@@ -1097,6 +1145,8 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
     p.o_sb = o_sb;
     p.o_sh = o_sh;
     p.o_sn = o_sn;
+    p.key_pad = key_padding_mask;
+    p.pad_vec = key_padding_mask && (reinterpret_cast<uintptr_t>(key_padding_mask) & 15) == 0 && N % 16 == 0;
     p.n_pairs = (N + kUnitRows - 1) / kUnitRows;
     p.n_kv_all = (N + kBlockN - 1) / kBlockN;
     const long long units = BH * p.n_pairs;
@@ -1107,17 +1157,26 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
     const int grid = static_cast<int>(units < sms ? units : sms);
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool mask = key_padding_mask != nullptr;
     if (d == 64) {
-        return causal ? launch<64, true>(mq, mk, mv, o, lse, p, grid, s) : launch<64, false>(mq, mk, mv, o, lse, p, grid, s);
+        if (mask)
+            return causal ? launch<64, true, true>(mq, mk, mv, o, lse, p, grid, s)
+                          : launch<64, false, true>(mq, mk, mv, o, lse, p, grid, s);
+        return causal ? launch<64, true, false>(mq, mk, mv, o, lse, p, grid, s)
+                      : launch<64, false, false>(mq, mk, mv, o, lse, p, grid, s);
     }
-    return causal ? launch<128, true>(mq, mk, mv, o, lse, p, grid, s) : launch<128, false>(mq, mk, mv, o, lse, p, grid, s);
+    if (mask)
+        return causal ? launch<128, true, true>(mq, mk, mv, o, lse, p, grid, s)
+                      : launch<128, false, true>(mq, mk, mv, o, lse, p, grid, s);
+    return causal ? launch<128, true, false>(mq, mk, mv, o, lse, p, grid, s)
+                  : launch<128, false, false>(mq, mk, mv, o, lse, p, grid, s);
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
              float scale, int causal, attn_stream_t stream) {
     // contiguous [B, H, N, d]
     const long long sn = d, sh = static_cast<long long>(N) * d, sb = static_cast<long long>(H) * N * d;
-    return attn_fwd_strided(q, k, v, o, lse, B, H, N, d, sb, sh, sn, sb, sh, sn, scale, causal, stream);
+    return attn_fwd_strided(q, k, v, o, lse, B, H, N, d, sb, sh, sn, sb, sh, sn, nullptr, scale, causal, stream);
 }
 
 int attn_check_device_status(attn_stream_t stream) {

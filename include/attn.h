@@ -63,7 +63,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
 
 /*
- * attn_fwd_strided -- attn_fwd on strided tensors, with no copy.
+ * attn_fwd_strided -- attn_fwd on strided tensors, with no copy, and an
+ * optional key-padding mask.
  *
  * Element (b, h, n, t) of Q, K and V is at ptr[b*qkv_sb + h*qkv_sh + n*qkv_sn
  * + t]; element (b, h, n, t) of O at o[b*o_sb + h*o_sh + n*o_sn + t] (strides in
@@ -75,16 +76,27 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  * (flash-attnの代役がVRAMを18GB溶かしていたので87%削った話, §4).  LSE stays
  * contiguous fp32 [B, H, N].
  *
+ * key_padding_mask: NULL, or a device byte mask [B, N] (contiguous, read
+ * only, any alignment) in which a nonzero byte marks a padded key of that
+ * batch: it is excluded from every query row, as the key_padding_mask of the
+ * pages' module (same page, §3 and §6: nonzero = ignore, the opposite of a
+ * boolean "attend" mask).  A query row with no visible key (all keys it may
+ * see padded) gets O = 0 and LSE = -inf.  Reading the mask 16 bytes at a time
+ * needs a 16-byte aligned mask and N % 16 == 0; otherwise it is read byte by
+ * byte (same result, slower).
+ *
  * Every stride must be a positive multiple of 8 (16 bytes, for the tensor
  * memory accelerator and the 16-byte O stores), qkv_sn and o_sn at least d,
  * and each pointer's allocation must cover its strided span; otherwise
  * ATTN_ERR_INVALID_ARG and nothing is launched.  Other arguments, ownership
- * and errors as attn_fwd (which is this call with contiguous strides).
+ * and errors as attn_fwd (which is this call with contiguous strides and no
+ * padding).
  */
 int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
                      int B, int H, int N, int d,
                      long long qkv_sb, long long qkv_sh, long long qkv_sn,
                      long long o_sb, long long o_sh, long long o_sn,
+                     const unsigned char* key_padding_mask,
                      float scale, int causal, attn_stream_t stream);
 
 /* Human-readable name of an attn_status value (static string, never NULL). */

@@ -185,3 +185,64 @@ def test_strided_headline_layout_sampled():
     o_gpu = np.take_along_axis(o.float().cpu().numpy().reshape(B * H, N, d), idx[..., None], 1)
     l_gpu = np.take_along_axis(lse.cpu().numpy().reshape(B * H, N), idx, 1)
     assert np.abs(o_gpu - o_ref).max() <= TOL_O and np.abs(l_gpu - lse_ref).max() <= TOL_LSE
+
+
+# ---- key padding (the pages' mask pass): nonzero = padded key
+def masked_check(B, H, N, d, causal, pad, seed=0):
+    dev = torch.device("cuda:0")
+    q, k, v = make_qkv(B, H, N, d, seed=seed)
+    pad_t = torch.as_tensor(pad, dtype=torch.bool)
+    o, lse = pkg.forward(q.to(dev), k.to(dev), v.to(dev), causal=causal, key_padding_mask=pad_t.to(dev))
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    o_ref, lse_ref = oracle.attention_rows(q, k, v, 1.0 / math.sqrt(d), causal, key_pad=pad.astype(np.uint8))
+    o = o.float().cpu().numpy().reshape(o_ref.shape)
+    lse = lse.cpu().numpy().reshape(lse_ref.shape)
+    assert np.abs(o - o_ref).max() <= TOL_O
+    empty = np.isneginf(lse_ref)
+    assert (np.isneginf(lse) == empty).all()
+    assert np.abs(lse[~empty] - lse_ref[~empty]).max() <= TOL_LSE if (~empty).any() else True
+    assert (o.reshape(-1, d)[empty.reshape(-1)] == 0).all()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [300, 512, 1000])   # 512: the 16-byte mask path; 300, 1000: bytewise
+def test_key_padding_trailing_and_scattered(N, d, causal):
+    B = 3
+    rng = np.random.default_rng(N + d)
+    pad = np.zeros((B, N), dtype=bool)
+    pad[0, N - 37:] = True                            # trailing padding
+    pad[1] = rng.random(N) < 0.3                      # scattered padding
+    pad[1, 0] = False
+    pad[2, : N // 2] = True                           # leading padding: causal rows < N/2 see nothing
+    masked_check(B, 2, N, d, causal, pad, seed=N)
+
+
+def test_key_padding_fully_padded_batch_and_no_padding():
+    dev = torch.device("cuda:0")
+    B, H, N, d = 2, 2, 640, 64
+    pad = np.zeros((B, N), dtype=bool)
+    pad[1] = True
+    masked_check(B, H, N, d, False, pad, seed=3)
+    # an all-False mask is the same computation as no mask
+    q, k, v = (x.to(dev) for x in make_qkv(B, H, N, d, seed=4))
+    none = torch.zeros(B, N, dtype=torch.bool, device=dev)
+    o1, l1 = pkg.forward(q, k, v, key_padding_mask=none)
+    o2, l2 = pkg.forward(q, k, v)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_key_padding_image_workload_sampled():
+    # 0.5 MP patch self-attention with its last 200 patches padded
+    dev = torch.device("cuda:0")
+    B, H, N, d = 2, 16, 1944, 64
+    q, k, v = make_qkv(B, H, N, d, seed=0)
+    pad = np.zeros((B, N), dtype=bool)
+    pad[1, N - 200:] = True
+    pad_t = torch.as_tensor(pad).to(dev)
+    o, lse = pkg.forward(q.to(dev), k.to(dev), v.to(dev), key_padding_mask=pad_t)
+    idx = sample_rows(B, H, N, 128).numpy()
+    o_ref, lse_ref = oracle.attention_rows(q, k, v, 1.0 / 8, False, rows=idx, key_pad=pad.astype(np.uint8))
+    o_gpu = np.take_along_axis(o.float().cpu().numpy().reshape(B * H, N, d), idx[..., None], 1)
+    l_gpu = np.take_along_axis(lse.cpu().numpy().reshape(B * H, N), idx, 1)
+    assert np.abs(o_gpu - o_ref).max() <= TOL_O and np.abs(l_gpu - lse_ref).max() <= TOL_LSE
