@@ -25,6 +25,13 @@
  * padded key, excluded from every row of that batch (the key_padding_mask
  * convention: nonzero = ignore, the opposite of a boolean "attend" mask).
  *
+ * Block sparsity (FlashAttention: Fast and Memory-Efficient Exact Attention
+ * with IO-Awareness, wiki notes, section "Block-sparse FlashAttention"): a
+ * predefined block mask M in {0,1}^{Tr x Tc}, Tr = ceil(N / Br) query blocks
+ * by Tc = ceil(N / Bc) key blocks, shared by every batch and head; key j is
+ * visible to query i only if M[i / Br][j / Bc] != 0.  Padding, causality and
+ * the block mask combine (a key must pass all of them).
+ *
  * Readings where the pages are silent:
  *   - scale is an explicit argument (the notes' formula omits it);
  *   - LSE is the natural log of sum_j exp(s_j), in scaled-logit units;
@@ -56,12 +63,12 @@ static double widen_bf16(uint16_t bits) {
  * of length N.  Keys 0..visible-1 are candidates; pad (NULL or [N]) removes
  * the padded ones.  Excluded keys get no score and probability 0. */
 static void one_row(const double* qi, const double* kh, const double* vh, int N, int d,
-                    double scale, int visible, const unsigned char* pad, double* s, double* p,
-                    double* oi, double* lse) {
+                    double scale, int visible, const unsigned char* pad, const unsigned char* brow,
+                    int bc, double* s, double* p, double* oi, double* lse) {
     double m = -INFINITY;
     int any = 0;
     for (int j = 0; j < visible; ++j) {
-        if (pad && pad[j]) continue;
+        if ((pad && pad[j]) || (brow && !brow[j / bc])) continue;
         double acc = 0.0;
         for (int t = 0; t < d; ++t) acc += qi[t] * kh[(size_t)j * d + t];
         s[j] = scale * acc;
@@ -75,7 +82,7 @@ static void one_row(const double* qi, const double* kh, const double* vh, int N,
     }
     double sum = 0.0;
     for (int j = 0; j < visible; ++j) {
-        p[j] = (pad && pad[j]) ? 0.0 : exp(s[j] - m);
+        p[j] = ((pad && pad[j]) || (brow && !brow[j / bc])) ? 0.0 : exp(s[j] - m);
         sum += p[j];
     }
     for (int j = 0; j < visible; ++j) p[j] /= sum;
@@ -89,8 +96,10 @@ static void one_row(const double* qi, const double* kh, const double* vh, int N,
 
 /* All selected rows of one head.  rows == NULL means every row 0..N-1. */
 static void one_head(const double* qh, const double* kh, const double* vh, int N, int d,
-                     double scale, int causal, const unsigned char* pad, const int32_t* rows,
+                     double scale, int causal, const unsigned char* pad,
+                     const unsigned char* block_mask, int br, int bc, const int32_t* rows,
                      int n_rows, double* o, double* lse, int n_threads) {
+    const int tc = bc > 0 ? (N + bc - 1) / bc : 0;
 #ifdef _OPENMP
 #pragma omp parallel num_threads(n_threads > 0 ? n_threads : omp_get_max_threads())
 #endif
@@ -103,7 +112,8 @@ static void one_head(const double* qh, const double* kh, const double* vh, int N
         for (int r = 0; r < n_rows; ++r) {
             int i = rows ? rows[r] : r;
             int visible = causal ? i + 1 : N;
-            one_row(qh + (size_t)i * d, kh, vh, N, d, scale, visible, pad, s, p,
+            const unsigned char* brow = block_mask ? block_mask + (size_t)(i / br) * tc : NULL;
+            one_row(qh + (size_t)i * d, kh, vh, N, d, scale, visible, pad, brow, bc, s, p,
                     o + (size_t)r * d, lse + r);
         }
         free(s);
@@ -126,19 +136,23 @@ static int args_ok(int B, int H, int N, int d, const int32_t* rows, int n_rows) 
 /*
  * fp64 inputs, layout [B, H, N, d] contiguous.
  * key_pad: NULL or [B, N] bytes, nonzero = padded key.
+ * block_mask: NULL or [ceil(N / br), ceil(N / bc)] bytes, nonzero = the
+ * (query block, key block) pair is computed; br, bc >= 1 when it is given.
  * rows: NULL (all rows, n_rows must equal N) or int32 [B*H, n_rows], the
  * query rows to evaluate for each head.  o: fp64 [B*H, n_rows, d];
  * lse: fp64 [B*H, n_rows].  Returns 0 on success, -1 on bad arguments.
  */
 int attn_oracle_f64(const double* q, const double* k, const double* v, int B, int H, int N,
                     int d, double scale, int causal, const unsigned char* key_pad,
-                    const int32_t* rows, int n_rows, double* o, double* lse, int n_threads) {
+                    const unsigned char* block_mask, int br, int bc, const int32_t* rows,
+                    int n_rows, double* o, double* lse, int n_threads) {
     if (!args_ok(B, H, N, d, rows, n_rows)) return -1;
+    if (block_mask && (br < 1 || bc < 1)) return -1;
     size_t head = (size_t)N * d;
     for (long bh = 0; bh < (long)B * H; ++bh) {
         const unsigned char* pad = key_pad ? key_pad + (size_t)(bh / H) * N : NULL;
-        one_head(q + bh * head, k + bh * head, v + bh * head, N, d, scale, causal, pad,
-                 rows ? rows + bh * n_rows : NULL, n_rows, o + (size_t)bh * n_rows * d,
+        one_head(q + bh * head, k + bh * head, v + bh * head, N, d, scale, causal, pad, block_mask,
+                 br, bc, rows ? rows + bh * n_rows : NULL, n_rows, o + (size_t)bh * n_rows * d,
                  lse + (size_t)bh * n_rows, n_threads);
     }
     return 0;
@@ -151,8 +165,10 @@ int attn_oracle_f64(const double* q, const double* k, const double* v, int B, in
  */
 int attn_oracle_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
                      int N, int d, double scale, int causal, const unsigned char* key_pad,
-                     const int32_t* rows, int n_rows, double* o, double* lse, int n_threads) {
+                     const unsigned char* block_mask, int br, int bc, const int32_t* rows,
+                     int n_rows, double* o, double* lse, int n_threads) {
     if (!args_ok(B, H, N, d, rows, n_rows)) return -1;
+    if (block_mask && (br < 1 || bc < 1)) return -1;
     size_t head = (size_t)N * d;
     double* qh = (double*)malloc(sizeof(double) * head);
     double* kh = (double*)malloc(sizeof(double) * head);
@@ -168,7 +184,8 @@ int attn_oracle_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
             vh[e] = widen_bf16(v[bh * head + e]);
         }
         const unsigned char* pad = key_pad ? key_pad + (size_t)(bh / H) * N : NULL;
-        one_head(qh, kh, vh, N, d, scale, causal, pad, rows ? rows + bh * n_rows : NULL, n_rows,
+        one_head(qh, kh, vh, N, d, scale, causal, pad, block_mask, br, bc,
+                 rows ? rows + bh * n_rows : NULL, n_rows,
                  o + (size_t)bh * n_rows * d, lse + (size_t)bh * n_rows, n_threads);
     }
     free(qh); free(kh); free(vh);

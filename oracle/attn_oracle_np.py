@@ -3,17 +3,22 @@
 Materialises S = scale * Q K^T, the row softmax P and O = P V for whole heads,
 exactly as the standard, non-tiled attention of "FlashAttention: Fast and
 Memory-Efficient Exact Attention with IO-Awareness" (wiki notes, sections
-"Problem setting" and "IO complexity analysis") does.  LSE is the natural
+"Problem setting" and "IO complexity analysis") does.  The block mask follows
+the same notes' section "Block-sparse FlashAttention": a key is visible only
+where the mask entry of its (query block, key block) pair is nonzero.  LSE is the natural
 log-sum-exp of each score row.  Causal means key j is visible to query i iff
 j <= i.
 """
 import numpy as np
 
 
-def attention_full(q, k, v, scale, causal=False, return_probs=False, key_pad=None):
+def attention_full(q, k, v, scale, causal=False, return_probs=False, key_pad=None, block_mask=None,
+                   block=(128, 128)):
     """q, k, v: float64 arrays [B, H, N, d]; key_pad: None or [B, N], nonzero =
-    padded key.  Returns (O [B,H,N,d], LSE [B,H,N]) and optionally P; a row
-    with no visible key has O = 0, LSE = -inf and P = 0."""
+    padded key; block_mask: None or [ceil(N / Br), ceil(N / Bc)], (Br, Bc) =
+    block, nonzero = that (query block, key block) pair is computed.  Returns (O [B,H,N,d],
+    LSE [B,H,N]) and optionally P; a row with no visible key has O = 0,
+    LSE = -inf and P = 0."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -24,6 +29,9 @@ def attention_full(q, k, v, scale, causal=False, return_probs=False, key_pad=Non
         visible &= np.tril(np.ones((n, n), dtype=bool))
     if key_pad is not None:
         visible &= ~np.asarray(key_pad, dtype=bool)[:, None, None, :]
+    if block_mask is not None:
+        br, bc = block
+        visible &= np.asarray(block_mask, dtype=bool)[(np.arange(n) // br)[:, None], (np.arange(n) // bc)[None, :]]
     s = np.where(visible, s, -np.inf)
     m = s.max(axis=-1, keepdims=True)
     empty = ~visible.any(axis=-1, keepdims=True)

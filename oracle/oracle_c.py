@@ -36,7 +36,8 @@ def _load():
             fn = getattr(lib, name)
             fn.restype = ctypes.c_int
             fn.argtypes = [ptr, ptr, ptr, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                           ctypes.c_double, ctypes.c_int, ptr, ptr, ctypes.c_int, ptr, ptr, ctypes.c_int]
+                           ctypes.c_double, ctypes.c_int, ptr, ptr, ctypes.c_int, ctypes.c_int, ptr,
+                           ctypes.c_int, ptr, ptr, ctypes.c_int]
         lib.attn_oracle_max_threads.restype = ctypes.c_int
         lib.attn_oracle_max_threads.argtypes = []
         _lib = lib
@@ -54,14 +55,17 @@ def _bf16_bits(t):
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def attention_rows(q, k, v, scale, causal=False, rows=None, n_threads=0, key_pad=None):
+def attention_rows(q, k, v, scale, causal=False, rows=None, n_threads=0, key_pad=None, block_mask=None,
+                   block=(128, 128)):
     """Evaluate the oracle on selected query rows.
 
     q, k, v: [B, H, N, d], either bf16 torch tensors (widened exactly) or
     float64 arrays.  rows: None (all rows) or an int array [B*H, R] (or [R],
     shared by every head) of query indices.  key_pad: None or a [B, N] array,
-    nonzero = padded key.  Returns (O [B*H, R, d], LSE [B*H, R]) as float64
-    numpy arrays; a row with no visible key has O = 0 and LSE = -inf.
+    nonzero = padded key.  block_mask: None or a [ceil(N / Br), ceil(N / Bc)]
+    array, (Br, Bc) = block, nonzero = that (query block, key block) pair is
+    computed.  Returns (O [B*H, R, d], LSE [B*H, R]) as float64 numpy arrays;
+    a row with no visible key has O = 0 and LSE = -inf.
     """
     lib = _load()
     try:
@@ -89,10 +93,19 @@ def attention_rows(q, k, v, scale, causal=False, rows=None, n_threads=0, key_pad
     if key_pad is not None:
         pad_a = np.ascontiguousarray(np.asarray(key_pad).astype(np.uint8).reshape(B, N))
         pad_p = pad_a.ctypes.data
+    bm_p = None
+    br, bc = (int(x) for x in block)
+    if block_mask is not None:
+        if br < 1 or bc < 1:
+            raise ValueError("block sizes must be >= 1")
+        tr, tc = (N + br - 1) // br, (N + bc - 1) // bc
+        bm_a = np.ascontiguousarray(np.asarray(block_mask).astype(np.uint8).reshape(tr, tc))
+        bm_p = bm_a.ctypes.data
     o = np.empty((B * H, n_rows, d), dtype=np.float64)
     lse = np.empty((B * H, n_rows), dtype=np.float64)
     rc = fn(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, B, H, N, d, float(scale),
-            int(bool(causal)), pad_p, rows_p, n_rows, o.ctypes.data, lse.ctypes.data, int(n_threads))
+            int(bool(causal)), pad_p, bm_p, br, bc, rows_p, n_rows, o.ctypes.data, lse.ctypes.data,
+            int(n_threads))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (code %d)" % rc)
     return o, lse

@@ -330,3 +330,106 @@ def test_masked_c_oracle_matches_numpy_twin(causal):
     np.testing.assert_array_equal(np.isneginf(lse.reshape(lse_np.shape)), np.isneginf(lse_np))
     fin = np.isfinite(lse_np)
     np.testing.assert_allclose(lse.reshape(lse_np.shape)[fin], lse_np[fin], rtol=0, atol=1e-12)
+
+
+# ---- block-sparse mask (FlashAttention: Fast and Memory-Efficient Exact
+# Attention with IO-Awareness, wiki notes, section "Block-sparse
+# FlashAttention": M in {0,1}^{N/Br x N/Bc}, only the non-zero blocks count)
+
+def test_all_ones_block_mask_is_dense_attention():
+    q, k, v = (RNG.normal(size=(2, 2, 37, 5)) for _ in range(3))
+    for causal in (False, True):
+        o, lse = oracle.attention_rows(q, k, v, 0.4, causal)
+        ones = np.ones((5, 3), dtype=np.uint8)             # Br = 8, Bc = 16 on N = 37
+        ob, lb = oracle.attention_rows(q, k, v, 0.4, causal, block_mask=ones, block=(8, 16))
+        np.testing.assert_array_equal(ob, o)
+        np.testing.assert_array_equal(lb, lse)
+
+
+def test_unit_blocks_lower_triangle_is_the_causal_mask():
+    # causal attention is the block-sparse case Br = Bc = 1, M lower triangular
+    N = 23
+    q, k, v = (RNG.normal(size=(1, 3, N, 4)) for _ in range(3))
+    tri = np.tril(np.ones((N, N), dtype=np.uint8))
+    o, lse = oracle.attention_rows(q, k, v, 0.6, False, block_mask=tri, block=(1, 1))
+    oc, lc = oracle.attention_rows(q, k, v, 0.6, True)
+    np.testing.assert_array_equal(o, oc)
+    np.testing.assert_array_equal(lse, lc)
+    # and the 40-digit decimal evaluation of the causal formula agrees
+    o_ref, l_ref = _decimal_attention(q[0, 1], k[0, 1], v[0, 1], 0.6, True)
+    np.testing.assert_allclose(o.reshape(1, 3, N, 4)[0, 1], o_ref, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse.reshape(1, 3, N)[0, 1], l_ref, rtol=0, atol=1e-13)
+
+
+def test_permutation_block_mask_is_attention_over_one_key_block():
+    # query block r sees only key block c(r): each row is plain attention over
+    # that block's keys.  A transposed mask or swapped block sizes fail this.
+    Br, Bc, N, d = 6, 4, 22, 3                 # Tr = 4 query blocks, Tc = 6 key blocks (last one ragged)
+    q, k, v = (RNG.normal(size=(1, 2, N, d)) for _ in range(3))
+    target = [5, 0, 3, 1]
+    M = np.zeros((4, 6), dtype=np.uint8)
+    for r, c in enumerate(target):
+        M[r, c] = 1
+    o, lse = oracle.attention_rows(q, k, v, 0.9, block_mask=M, block=(Br, Bc))
+    o, lse = o.reshape(1, 2, N, d), lse.reshape(1, 2, N)
+    for i in range(N):
+        c = target[i // Br]
+        ks = slice(c * Bc, min(N, (c + 1) * Bc))
+        o1, l1 = oracle.attention_full(q[:, :, i:i + 1], k[:, :, ks], v[:, :, ks], 0.9)
+        np.testing.assert_allclose(o[:, :, i], o1[:, :, 0], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, i], l1[:, :, 0], rtol=0, atol=1e-13)
+
+
+def test_block_diagonal_mask_splits_the_sequence():
+    # a block-diagonal mask is independent attention on each segment
+    N, blk = 30, 10
+    q, k, v = (RNG.normal(size=(2, 1, N, 4)) for _ in range(3))
+    M = np.eye(3, dtype=np.uint8)
+    o, lse = oracle.attention_rows(q, k, v, 0.5, block_mask=M, block=(blk, blk))
+    o, lse = o.reshape(2, 1, N, 4), lse.reshape(2, 1, N)
+    for s in range(3):
+        seg = slice(s * blk, (s + 1) * blk)
+        o1, l1 = oracle.attention_full(q[:, :, seg], k[:, :, seg], v[:, :, seg], 0.5)
+        np.testing.assert_allclose(o[:, :, seg], o1, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, seg], l1, rtol=0, atol=1e-13)
+
+
+def test_query_blocks_with_no_key_block_are_empty():
+    N = 20
+    q, k, v = (RNG.normal(size=(1, 2, N, 3)) for _ in range(3))
+    M = np.ones((3, 3), dtype=np.uint8)        # Br = Bc = 8
+    M[1, :] = 0                                # rows 8..15 see nothing
+    o, lse = oracle.attention_rows(q, k, v, 0.5, block_mask=M, block=(8, 8))
+    o, lse = o.reshape(1, 2, N, 3), lse.reshape(1, 2, N)
+    assert (o[:, :, 8:16] == 0).all() and np.isneginf(lse[:, :, 8:16]).all()
+    assert np.isfinite(lse[:, :, :8]).all() and np.isfinite(lse[:, :, 16:]).all()
+    # causal + block mask: row block 0 allowed only key block 2 (above the diagonal)
+    M2 = np.ones((3, 3), dtype=np.uint8)
+    M2[0, :2] = 0
+    o2, l2 = oracle.attention_rows(q, k, v, 0.5, True, block_mask=M2, block=(8, 8))
+    o2, l2 = o2.reshape(1, 2, N, 3), l2.reshape(1, 2, N)
+    assert (o2[:, :, :8] == 0).all() and np.isneginf(l2[:, :, :8]).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_sparse_c_oracle_matches_numpy_twin(causal):
+    N = 300
+    q, k, v = make_qkv(1, 2, N, 16, seed=17)
+    rng = np.random.default_rng(7)
+    M = (rng.random((3, 3)) < 0.6).astype(np.uint8)   # Br = Bc = 128
+    M[2, :] = 0
+    pad = (rng.random((1, N)) < 0.2).astype(np.uint8)
+    o, lse = oracle.attention_rows(q, k, v, 0.25, causal, key_pad=pad, block_mask=M)
+    qd, kd, vd = (x.double().numpy() for x in (q, k, v))
+    o_np, lse_np = oracle.attention_full(qd, kd, vd, 0.25, causal, key_pad=pad, block_mask=M)
+    np.testing.assert_allclose(o.reshape(o_np.shape), o_np, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(np.isneginf(lse.reshape(lse_np.shape)), np.isneginf(lse_np))
+    fin = np.isfinite(lse_np)
+    np.testing.assert_allclose(lse.reshape(lse_np.shape)[fin], lse_np[fin], rtol=0, atol=1e-12)
+    assert np.isneginf(lse_np[..., 256:]).all()
+
+
+def test_oracle_rejects_bad_block_sizes():
+    q = np.zeros((1, 1, 4, 2))
+    with pytest.raises(ValueError):
+        oracle.attention_rows(q, q, q, 1.0, block_mask=np.ones((4, 4)), block=(0, 1))
