@@ -6,7 +6,7 @@ supplies device memory and the current stream.  There is no fallback: if the
 library is missing, every entry point raises.
 
 The C entry points keep their names here (``attn_fwd``, ``attn_fwd_strided``,
-``attn_status_string``, ``attn_check_device_status``,
+``attn_fwd_block_sparse``, ``attn_status_string``, ``attn_check_device_status``,
 ``attn_selftest_wait_timeout``, ``attn_version``); ``forward`` is the tensor
 convenience wrapper.
 """
@@ -15,7 +15,7 @@ import math
 import os
 
 __all__ = [
-    "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_fwd_strided", "attn_status_string", "attn_check_device_status",
+    "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_status_string", "attn_check_device_status",
     "attn_selftest_wait_timeout", "attn_version", "forward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
 ]
@@ -50,6 +50,9 @@ def library():
         lib.attn_fwd_strided.restype = i32
         lib.attn_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i64, i64, i64, i64, i64,
                                          vp, ctypes.c_float, i32, vp]
+        lib.attn_fwd_block_sparse.restype = i32
+        lib.attn_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i64, i64, i64, i64,
+                                              i64, vp, vp, ctypes.c_float, i32, vp]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_status_string.argtypes = [i32]
         lib.attn_check_device_status.restype = i32
@@ -78,6 +81,17 @@ def attn_fwd_strided(q, k, v, o, lse, B, H, N, d, qkv_strides, o_strides, scale,
                                       key_padding_mask, float(scale), int(bool(causal)), stream)
 
 
+def attn_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, qkv_strides, o_strides, scale, causal, stream,
+                          key_padding_mask=None, block_mask=None):
+    """Raw C call: attn_fwd_strided plus the device address of a
+    [ceil(N/128), ceil(N/128)] byte block mask (nonzero = block computed)."""
+    sb, sh, sn = (int(x) for x in qkv_strides)
+    ob, oh, on = (int(x) for x in o_strides)
+    return library().attn_fwd_block_sparse(q, k, v, o, lse, int(B), int(H), int(N), int(d), sb, sh, sn, ob, oh,
+                                           on, key_padding_mask, block_mask, float(scale), int(bool(causal)),
+                                           stream)
+
+
 def attn_status_string(status):
     return library().attn_status_string(int(status)).decode()
 
@@ -104,7 +118,11 @@ def _stream_handle(stream):
     return stream.cuda_stream
 
 
-def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None, key_padding_mask=None):
+BLOCK = 128  # query rows / keys per block of the block-sparse mask
+
+
+def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None, key_padding_mask=None,
+            block_mask=None):
     """Exact attention forward on bf16 CUDA tensors [B, H, N, d] (d = 64 or 128).
 
     q, k and v may be strided views (for example of one packed projection
@@ -115,7 +133,11 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None, 
     ``scale`` defaults to 1/sqrt(d).  ``key_padding_mask``: None or a bool /
     uint8 CUDA tensor [B, N], True (nonzero) = padded key, excluded from every
     query row of that batch; a row with no visible key gets O = 0 and LSE =
-    -inf.  The call is asynchronous on ``stream`` (default: the current stream).
+    -inf.  ``block_mask``: None or a bool / uint8 CUDA tensor [T, T], T =
+    ceil(N / 128), contiguous and 16-byte aligned: entry (r, c) nonzero lets
+    query rows [128 r, 128 r + 128) see keys [128 c, 128 c + 128), for every
+    batch and head; only those blocks are computed.  The call is asynchronous
+    on ``stream`` (default: the current stream).
     """
     import torch
     if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
@@ -142,13 +164,27 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None, 
                 or not key_padding_mask.is_cuda or not key_padding_mask.is_contiguous()):
             raise ValueError("key_padding_mask must be a contiguous bool/uint8 CUDA tensor [B, N]")
         pad_ptr = key_padding_mask.data_ptr()
+    bm_ptr = None
+    if block_mask is not None:
+        T = (N + BLOCK - 1) // BLOCK
+        if (block_mask.shape != (T, T) or block_mask.dtype not in (torch.bool, torch.uint8)
+                or not block_mask.is_cuda or not block_mask.is_contiguous()):
+            raise ValueError("block_mask must be a contiguous bool/uint8 CUDA tensor [ceil(N/128), ceil(N/128)]")
+        bm_ptr = block_mask.data_ptr()
     # the stride of a size-1 dimension is never used: give it the contiguous value
     def strides(t):
         dense = (H * N * d, N * d, d)
         return [st if n > 1 else c for n, st, c in zip(t.shape[:3], t.stride()[:3], dense)]
-    status = attn_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                              B, H, N, d, strides(q), strides(out), scale, causal, _stream_handle(stream),
-                              key_padding_mask=pad_ptr)
+    if bm_ptr is None:
+        status = attn_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  B, H, N, d, strides(q), strides(out), scale, causal, _stream_handle(stream),
+                                  key_padding_mask=pad_ptr)
+        what = "attn_fwd_strided"
+    else:
+        status = attn_fwd_block_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                       B, H, N, d, strides(q), strides(out), scale, causal,
+                                       _stream_handle(stream), key_padding_mask=pad_ptr, block_mask=bm_ptr)
+        what = "attn_fwd_block_sparse"
     if status != ATTN_OK:
-        raise AttnError(status, "attn_fwd_strided")
+        raise AttnError(status, what)
     return out, lse

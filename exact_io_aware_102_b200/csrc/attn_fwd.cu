@@ -95,6 +95,7 @@ struct Cfg {
     static constexpr int kRingOff = 2 * kTileBytes;
     static constexpr int kVRingOff = kRingOff + kKSlots * kTileBytes;
     static constexpr int kBarOff = kVRingOff + kVSlots * kTileBytes;
+    static constexpr int kMaskOff = kBarOff + 512;             // sparse mode: block mask bits
     static constexpr int kSmemBytes = kBarOff + 512 + 1024;   // barriers + 1 KB alignment slack
     static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
     static constexpr uint32_t kColP0 = kSplit ? 256 + 2 * D : kColS0;
@@ -386,29 +387,36 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool b_mn_ma
 }
 
 // ------------------------------------------------------------- the scheduler
+// Which key tiles a work unit visits.  Full: all of them.  Causal: a Q tile
+// stops at the key tile holding its last row (tiles above the diagonal are
+// never loaded or multiplied).  Sparse: the non-zero entries of the block mask
+// row of each Q tile (with the causal bound as well when causal is set).
+enum : int { kModeFull = 0, kModeCausal = 1, kModeSparse = 2 };
+
 struct Params {
     int BH, H, N, n_pairs, n_kv_all, total_units;
     long long o_sb, o_sh, o_sn;  // element strides of O over (batch, head, row)
     const uint8_t* key_pad;      // [B, N] key-padding mask (nonzero = padded) or null
     int pad_vec;                 // key_pad rows may be read 16 bytes at a time
+    const uint8_t* block_mask;   // [n_kv_all, n_kv_all] block mask (nonzero = computed), sparse mode
+    int causal;                  // causal bound on top of the block mask (sparse mode)
     float scale_log2;  // scale * log2(e)
     unsigned long long wait_ns;
 };
 
 struct Unit {
-    int bh, b, h, q0, n0, n1;  // head (flat, batch, within batch), first query row, key tiles for Q tile 0 / 1
+    int bh, b, h, q0;  // head (flat, batch, within batch), first query row
 };
 
 // Work units: (head, pair of Q tiles).  Non-causal: heads-major so the CTAs
 // running at one time share K/V of few heads (L2 reuse).  Causal: the pairs
-// with the most key tiles first, so the short units fill the tail; a Q tile
-// stops at the key tile holding its last row (tiles above the diagonal are
-// never loaded or multiplied).
-template <bool CAUSAL>
+// with the most key tiles first, so the short units fill the tail.
+template <int MODE>
 __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     Unit w;
     int pair;
-    if (CAUSAL) {
+    const bool longest_first = MODE == kModeCausal || (MODE == kModeSparse && p.causal);
+    if (longest_first) {
         pair = p.n_pairs - 1 - u / p.BH;
         w.bh = u % p.BH;
     } else {
@@ -418,13 +426,110 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     w.b = w.bh / p.H;
     w.h = w.bh - w.b * p.H;
     w.q0 = pair * kUnitRows;
-    if (CAUSAL) {
-        w.n1 = min(p.n_kv_all, (w.q0 + kUnitRows) / kBlockN);  // tiles touching rows < q0 + 256
-        w.n0 = min(w.n1, w.q0 / kBlockN + 1);                 // tiles touching rows < q0 + 128
-    } else {
-        w.n0 = w.n1 = p.n_kv_all;
-    }
     return w;
+}
+
+constexpr int kNoTile = 0x7fffffff;
+
+// The key tiles one Q tile visits, in increasing order.
+template <int MODE>
+struct KeyTiles {
+    int lim;               // last key tile it may visit (-1: the tile has no rows)
+    int off;               // sparse: bit index of its mask row, column 0
+    const uint32_t* bits;  // sparse: the block mask as bits, row-major, in shared memory
+
+    __device__ __forceinline__ bool has(int j) const {
+        if constexpr (MODE != kModeSparse) return j <= lim;
+        else return j <= lim && ((bits[(off + j) >> 5] >> ((off + j) & 31)) & 1u);
+    }
+    // first key tile >= j (kNoTile if none)
+    __device__ __forceinline__ int next(int j) const {
+        if constexpr (MODE != kModeSparse) {
+            return j <= lim ? j : kNoTile;
+        } else {
+            while (j <= lim) {
+                const int f = off + j;
+                const uint32_t word = bits[f >> 5] >> (f & 31);
+                if (word != 0u) {
+                    const int jj = j + __ffs(static_cast<int>(word)) - 1;
+                    return jj <= lim ? jj : kNoTile;
+                }
+                j += 32 - (f & 31);
+            }
+            return kNoTile;
+        }
+    }
+    // number of key tiles
+    __device__ __forceinline__ int count() const {
+        if constexpr (MODE != kModeSparse) {
+            return lim + 1;
+        } else {
+            if (lim < 0) return 0;
+            const int f = off, e = off + lim;  // first and last bit, inclusive
+            int n = 0;
+            for (int wd = f >> 5; wd <= (e >> 5); ++wd) {
+                uint32_t x = bits[wd];
+                if (wd == (f >> 5)) x &= ~0u << (f & 31);
+                if (wd == (e >> 5)) x &= ~0u >> (31 - (e & 31));
+                n += __popc(x);
+            }
+            return n;
+        }
+    }
+    // last key tile (-1 if none)
+    __device__ __forceinline__ int last() const {
+        if constexpr (MODE != kModeSparse) {
+            return lim;
+        } else {
+            int j = lim;
+            while (j >= 0) {
+                const int f = off + j;
+                const uint32_t word = bits[f >> 5] << (31 - (f & 31));
+                if (word != 0u) {
+                    const int jj = j - __clz(static_cast<int>(word));
+                    return jj >= 0 ? jj : -1;
+                }
+                j -= (f & 31) + 1;
+            }
+            return -1;
+        }
+    }
+};
+
+template <int MODE>
+__device__ __forceinline__ KeyTiles<MODE> key_tiles(const Unit& w, const Params& p, const uint32_t* bits, int t) {
+    const bool causal = MODE == kModeCausal || (MODE == kModeSparse && p.causal);
+    const int qt = w.q0 / kBlockM + t;
+    KeyTiles<MODE> k;
+    // full and causal modes also walk Q tile 1 of the last unit when it has no
+    // rows (nothing of it is stored); the sparse mode skips it
+    k.lim = (MODE == kModeSparse && w.q0 + t * kBlockM >= p.N) ? -1
+            : causal ? min(p.n_kv_all - 1, qt) : p.n_kv_all - 1;
+    k.off = qt * p.n_kv_all;
+    k.bits = bits;
+    return k;
+}
+
+// The key tiles of one unit, as the load and MMA roles walk them: the union
+// over the two Q tiles in increasing order; Q tile t takes part in tile j iff
+// q[t].has(j).  Every role derives the same tiles from the same unit, so
+// their barrier counts agree.
+template <int MODE>
+struct Plan {
+    KeyTiles<MODE> q[2];
+    __device__ __forceinline__ bool need(int t, int j) const { return q[t].has(j); }
+    __device__ __forceinline__ int next(int j) const {
+        if constexpr (MODE != kModeSparse) return j <= max(q[0].lim, q[1].lim) ? j : kNoTile;
+        else return min(q[0].next(j), q[1].next(j));
+    }
+};
+
+template <int MODE>
+__device__ __forceinline__ Plan<MODE> make_plan(const Unit& w, const Params& p, const uint32_t* bits) {
+    Plan<MODE> pl;
+    pl.q[0] = key_tiles<MODE>(w, p, bits, 0);
+    pl.q[1] = key_tiles<MODE>(w, p, bits, 1);
+    return pl;
 }
 
 // What every role of one CTA shares.
@@ -433,6 +538,7 @@ struct Ctx {
     uint32_t bar;    // barrier block
     uint32_t tmem;   // TMEM base address
     volatile uint32_t* abort_flag;
+    const uint32_t* mask_bits;  // sparse mode: staged block mask bits
     Params p;
 };
 
@@ -444,57 +550,112 @@ struct Ring {
 };
 
 // ------------------------------------------------------------ TMA producer
-// Per unit: Q0, Q1 once; then the key tiles in the order the MMA warps use
-// them (split: K_j into the K ring and V_j into the V ring; shared ring:
-// K_j then V_j).
-template <int D, bool CAUSAL>
+// Per unit with at least one key tile: Q0, Q1 once; then the key tiles in
+// the order the MMA warps use them (split: K_j into the K ring and V_j into
+// the V ring; shared ring: K_j then V_j).
+template <int D, int MODE>
 __device__ __forceinline__ void role_producer(const Ctx& c, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                               const CUtensorMap* tm_v) {
-    using C = Cfg<D>;
-    Ring rk{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
-    Ring rv{c.base + C::kVRingOff, c.bar + Bars::kVFull, c.bar + Bars::kVEmpty, (uint32_t)C::kVSlots, 0};
-    uint32_t q_issued = 0;
-    bool ok = true;
-    auto load = [&](Ring& r, const CUtensorMap* map, int key0, const Unit& w) {
-        const uint32_t s = r.slot();
-        if (!wait_bounded(r.empty + 8 * s, r.phase() ^ 1u, c.abort_flag, c.p.wait_ns)) return false;
-        const uint32_t fb = r.full + 8 * s;
-        const uint32_t dst = r.smem + s * C::kTileBytes;
-        mbar_expect_tx(fb, C::kTileBytes);
+    if constexpr (MODE != kModeSparse) {
+        // full / causal: key tiles [0, n1) of every unit
+        using C = Cfg<D>;
+        Ring rk{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
+        Ring rv{c.base + C::kVRingOff, c.bar + Bars::kVFull, c.bar + Bars::kVEmpty, (uint32_t)C::kVSlots, 0};
+        uint32_t q_issued = 0;
+        bool ok = true;
+        auto load = [&](Ring& r, const CUtensorMap* map, int key0, const Unit& w) {
+            const uint32_t s = r.slot();
+            if (!wait_bounded(r.empty + 8 * s, r.phase() ^ 1u, c.abort_flag, c.p.wait_ns)) return false;
+            const uint32_t fb = r.full + 8 * s;
+            const uint32_t dst = r.smem + s * C::kTileBytes;
+            mbar_expect_tx(fb, C::kTileBytes);
 #pragma unroll
-        for (int x = 0; x < D / 64; ++x) tma_load_4d(dst + x * C::kHalfBytes, map, fb, x * 64, key0, w.h, w.b);
-        ++r.i;
-        return true;
-    };
-    int local = 0;
-    for (int u = blockIdx.x; ok && u < c.p.total_units; u += gridDim.x, ++local) {
-        const Unit w = decode_unit<CAUSAL>(u, c.p);
-        if (!wait_bounded(c.bar + Bars::kQEmpty, (local & 1) ^ 1, c.abort_flag, c.p.wait_ns)) {
-            ok = false;
-            break;
-        }
-        for (int t = 0; t < 2; ++t) {
-            const uint32_t qb = c.bar + Bars::kQFull + 8 * t;
-            const uint32_t dst = c.base + C::kQOff + t * C::kTileBytes;
-            mbar_expect_tx(qb, C::kTileBytes);
+            for (int x = 0; x < D / 64; ++x) tma_load_4d(dst + x * C::kHalfBytes, map, fb, x * 64, key0, w.h, w.b);
+            ++r.i;
+            return true;
+        };
+        int local = 0;
+        for (int u = blockIdx.x; ok && u < c.p.total_units; u += gridDim.x, ++local) {
+            const Unit w = decode_unit<MODE>(u, c.p);
+            const int n1 = make_plan<MODE>(w, c.p, c.mask_bits).q[1].lim + 1;
+            if (!wait_bounded(c.bar + Bars::kQEmpty, (local & 1) ^ 1, c.abort_flag, c.p.wait_ns)) {
+                ok = false;
+                break;
+            }
+            for (int t = 0; t < 2; ++t) {
+                const uint32_t qb = c.bar + Bars::kQFull + 8 * t;
+                const uint32_t dst = c.base + C::kQOff + t * C::kTileBytes;
+                mbar_expect_tx(qb, C::kTileBytes);
 #pragma unroll
-            for (int x = 0; x < D / 64; ++x)
-                tma_load_4d(dst + x * C::kHalfBytes, tm_q, qb, x * 64, w.q0 + t * kBlockM, w.h, w.b);
+                for (int x = 0; x < D / 64; ++x)
+                    tma_load_4d(dst + x * C::kHalfBytes, tm_q, qb, x * 64, w.q0 + t * kBlockM, w.h, w.b);
+            }
+            q_issued = local + 1;
+            for (int j = 0; ok && j < n1; ++j) {
+                ok = load(rk, tm_k, j * kBlockN, w);
+                if (ok) ok = load(C::kSplit ? rv : rk, tm_v, j * kBlockN, w);
+            }
         }
-        q_issued = local + 1;
-        for (int j = 0; ok && j < w.n1; ++j) {
-            ok = load(rk, tm_k, j * kBlockN, w);
-            if (ok) ok = load(C::kSplit ? rv : rk, tm_v, j * kBlockN, w);
+        if (!ok) {
+            // Drain: every issued copy lands before the CTA may exit.
+            for (Ring* r : {&rk, &rv})
+                for (uint32_t i = (r->i > r->slots ? r->i - r->slots : 0); i < r->i; ++i)
+                    wait_bounded(r->full + 8 * (i % r->slots), (i / r->slots) & 1, nullptr, kDrainWaitNs);
+            if (q_issued > 0)
+                for (int t = 0; t < 2; ++t)
+                    wait_bounded(c.bar + Bars::kQFull + 8 * t, (q_issued - 1) & 1, nullptr, kDrainWaitNs);
         }
-    }
-    if (!ok) {
-        // Drain: every issued copy lands before the CTA may exit.
-        for (Ring* r : {&rk, &rv})
-            for (uint32_t i = (r->i > r->slots ? r->i - r->slots : 0); i < r->i; ++i)
-                wait_bounded(r->full + 8 * (i % r->slots), (i / r->slots) & 1, nullptr, kDrainWaitNs);
-        if (q_issued > 0)
-            for (int t = 0; t < 2; ++t)
-                wait_bounded(c.bar + Bars::kQFull + 8 * t, (q_issued - 1) & 1, nullptr, kDrainWaitNs);
+    } else {
+        // sparse: the union of both Q tiles' key tiles; units without any are skipped
+        using C = Cfg<D>;
+        Ring rk{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
+        Ring rv{c.base + C::kVRingOff, c.bar + Bars::kVFull, c.bar + Bars::kVEmpty, (uint32_t)C::kVSlots, 0};
+        uint32_t q_issued = 0;  // units whose Q tiles were loaded
+        bool ok = true;
+        auto load = [&](Ring& r, const CUtensorMap* map, int key0, const Unit& w) {
+            const uint32_t s = r.slot();
+            if (!wait_bounded(r.empty + 8 * s, r.phase() ^ 1u, c.abort_flag, c.p.wait_ns)) return false;
+            const uint32_t fb = r.full + 8 * s;
+            const uint32_t dst = r.smem + s * C::kTileBytes;
+            mbar_expect_tx(fb, C::kTileBytes);
+#pragma unroll
+            for (int x = 0; x < D / 64; ++x) tma_load_4d(dst + x * C::kHalfBytes, map, fb, x * 64, key0, w.h, w.b);
+            ++r.i;
+            return true;
+        };
+        for (int u = blockIdx.x; ok && u < c.p.total_units; u += gridDim.x) {
+            const Unit w = decode_unit<MODE>(u, c.p);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            int j = pl.next(0);
+            if (j == kNoTile) continue;
+            if (!wait_bounded(c.bar + Bars::kQEmpty, (q_issued & 1) ^ 1, c.abort_flag, c.p.wait_ns)) {
+                ok = false;
+                break;
+            }
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const uint32_t qb = c.bar + Bars::kQFull + 8 * t;
+                const uint32_t dst = c.base + C::kQOff + t * C::kTileBytes;
+                mbar_expect_tx(qb, C::kTileBytes);
+#pragma unroll
+                for (int x = 0; x < D / 64; ++x)
+                    tma_load_4d(dst + x * C::kHalfBytes, tm_q, qb, x * 64, w.q0 + t * kBlockM, w.h, w.b);
+            }
+            ++q_issued;
+            for (; ok && j != kNoTile; j = pl.next(j + 1)) {
+                ok = load(rk, tm_k, j * kBlockN, w);
+                if (ok) ok = load(C::kSplit ? rv : rk, tm_v, j * kBlockN, w);
+            }
+        }
+        if (!ok) {
+            // Drain: every issued copy lands before the CTA may exit.
+            for (Ring* r : {&rk, &rv})
+                for (uint32_t i = (r->i > r->slots ? r->i - r->slots : 0); i < r->i; ++i)
+                    wait_bounded(r->full + 8 * (i % r->slots), (i / r->slots) & 1, nullptr, kDrainWaitNs);
+            if (q_issued > 0)
+                for (int t = 0; t < 2; ++t)
+                    wait_bounded(c.bar + Bars::kQFull + 8 * t, (q_issued - 1) & 1, nullptr, kDrainWaitNs);
+        }
     }
 }
 
@@ -548,130 +709,281 @@ __device__ __forceinline__ void mma_drain(const Ctx& c, int which) {
     wait_bounded(c.bar + Bars::kDrain + 8 * which, 0, nullptr, kDrainWaitNs);
 }
 
-// Split layout, S stream: S_t(j) once the softmax has loaded S_t(j-1).
-template <int D, bool CAUSAL>
+// Split layout, S stream: S_t(j) once the softmax has loaded S_t's previous tile.
+template <int D, int MODE>
 __device__ __forceinline__ void role_mma_s(const Ctx& c) {
-    using C = Cfg<D>;
-    Ring rk{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
-    Waiter wait{c, true};
-    uint32_t s_issued[2] = {0u, 0u};
-    int local = 0;
-    for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
-        const Unit w = decode_unit<CAUSAL>(u, c.p);
-        if (!wait(c.bar + Bars::kQFull + 0, local & 1) || !wait(c.bar + Bars::kQFull + 8, local & 1)) break;
-        for (int j = 0; j < w.n1; ++j) {
-            uint32_t ks;
-            if (!wait.take(rk, ks)) break;
-            for (int t = 0; t < 2; ++t) {
-                if (t == 0 && j >= w.n0) continue;
-                if (s_issued[t] > 0 && !wait(c.bar + Bars::kSFree + 8 * t, (s_issued[t] - 1) & 1)) break;
-                tc_fence_after();
-                Mma<D>::qk(c, t, rk.smem + ks * C::kTileBytes);
-                tc_commit(c.bar + Bars::kSFull + 8 * t);
-                ++s_issued[t];
+    if constexpr (MODE != kModeSparse) {
+        // full / causal: Q tile 0 visits key tiles [0, n0), Q tile 1 [0, n1), n0 <= n1
+        using C = Cfg<D>;
+        Ring rk{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
+        Waiter wait{c, true};
+        uint32_t s_issued[2] = {0u, 0u};
+        int local = 0;
+        for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
+            const Unit w = decode_unit<MODE>(u, c.p);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const int n0 = pl.q[0].lim + 1, n1 = pl.q[1].lim + 1;
+            if (!wait(c.bar + Bars::kQFull + 0, local & 1) || !wait(c.bar + Bars::kQFull + 8, local & 1)) break;
+            for (int j = 0; j < n1; ++j) {
+                uint32_t ks;
+                if (!wait.take(rk, ks)) break;
+                for (int t = 0; t < 2; ++t) {
+                    if (t == 0 && j >= n0) continue;
+                    if (s_issued[t] > 0 && !wait(c.bar + Bars::kSFree + 8 * t, (s_issued[t] - 1) & 1)) break;
+                    tc_fence_after();
+                    Mma<D>::qk(c, t, rk.smem + ks * C::kTileBytes);
+                    tc_commit(c.bar + Bars::kSFull + 8 * t);
+                    ++s_issued[t];
+                }
+                if (!wait.ok) break;
+                if (j + 1 == n1) tc_commit(c.bar + Bars::kQEmpty);
+                tc_commit(rk.empty + 8 * ks);
             }
-            if (!wait.ok) break;
-            if (j + 1 == w.n1) tc_commit(c.bar + Bars::kQEmpty);
-            tc_commit(rk.empty + 8 * ks);
         }
+        if (!wait.ok) mma_drain(c, 0);
+    } else {
+        // sparse: the union of both Q tiles' key tiles
+        using C = Cfg<D>;
+        Ring rk{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
+        Waiter wait{c, true};
+        uint32_t s_issued[2] = {0u, 0u};
+        uint32_t q_units = 0;
+        for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x) {
+            const Unit w = decode_unit<MODE>(u, c.p);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            int j = pl.next(0);
+            if (j == kNoTile) continue;
+            if (!wait(c.bar + Bars::kQFull + 0, q_units & 1) || !wait(c.bar + Bars::kQFull + 8, q_units & 1)) break;
+            ++q_units;
+            while (j != kNoTile) {
+                uint32_t ks;
+                if (!wait.take(rk, ks)) break;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (!pl.need(t, j)) continue;
+                    if (s_issued[t] > 0 && !wait(c.bar + Bars::kSFree + 8 * t, (s_issued[t] - 1) & 1)) break;
+                    tc_fence_after();
+                    Mma<D>::qk(c, t, rk.smem + ks * C::kTileBytes);
+                    tc_commit(c.bar + Bars::kSFull + 8 * t);
+                    ++s_issued[t];
+                }
+                if (!wait.ok) break;
+                j = pl.next(j + 1);
+                if (j == kNoTile) tc_commit(c.bar + Bars::kQEmpty);
+                tc_commit(rk.empty + 8 * ks);
+            }
+        }
+        if (!wait.ok) mma_drain(c, 0);
     }
-    if (!wait.ok) mma_drain(c, 0);
 }
 
-// Split layout, P V stream: O_t += P_t(j) V_j once the softmax has written P_t(j).
-template <int D, bool CAUSAL>
+// Split layout, P V stream: O_t (+)= P_t(j) V_j once the softmax has written P_t(j).
+template <int D, int MODE>
 __device__ __forceinline__ void role_mma_pv(const Ctx& c) {
-    using C = Cfg<D>;
-    Ring rv{c.base + C::kVRingOff, c.bar + Bars::kVFull, c.bar + Bars::kVEmpty, (uint32_t)C::kVSlots, 0};
-    Waiter wait{c, true};
-    uint32_t p_phase[2] = {0u, 0u};
-    int local = 0;
-    for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
-        const Unit w = decode_unit<CAUSAL>(u, c.p);
-        for (int j = 0; j < w.n1; ++j) {
-            uint32_t vs;
-            if (!wait.take(rv, vs)) break;
-            for (int t = 0; t < 2; ++t) {
-                const int n = t == 0 ? w.n0 : w.n1;
-                if (j >= n) continue;
-                if (!wait(c.bar + Bars::kPFull + 8 * t, p_phase[t])) break;
-                p_phase[t] ^= 1u;
-                if (j == 0 && !wait(c.bar + Bars::kOEmpty + 8 * t, (local & 1) ^ 1)) break;
-                tc_fence_after();
-                Mma<D>::pv(c, t, rv.smem + vs * C::kTileBytes, j > 0);
-                tc_commit(c.bar + Bars::kPFree + 8 * t);
-                if (j + 1 == n) tc_commit(c.bar + Bars::kOFull + 8 * t);
+    if constexpr (MODE != kModeSparse) {
+        // full / causal: Q tile 0 visits key tiles [0, n0), Q tile 1 [0, n1), n0 <= n1
+        using C = Cfg<D>;
+        Ring rv{c.base + C::kVRingOff, c.bar + Bars::kVFull, c.bar + Bars::kVEmpty, (uint32_t)C::kVSlots, 0};
+        Waiter wait{c, true};
+        uint32_t p_phase[2] = {0u, 0u};
+        int local = 0;
+        for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
+            const Unit w = decode_unit<MODE>(u, c.p);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const int n0 = pl.q[0].lim + 1, n1 = pl.q[1].lim + 1;
+            for (int j = 0; j < n1; ++j) {
+                uint32_t vs;
+                if (!wait.take(rv, vs)) break;
+                for (int t = 0; t < 2; ++t) {
+                    const int n = t == 0 ? n0 : n1;
+                    if (j >= n) continue;
+                    if (!wait(c.bar + Bars::kPFull + 8 * t, p_phase[t])) break;
+                    p_phase[t] ^= 1u;
+                    if (j == 0 && !wait(c.bar + Bars::kOEmpty + 8 * t, (local & 1) ^ 1)) break;
+                    tc_fence_after();
+                    Mma<D>::pv(c, t, rv.smem + vs * C::kTileBytes, j > 0);
+                    tc_commit(c.bar + Bars::kPFree + 8 * t);
+                    if (j + 1 == n) tc_commit(c.bar + Bars::kOFull + 8 * t);
+                }
+                if (!wait.ok) break;
+                tc_commit(rv.empty + 8 * vs);
             }
-            if (!wait.ok) break;
-            tc_commit(rv.empty + 8 * vs);
         }
+        if (!wait.ok) mma_drain(c, 1);
+    } else {
+        // sparse: the union of both Q tiles' key tiles
+        using C = Cfg<D>;
+        Ring rv{c.base + C::kVRingOff, c.bar + Bars::kVFull, c.bar + Bars::kVEmpty, (uint32_t)C::kVSlots, 0};
+        Waiter wait{c, true};
+        uint32_t p_phase[2] = {0u, 0u};
+        uint32_t o_units[2] = {0u, 0u};  // units in which Q tile t accumulated an O
+        for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x) {
+            const Unit w = decode_unit<MODE>(u, c.p);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const int first[2] = {pl.q[0].next(0), pl.q[1].next(0)};
+            const int last[2] = {pl.q[0].last(), pl.q[1].last()};
+            for (int j = pl.next(0); j != kNoTile; j = pl.next(j + 1)) {
+                uint32_t vs;
+                if (!wait.take(rv, vs)) break;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (!pl.need(t, j)) continue;
+                    if (!wait(c.bar + Bars::kPFull + 8 * t, p_phase[t])) break;
+                    p_phase[t] ^= 1u;
+                    const bool is_first = j == first[t];
+                    if (is_first && !wait(c.bar + Bars::kOEmpty + 8 * t, (o_units[t] & 1) ^ 1)) break;
+                    tc_fence_after();
+                    Mma<D>::pv(c, t, rv.smem + vs * C::kTileBytes, !is_first);
+                    tc_commit(c.bar + Bars::kPFree + 8 * t);
+                    if (j == last[t]) {
+                        tc_commit(c.bar + Bars::kOFull + 8 * t);
+                        ++o_units[t];
+                    }
+                }
+                if (!wait.ok) break;
+                tc_commit(rv.empty + 8 * vs);
+            }
+        }
+        if (!wait.ok) mma_drain(c, 1);
     }
-    if (!wait.ok) mma_drain(c, 1);
 }
 
-// Shared layout (P over S): one ordered stream per key tile j:
-// P_0 V_j, S_0(j+1), P_1 V_j, S_1(j+1) -- S_t(j+1) overwrites P_t(j) after
-// the product that reads it, by issue order.
-template <int D, bool CAUSAL>
+// Shared layout (P over S): one ordered stream per key tile j of the union,
+// with j' the next one: P_0 V_j, S_0(j'), P_1 V_j, S_1(j') (each product only
+// where Q tile t takes part in that tile).  S_t(j') overwrites P_t of t's
+// previous tile after the product that reads it, by issue order.
+template <int D, int MODE>
 __device__ __forceinline__ void role_mma_ordered(const Ctx& c) {
-    using C = Cfg<D>;
-    Ring r{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
-    Waiter wait{c, true};
-    uint32_t p_phase[2] = {0u, 0u};
-    int local = 0;
-    auto smem = [&](uint32_t slot) { return r.smem + slot * C::kTileBytes; };
-    for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
-        const Unit w = decode_unit<CAUSAL>(u, c.p);
-        if (!wait(c.bar + Bars::kQFull + 0, local & 1) || !wait(c.bar + Bars::kQFull + 8, local & 1)) break;
-        uint32_t ks;
-        if (!wait.take(r, ks)) break;
-        tc_fence_after();
-        Mma<D>::qk(c, 0, smem(ks));
-        tc_commit(c.bar + Bars::kSFull + 0);
-        Mma<D>::qk(c, 1, smem(ks));
-        tc_commit(c.bar + Bars::kSFull + 8);
-        if (w.n1 == 1) tc_commit(c.bar + Bars::kQEmpty);
-        tc_commit(r.empty + 8 * ks);
-        for (int j = 0; j < w.n1; ++j) {
-            uint32_t vs, ks2 = 0;
-            const bool has_next = j + 1 < w.n1;
-            if (!wait.take(r, vs)) break;
-            if (has_next && !wait.take(r, ks2)) break;
-            if (j < w.n0) {
-                if (!wait(c.bar + Bars::kPFull + 0, p_phase[0])) break;
-                p_phase[0] ^= 1u;
-                if (j == 0 && !wait(c.bar + Bars::kOEmpty + 0, (local & 1) ^ 1)) break;
+    if constexpr (MODE != kModeSparse) {
+        // full / causal: Q tile 0 visits key tiles [0, n0), Q tile 1 [0, n1), n0 <= n1
+        using C = Cfg<D>;
+        Ring r{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
+        Waiter wait{c, true};
+        uint32_t p_phase[2] = {0u, 0u};
+        int local = 0;
+        auto smem = [&](uint32_t slot) { return r.smem + slot * C::kTileBytes; };
+        for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
+            const Unit w = decode_unit<MODE>(u, c.p);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const int n0 = pl.q[0].lim + 1, n1 = pl.q[1].lim + 1;
+            if (!wait(c.bar + Bars::kQFull + 0, local & 1) || !wait(c.bar + Bars::kQFull + 8, local & 1)) break;
+            uint32_t ks;
+            if (!wait.take(r, ks)) break;
+            tc_fence_after();
+            Mma<D>::qk(c, 0, smem(ks));
+            tc_commit(c.bar + Bars::kSFull + 0);
+            Mma<D>::qk(c, 1, smem(ks));
+            tc_commit(c.bar + Bars::kSFull + 8);
+            if (n1 == 1) tc_commit(c.bar + Bars::kQEmpty);
+            tc_commit(r.empty + 8 * ks);
+            for (int j = 0; j < n1; ++j) {
+                uint32_t vs, ks2 = 0;
+                const bool has_next = j + 1 < n1;
+                if (!wait.take(r, vs)) break;
+                if (has_next && !wait.take(r, ks2)) break;
+                if (j < n0) {
+                    if (!wait(c.bar + Bars::kPFull + 0, p_phase[0])) break;
+                    p_phase[0] ^= 1u;
+                    if (j == 0 && !wait(c.bar + Bars::kOEmpty + 0, (local & 1) ^ 1)) break;
+                    tc_fence_after();
+                    Mma<D>::pv(c, 0, smem(vs), j > 0);
+                    if (j + 1 < n0) {
+                        Mma<D>::qk(c, 0, smem(ks2));
+                        tc_commit(c.bar + Bars::kSFull + 0);
+                    } else {
+                        tc_commit(c.bar + Bars::kOFull + 0);
+                    }
+                }
+                if (!wait(c.bar + Bars::kPFull + 8, p_phase[1])) break;
+                p_phase[1] ^= 1u;
+                if (j == 0 && !wait(c.bar + Bars::kOEmpty + 8, (local & 1) ^ 1)) break;
                 tc_fence_after();
-                Mma<D>::pv(c, 0, smem(vs), j > 0);
-                if (j + 1 < w.n0) {
-                    Mma<D>::qk(c, 0, smem(ks2));
-                    tc_commit(c.bar + Bars::kSFull + 0);
+                Mma<D>::pv(c, 1, smem(vs), j > 0);
+                tc_commit(r.empty + 8 * vs);
+                if (has_next) {
+                    Mma<D>::qk(c, 1, smem(ks2));
+                    tc_commit(c.bar + Bars::kSFull + 8);
+                    if (j + 2 == n1) tc_commit(c.bar + Bars::kQEmpty);
+                    tc_commit(r.empty + 8 * ks2);
                 } else {
-                    tc_commit(c.bar + Bars::kOFull + 0);
+                    tc_commit(c.bar + Bars::kOFull + 8);
                 }
             }
-            if (!wait(c.bar + Bars::kPFull + 8, p_phase[1])) break;
-            p_phase[1] ^= 1u;
-            if (j == 0 && !wait(c.bar + Bars::kOEmpty + 8, (local & 1) ^ 1)) break;
+        }
+        if (!wait.ok) mma_drain(c, 0);
+    } else {
+        // sparse: the union of both Q tiles' key tiles
+        using C = Cfg<D>;
+        Ring r{c.base + C::kRingOff, c.bar + Bars::kKFull, c.bar + Bars::kKEmpty, (uint32_t)C::kKSlots, 0};
+        Waiter wait{c, true};
+        uint32_t p_phase[2] = {0u, 0u};
+        uint32_t o_units[2] = {0u, 0u};
+        uint32_t q_units = 0;
+        auto smem = [&](uint32_t slot) { return r.smem + slot * C::kTileBytes; };
+        for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x) {
+            const Unit w = decode_unit<MODE>(u, c.p);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            int j = pl.next(0);
+            if (j == kNoTile) continue;
+            const int first[2] = {pl.q[0].next(0), pl.q[1].next(0)};
+            const int last[2] = {pl.q[0].last(), pl.q[1].last()};
+            if (!wait(c.bar + Bars::kQFull + 0, q_units & 1) || !wait(c.bar + Bars::kQFull + 8, q_units & 1)) break;
+            ++q_units;
+            uint32_t ks;
+            if (!wait.take(r, ks)) break;
             tc_fence_after();
-            Mma<D>::pv(c, 1, smem(vs), j > 0);
-            tc_commit(r.empty + 8 * vs);
-            if (has_next) {
-                Mma<D>::qk(c, 1, smem(ks2));
-                tc_commit(c.bar + Bars::kSFull + 8);
-                if (j + 2 == w.n1) tc_commit(c.bar + Bars::kQEmpty);
-                tc_commit(r.empty + 8 * ks2);
-            } else {
-                tc_commit(c.bar + Bars::kOFull + 8);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (!pl.need(t, j)) continue;
+                Mma<D>::qk(c, t, smem(ks));
+                tc_commit(c.bar + Bars::kSFull + 8 * t);
+            }
+            int jn = pl.next(j + 1);
+            if (jn == kNoTile) tc_commit(c.bar + Bars::kQEmpty);
+            tc_commit(r.empty + 8 * ks);
+            while (j != kNoTile) {
+                const bool has_next = jn != kNoTile;
+                uint32_t vs, ks2 = 0;
+                if (!wait.take(r, vs)) break;
+                if (has_next && !wait.take(r, ks2)) break;
+                const int jnn = has_next ? pl.next(jn + 1) : kNoTile;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (pl.need(t, j)) {
+                        if (!wait(c.bar + Bars::kPFull + 8 * t, p_phase[t])) break;
+                        p_phase[t] ^= 1u;
+                        const bool is_first = j == first[t];
+                        if (is_first && !wait(c.bar + Bars::kOEmpty + 8 * t, (o_units[t] & 1) ^ 1)) break;
+                        tc_fence_after();
+                        Mma<D>::pv(c, t, smem(vs), !is_first);
+                        if (j == last[t]) {
+                            tc_commit(c.bar + Bars::kOFull + 8 * t);
+                            ++o_units[t];
+                        }
+                    }
+                    if (t == 1) tc_commit(r.empty + 8 * vs);
+                    if (has_next && pl.need(t, jn)) {
+                        tc_fence_after();
+                        Mma<D>::qk(c, t, smem(ks2));
+                        tc_commit(c.bar + Bars::kSFull + 8 * t);
+                    }
+                }
+                if (!wait.ok) break;
+                if (has_next) {
+                    if (jnn == kNoTile) tc_commit(c.bar + Bars::kQEmpty);
+                    tc_commit(r.empty + 8 * ks2);
+                }
+                j = jn;
+                jn = jnn;
             }
         }
+        if (!wait.ok) mma_drain(c, 0);
     }
-    if (!wait.ok) mma_drain(c, 0);
 }
 
 // ------------------------------------------------------- softmax + epilogue
 // Warpgroup t owns Q tile t; thread = one query row = one TMEM lane.
-template <int D, bool CAUSAL, bool MASK>
+template <int D, int MODE, bool MASK>
 __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, uint16_t* __restrict__ out_o,
                                              float* __restrict__ out_lse) {
     using C = Cfg<D>;
@@ -694,17 +1006,37 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
     uint32_t pv_count = 0;  // P_t V products issued before the current step (split layout)
     bool ok = true;
     int local = 0;
+    uint32_t o_units = 0;  // sparse: units in which this Q tile has key tiles
 
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++local) {
-        const Unit w = decode_unit<CAUSAL>(u, p);
+        const Unit w = decode_unit<MODE>(u, p);
         const int row = w.q0 + t * kBlockM + r_in_tile;
-        const int n_kv = (t == 0) ? w.n0 : w.n1;
+        // step j visits key tile j (full, causal) or the j-th key tile kj of
+        // this Q tile's mask row (sparse)
+        const KeyTiles<MODE> kt = key_tiles<MODE>(w, p, c.mask_bits, t);
+        const int n_kv = kt.count();
+        int kj = kt.next(0);
+        if constexpr (MODE == kModeSparse) {
+            if (n_kv == 0) {
+                // no key block at all: O = 0 and LSE = -inf, as for a row
+                // whose keys are all masked (no barrier of this unit is used)
+                if (row < p.N) {
+                    uint4* dst = reinterpret_cast<uint4*>(out_o + w.b * p.o_sb + w.h * p.o_sh + row * p.o_sn);
+#pragma unroll
+                    for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+                    out_lse[static_cast<size_t>(w.bh) * p.N + row] = -INFINITY;
+                }
+                continue;
+            }
+        }
         // last visible key of this row (the row itself when causal)
-        const int last_key = CAUSAL ? min(row, p.N - 1) : p.N - 1;
+        const bool causal = MODE == kModeCausal || (MODE == kModeSparse && p.causal);
+        const int last_key = causal ? min(row, p.N - 1) : p.N - 1;
         float m = -INFINITY;  // reference max of scale*log2(e)*s (log2 units), shared by O and l
         float l = 0.f;        // sum of exp2(scale*log2(e)*s - m) over the keys seen so far
 
         for (int j = 0; j < n_kv; ++j) {
+            const int key_tile = MODE == kModeSparse ? kj : j;
             bool got = wait_bounded(b_s, s_phase, c.abort_flag, p.wait_ns);
             got = __all_sync(0xffffffffu, got);
             if (!got) {
@@ -735,7 +1067,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
             // key padding: the 128 mask bytes of this key tile, 16 at a time;
             // only 16-key groups that hold a padded key are touched
             if (MASK) {
-                const int key0 = j * kBlockN;
+                const int key0 = key_tile * kBlockN;
                 const uint8_t* mrow = p.key_pad + static_cast<size_t>(w.b) * p.N + key0;
                 const bool vec = p.pad_vec && key0 + kBlockN <= p.N;
 #pragma unroll
@@ -760,7 +1092,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
                 }
             }
             // key-tail and causal mask: keys past last_key get -inf
-            const int lim = last_key - j * kBlockN;
+            const int lim = last_key - key_tile * kBlockN;
             if (lim < kBlockN - 1) {
 #pragma unroll
                 for (int cc = 0; cc < kBlockN; ++cc)
@@ -844,11 +1176,12 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(b_p);
+            if constexpr (MODE == kModeSparse) kj = kt.next(kj + 1);
         }
         if (!ok) break;
 
         // ---------------------------------------------------------- epilogue
-        bool got = wait_bounded(b_of, local & 1, c.abort_flag, p.wait_ns);
+        bool got = wait_bounded(b_of, (MODE == kModeSparse ? o_units++ : local) & 1, c.abort_flag, p.wait_ns);
         got = __all_sync(0xffffffffu, got);
         if (!got) {
             ok = false;
@@ -886,8 +1219,35 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
     }
 }
 
+// Sparse mode: the [n_kv_all, n_kv_all] block-mask bytes become bits in shared
+// memory (bit f = byte f != 0, row-major), every thread taking whole 32-bit
+// words; full words read the bytes 16 at a time (the mask is 16-byte aligned).
+__device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t x) {
+    const uint32_t y = __vcmpne4(x, 0u);  // 0xFF per nonzero byte
+    return ((y >> 7) & 1u) | ((y >> 14) & 2u) | ((y >> 21) & 4u) | ((y >> 28) & 8u);
+}
+__device__ __forceinline__ void stage_block_mask(const Params& p, uint32_t* bits) {
+    const long long total = static_cast<long long>(p.n_kv_all) * p.n_kv_all;
+    const int words = static_cast<int>((total + 31) / 32);
+    for (int wi = threadIdx.x; wi < words; wi += kThreads) {
+        const long long f0 = static_cast<long long>(wi) * 32;
+        uint32_t word = 0u;
+        if (f0 + 32 <= total) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 x = ldg_nc16(p.block_mask + f0 + 16 * h);
+                word |= (nonzero_bytes4(x.x) | (nonzero_bytes4(x.y) << 4) | (nonzero_bytes4(x.z) << 8) |
+                         (nonzero_bytes4(x.w) << 12)) << (16 * h);
+            }
+        } else {
+            for (int e = 0; f0 + e < total; ++e) word |= static_cast<uint32_t>(p.block_mask[f0 + e] != 0) << e;
+        }
+        bits[wi] = word;
+    }
+}
+
 // ----------------------------------------------------------------- the kernel
-template <int D, bool CAUSAL, bool MASK>
+template <int D, int MODE, bool MASK>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out_o,
@@ -935,27 +1295,29 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_alloc(smem_addr(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
+    uint32_t* const mask_bits = reinterpret_cast<uint32_t*>(gbase + C::kMaskOff);
+    if (MODE == kModeSparse) stage_block_mask(p, mask_bits);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const Ctx ctx{base, bar, *tmem_slot, abort_flag, p};
+    const Ctx ctx{base, bar, *tmem_slot, abort_flag, mask_bits, p};
 
     if (warp >= kLoadWarp) {
         regs_decrease<kOtherRegs>();
         if (lane == 0) {
             if (warp == kLoadWarp) {
-                role_producer<D, CAUSAL>(ctx, &tm_q, &tm_k, &tm_v);
+                role_producer<D, MODE>(ctx, &tm_q, &tm_k, &tm_v);
             } else if (warp == kMmaWarp) {
-                if (C::kSplit) role_mma_s<D, CAUSAL>(ctx);
-                else role_mma_ordered<D, CAUSAL>(ctx);
+                if (C::kSplit) role_mma_s<D, MODE>(ctx);
+                else role_mma_ordered<D, MODE>(ctx);
             } else if (warp == kMmaPvWarp && C::kSplit) {
-                role_mma_pv<D, CAUSAL>(ctx);
+                role_mma_pv<D, MODE>(ctx);
             }
         }
         __syncwarp();
     } else {
         regs_increase<kSoftmaxRegs>();
-        role_softmax<D, CAUSAL, MASK>(ctx, warp, lane, out_o, out_lse);
+        role_softmax<D, MODE, MASK>(ctx, warp, lane, out_o, out_lse);
     }
 
     tc_fence_before();
@@ -1058,11 +1420,15 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
-template <int D, bool CAUSAL, bool MASK>
+// Largest block-mask side the shared-memory bit copy takes (N <= 65536).
+constexpr int kMaxMaskTiles = 512;
+
+template <int D, int MODE, bool MASK>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
            const Params& p, int grid, cudaStream_t stream) {
-    auto kernel = attn_fwd_kernel<D, CAUSAL, MASK>;
-    const int smem = Cfg<D>::kSmemBytes;
+    auto kernel = attn_fwd_kernel<D, MODE, MASK>;
+    const long long bits = static_cast<long long>(p.n_kv_all) * p.n_kv_all;
+    const int smem = Cfg<D>::kSmemBytes + (MODE == kModeSparse ? static_cast<int>((bits + 127) / 128) * 16 : 0);
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return ATTN_ERR_CUDA;
     kernel<<<grid, kThreads, smem, stream>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, p);
@@ -1086,10 +1452,10 @@ const char* attn_status_string(int status) {
     }
 }
 
-int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-                     long long qkv_sb, long long qkv_sh, long long qkv_sn, long long o_sb, long long o_sh,
-                     long long o_sn, const unsigned char* key_padding_mask, float scale, int causal,
-                     attn_stream_t stream) {
+int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                          int d, long long qkv_sb, long long qkv_sh, long long qkv_sn, long long o_sb, long long o_sh,
+                          long long o_sn, const unsigned char* key_padding_mask, const unsigned char* block_mask,
+                          float scale, int causal, attn_stream_t stream) {
     // ---- host-side validation: nothing touches the GPU until all of it passes
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
@@ -1120,13 +1486,19 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
     if (key_padding_mask &&
         (overlaps(o, out_bytes, key_padding_mask, pad_bytes) || overlaps(lse, lbytes, key_padding_mask, pad_bytes)))
         return ATTN_ERR_INVALID_ARG;
+    const int n_tiles = (N + kBlockN - 1) / kBlockN;
+    const size_t bm_bytes = static_cast<size_t>(n_tiles) * n_tiles;
+    if (block_mask && (n_tiles > kMaxMaskTiles || misaligned(block_mask, 16) ||
+                       overlaps(o, out_bytes, block_mask, bm_bytes) || overlaps(lse, lbytes, block_mask, bm_bytes)))
+        return ATTN_ERR_INVALID_ARG;
 
     if (!driver_fns().ok) return ATTN_ERR_CUDA;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
     if (!device_span_ok(q, in_bytes, dev) || !device_span_ok(k, in_bytes, dev) || !device_span_ok(v, in_bytes, dev) ||
         !device_span_ok(o, out_bytes, dev) || !device_span_ok(lse, lbytes, dev) ||
-        (key_padding_mask && !device_span_ok(key_padding_mask, pad_bytes, dev)))
+        (key_padding_mask && !device_span_ok(key_padding_mask, pad_bytes, dev)) ||
+        (block_mask && !device_span_ok(block_mask, bm_bytes, dev)))
         return ATTN_ERR_INVALID_ARG;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
@@ -1147,6 +1519,8 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
     p.o_sn = o_sn;
     p.key_pad = key_padding_mask;
     p.pad_vec = key_padding_mask && (reinterpret_cast<uintptr_t>(key_padding_mask) & 15) == 0 && N % 16 == 0;
+    p.block_mask = block_mask;
+    p.causal = causal ? 1 : 0;
     p.n_pairs = (N + kUnitRows - 1) / kUnitRows;
     p.n_kv_all = (N + kBlockN - 1) / kBlockN;
     const long long units = BH * p.n_pairs;
@@ -1157,19 +1531,25 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
     const int grid = static_cast<int>(units < sms ? units : sms);
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const bool mask = key_padding_mask != nullptr;
-    if (d == 64) {
-        if (mask)
-            return causal ? launch<64, true, true>(mq, mk, mv, o, lse, p, grid, s)
-                          : launch<64, false, true>(mq, mk, mv, o, lse, p, grid, s);
-        return causal ? launch<64, true, false>(mq, mk, mv, o, lse, p, grid, s)
-                      : launch<64, false, false>(mq, mk, mv, o, lse, p, grid, s);
-    }
-    if (mask)
-        return causal ? launch<128, true, true>(mq, mk, mv, o, lse, p, grid, s)
-                      : launch<128, false, true>(mq, mk, mv, o, lse, p, grid, s);
-    return causal ? launch<128, true, false>(mq, mk, mv, o, lse, p, grid, s)
-                  : launch<128, false, false>(mq, mk, mv, o, lse, p, grid, s);
+    const bool pad = key_padding_mask != nullptr;
+    const int mode = block_mask ? kModeSparse : causal ? kModeCausal : kModeFull;
+#define ATTN_LAUNCH(D_, M_, P_) launch<D_, M_, P_>(mq, mk, mv, o, lse, p, grid, s)
+#define ATTN_BY_MODE(D_, P_)                                      \
+    (mode == kModeSparse   ? ATTN_LAUNCH(D_, kModeSparse, P_)     \
+     : mode == kModeCausal ? ATTN_LAUNCH(D_, kModeCausal, P_)     \
+                           : ATTN_LAUNCH(D_, kModeFull, P_))
+    if (d == 64) return pad ? ATTN_BY_MODE(64, true) : ATTN_BY_MODE(64, false);
+    return pad ? ATTN_BY_MODE(128, true) : ATTN_BY_MODE(128, false);
+#undef ATTN_BY_MODE
+#undef ATTN_LAUNCH
+}
+
+int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                     long long qkv_sb, long long qkv_sh, long long qkv_sn, long long o_sb, long long o_sh,
+                     long long o_sn, const unsigned char* key_padding_mask, float scale, int causal,
+                     attn_stream_t stream) {
+    return attn_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, qkv_sb, qkv_sh, qkv_sn, o_sb, o_sh, o_sn,
+                                 key_padding_mask, nullptr, scale, causal, stream);
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,

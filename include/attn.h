@@ -99,6 +99,36 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
                      const unsigned char* key_padding_mask,
                      float scale, int causal, attn_stream_t stream);
 
+/*
+ * attn_fwd_block_sparse -- attn_fwd_strided with a block-sparse mask: only the
+ * (query block, key block) pairs whose mask entry is nonzero are loaded and
+ * multiplied (FlashAttention: Fast and Memory-Efficient Exact Attention with
+ * IO-Awareness, wiki notes, section "Block-sparse FlashAttention": a
+ * predefined mask M in {0,1}^{N/Br x N/Bc} over the kernel's blocks).
+ *
+ * block_mask: NULL (then this is exactly attn_fwd_strided), or a device byte
+ * matrix [T, T], T = ceil(N / 128), row-major, 16-byte aligned, read only:
+ * entry (r, c) nonzero means query rows [128 r, 128 r + 128) may see keys
+ * [128 c, 128 c + 128).  Br = Bc = 128 are the kernel's tile sizes.  One mask
+ * serves every batch and head.  It combines with causal (a key must also be
+ * at or before its query) and with key_padding_mask (and not padded).  A
+ * query row left with no visible key gets O = 0 and LSE = -inf.  T must be at
+ * most 512 (N <= 65536): the mask is copied to on-chip memory as bits.
+ *
+ * Work and memory traffic scale with the number of nonzero blocks.  The two
+ * 128-row Q tiles of a work unit walk the union of their mask rows, so
+ * neighbouring rows with similar patterns cost least.  Other arguments,
+ * ownership and errors as attn_fwd_strided; a misaligned or too large mask,
+ * or one that overlaps o or lse, gives ATTN_ERR_INVALID_ARG.
+ */
+int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int N, int d,
+                          long long qkv_sb, long long qkv_sh, long long qkv_sn,
+                          long long o_sb, long long o_sh, long long o_sn,
+                          const unsigned char* key_padding_mask,
+                          const unsigned char* block_mask,
+                          float scale, int causal, attn_stream_t stream);
+
 /* Human-readable name of an attn_status value (static string, never NULL). */
 const char* attn_status_string(int status);
 

@@ -27,7 +27,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    assert {"attn_fwd", "attn_fwd_strided", "attn_status_string", "attn_check_device_status",
+    assert {"attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_status_string", "attn_check_device_status",
             "attn_selftest_wait_timeout", "attn_version"} <= set(names)
 
 
@@ -111,6 +111,30 @@ def test_strided_overlap_uses_the_strided_span(lib):
     assert pkg.attn_fwd_strided(base, base + (1 << 22), base + (2 << 22), base - 4096, base + (3 << 22),
                                 1, 2, 64, 64, (8192, 64, 128), (8192, 64, 128), 0.125, 0,
                                 None) == pkg.ATTN_ERR_INVALID_ARG
+
+
+GIB = 1 << 30  # spacing of fake buffers large enough for N = 65536
+
+
+def _sparse(N, bm):
+    dense = (2 * N * 64, N * 64, 64)
+    return pkg.attn_fwd_block_sparse(GIB, 2 * GIB, 3 * GIB, 4 * GIB, 5 * GIB, 1, 2, N, 64, dense, dense, 0.125, 0,
+                                     None, block_mask=bm)
+
+
+def test_block_mask_checked_on_host(lib):
+    # misaligned (the mask is read 16 bytes at a time)
+    assert _sparse(1000, 6 * GIB + 8) == pkg.ATTN_ERR_INVALID_ARG
+    # more than 512 x 512 blocks (N > 65536) does not fit the on-chip bit copy
+    assert _sparse(65537, 6 * GIB) == pkg.ATTN_ERR_INVALID_ARG
+    # the mask must not overlap O or LSE
+    assert _sparse(1000, 4 * GIB + 64) == pkg.ATTN_ERR_INVALID_ARG
+    assert _sparse(1000, 5 * GIB) == pkg.ATTN_ERR_INVALID_ARG
+    # a well-formed call passes host validation (and, with no GPU here, fails
+    # only when it reaches the CUDA driver)
+    assert _sparse(65536, 6 * GIB) not in (pkg.ATTN_ERR_INVALID_ARG, pkg.ATTN_OK)
+    # without a mask it is attn_fwd_strided
+    assert _sparse(1000, None) not in (pkg.ATTN_ERR_INVALID_ARG, pkg.ATTN_OK)
 
 
 def test_selftest_limit_validated(lib):

@@ -246,3 +246,112 @@ def test_key_padding_image_workload_sampled():
     o_gpu = np.take_along_axis(o.float().cpu().numpy().reshape(B * H, N, d), idx[..., None], 1)
     l_gpu = np.take_along_axis(lse.cpu().numpy().reshape(B * H, N), idx, 1)
     assert np.abs(o_gpu - o_ref).max() <= TOL_O and np.abs(l_gpu - lse_ref).max() <= TOL_LSE
+
+
+# ---- block-sparse mask (FlashAttention wiki notes, "Block-sparse
+# FlashAttention"): [T, T] over 128-row query blocks x 128-key blocks
+def sparse_check(B, H, N, d, causal, bm, pad=None, seed=0, rows=None):
+    dev = torch.device("cuda:0")
+    q, k, v = make_qkv(B, H, N, d, seed=seed)
+    bm_t = torch.as_tensor(bm, dtype=torch.bool).to(dev)
+    pad_t = None if pad is None else torch.as_tensor(pad, dtype=torch.bool).to(dev)
+    o, lse = pkg.forward(q.to(dev), k.to(dev), v.to(dev), causal=causal, key_padding_mask=pad_t, block_mask=bm_t)
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    kp = None if pad is None else pad.astype(np.uint8)
+    o = o.float().cpu().numpy().reshape(B * H, N, d)
+    lse = lse.cpu().numpy().reshape(B * H, N)
+    if rows is None:
+        o_ref, lse_ref = oracle.attention_rows(q, k, v, 1.0 / math.sqrt(d), causal, key_pad=kp,
+                                               block_mask=bm.astype(np.uint8))
+    else:
+        idx = sample_rows(B, H, N, rows).numpy()
+        o_ref, lse_ref = oracle.attention_rows(q, k, v, 1.0 / math.sqrt(d), causal, rows=idx, key_pad=kp,
+                                               block_mask=bm.astype(np.uint8))
+        o = np.take_along_axis(o, idx[..., None], 1)
+        lse = np.take_along_axis(lse, idx, 1)
+    assert np.abs(o - o_ref).max() <= TOL_O
+    empty = np.isneginf(lse_ref)
+    assert (np.isneginf(lse) == empty).all()
+    if (~empty).any():
+        assert np.abs(lse[~empty] - lse_ref[~empty]).max() <= TOL_LSE
+    assert (o.reshape(-1, d)[empty.reshape(-1)] == 0).all()
+    return empty.mean()
+
+
+def random_block_mask(T, density, seed):
+    rng = np.random.default_rng(seed)
+    bm = rng.random((T, T)) < density
+    if T >= 4:
+        bm[1, :] = False          # a query block with no key block at all
+        bm[2, :] = False
+        bm[2, T - 1] = True       # only the last (ragged) key block
+    return bm
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [129, 300, 700, 1000])
+def test_block_sparse_random_full(N, d, causal):
+    T = (N + 127) // 128
+    sparse_check(2, 3, N, d, causal, random_block_mask(T, 0.5, N + d), seed=N)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_sparse_with_key_padding_full(d):
+    N, B = 777, 2
+    T = (N + 127) // 128
+    rng = np.random.default_rng(d)
+    pad = rng.random((B, N)) < 0.25
+    pad[1, 256:512] = True            # a whole key block padded for batch 1
+    for causal in (False, True):
+        sparse_check(B, 2, N, d, causal, random_block_mask(T, 0.6, d + 1), pad=pad, seed=d)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_sparse_empty_units_between_busy_ones(d):
+    # 256 work units (more than one per CTA): whole pairs of query blocks
+    # without any key block sit between busy ones, and pairs whose two query
+    # blocks use disjoint key blocks
+    N = 1000
+    bm = np.zeros((8, 8), dtype=bool)
+    bm[0, [0, 3]] = True
+    bm[1, [1, 6, 7]] = True           # pair 0: disjoint key blocks
+    bm[4, :] = True                   # pair 2: only its first query block; pair 1 empty
+    bm[7, 2] = True                   # pair 3: only its second query block
+    sparse_check(2, 32, N, d, False, bm, seed=5)
+    sparse_check(2, 32, N, d, True, bm, seed=6)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_all_ones_and_lower_triangle_block_masks_match_the_dense_kernel(d):
+    dev = torch.device("cuda:0")
+    B, H, N = 2, 3, 900
+    T = (N + 127) // 128
+    q, k, v = (x.to(dev) for x in make_qkv(B, H, N, d, seed=21))
+    ones = torch.ones(T, T, dtype=torch.bool, device=dev)
+    tri = torch.tril(ones)
+    for causal, bm in ((False, ones), (True, ones), (True, tri)):
+        o1, l1 = pkg.forward(q, k, v, causal=causal, block_mask=bm)
+        o2, l2 = pkg.forward(q, k, v, causal=causal)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_block_sparse_local_global_pattern_image_workload_sampled():
+    # the 3 MP patch self-attention shape with a local band (3 key blocks on
+    # each side) plus one global key block: about 8% of the blocks
+    N = 11616
+    T = (N + 127) // 128
+    bm = np.zeros((T, T), dtype=bool)
+    for r in range(T):
+        bm[r, max(0, r - 3):r + 4] = True
+    bm[:, 0] = True
+    sparse_check(1, 16, N, 64, False, bm, rows=256)
+
+
+def test_block_sparse_largest_mask_d128_sampled():
+    # T = 512 (N = 65536): the largest mask, at the head size with the least
+    # shared memory to spare
+    N = 65536
+    bm = random_block_mask(512, 0.05, 9)
+    np.fill_diagonal(bm, True)
+    sparse_check(1, 2, N, 128, True, bm, rows=64)
