@@ -16,9 +16,14 @@ section "IO complexity analysis"):
 * ``attn_oracle_np``  -- NumPy fp64 twin that materialises the whole N x N
   matrix (used to cross-check the C oracle on small cases).
 
+The backward (exact dQ, dK, dV for an upstream dO; wiki notes, section
+"Recomputation") has the same pair: ``attn_bwd_oracle.c`` and
+``attention_bwd_full`` in the NumPy twin.
+
 Parity status: pinned (see tests/test_oracle_pins.py).
 """
-from .oracle_c import attention_rows, build, library_path, max_threads
-from .attn_oracle_np import attention_full
+from .oracle_c import attention_bwd_rows, attention_rows, build, library_path, max_threads
+from .attn_oracle_np import attention_bwd_full, attention_full
 
-__all__ = ["attention_rows", "attention_full", "build", "library_path", "max_threads"]
+__all__ = ["attention_rows", "attention_full", "attention_bwd_rows", "attention_bwd_full", "build",
+           "library_path", "max_threads"]

@@ -7,6 +7,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "attn_oracle.c")
+_SRC_BWD = os.path.join(_HERE, "attn_bwd_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
@@ -16,12 +17,13 @@ def library_path():
 
 
 def build(force=False):
-    """Compile attn_oracle.c with gcc -O2 -fopenmp into liboracle.so (in place)."""
-    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+    """Compile attn_oracle.c and attn_bwd_oracle.c with gcc -O2 -fopenmp into liboracle.so (in place)."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_BWD))
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= newest:
         return _LIB
     tmp = _LIB + ".tmp%d" % os.getpid()
     subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
-                           "-o", tmp, _SRC, "-lm"])
+                           "-o", tmp, _SRC, _SRC_BWD, "-lm"])
     os.replace(tmp, _LIB)
     return _LIB
 
@@ -38,6 +40,12 @@ def _load():
             fn.argtypes = [ptr, ptr, ptr, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                            ctypes.c_double, ctypes.c_int, ptr, ptr, ctypes.c_int, ctypes.c_int, ptr,
                            ctypes.c_int, ptr, ptr, ctypes.c_int]
+        for name in ("attn_oracle_bwd_f64", "attn_oracle_bwd_bf16"):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = [ptr, ptr, ptr, ptr, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                           ctypes.c_double, ctypes.c_int, ptr, ctypes.c_int, ptr, ctypes.c_int, ptr, ptr, ptr,
+                           ctypes.c_int]
         lib.attn_oracle_max_threads.restype = ctypes.c_int
         lib.attn_oracle_max_threads.argtypes = []
         _lib = lib
@@ -109,3 +117,50 @@ def attention_rows(q, k, v, scale, causal=False, rows=None, n_threads=0, key_pad
     if rc != 0:
         raise ValueError("oracle rejected its arguments (code %d)" % rc)
     return o, lse
+
+
+def _select(rows, B, H, N):
+    if rows is None:
+        return N, None, None
+    a = np.asarray(rows, dtype=np.int32)
+    if a.ndim == 1:
+        a = np.broadcast_to(a, (B * H, a.shape[0]))
+    a = np.ascontiguousarray(a.reshape(B * H, -1))
+    return a.shape[1], a, a.ctypes.data
+
+
+def attention_bwd_rows(q, k, v, do, scale, causal=False, q_rows=None, k_rows=None, n_threads=0):
+    """Exact gradients of O = softmax(scale Q K^T) V for the upstream gradient dO.
+
+    q, k, v, do: [B, H, N, d], bf16 torch tensors (widened exactly) or float64
+    arrays.  q_rows / k_rows: None (all rows) or int arrays [B*H, R] (or [R],
+    shared by every head) of distinct rows: dQ is evaluated at q_rows, dK and
+    dV at k_rows.  Returns (dQ [B*H, Rq, d], dK [B*H, Rk, d], dV [B*H, Rk, d])
+    as float64 numpy arrays.
+    """
+    lib = _load()
+    try:
+        import torch
+        is_bf16 = isinstance(q, torch.Tensor) and q.dtype == torch.bfloat16
+    except ImportError:  # pragma: no cover
+        is_bf16 = False
+    B, H, N, d = (int(x) for x in q.shape)
+    if is_bf16:
+        arrs = [_bf16_bits(x) for x in (q, k, v, do)]
+        fn = lib.attn_oracle_bwd_bf16
+    else:
+        arrs = [np.ascontiguousarray(np.asarray(x, dtype=np.float64)) for x in (q, k, v, do)]
+        fn = lib.attn_oracle_bwd_f64
+    n_q, qa, qp = _select(q_rows, B, H, N)
+    n_k, ka, kp = _select(k_rows, B, H, N)
+    for sel in (qa, ka):
+        if sel is not None and any(len(set(r.tolist())) != len(r) for r in sel):
+            raise ValueError("selected rows must be distinct within a head")
+    dq = np.empty((B * H, n_q, d), dtype=np.float64)
+    dk = np.empty((B * H, n_k, d), dtype=np.float64)
+    dv = np.empty((B * H, n_k, d), dtype=np.float64)
+    rc = fn(*(a.ctypes.data for a in arrs), B, H, N, d, float(scale), int(bool(causal)), qp, n_q, kp, n_k,
+            dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments (code %d)" % rc)
+    return dq, dk, dv
