@@ -35,7 +35,7 @@ DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_d64_h16_n11616.md")
-KERNEL_SOURCE = os.path.join(ROOT, "exact_io_aware_102_b200", "csrc", "attn_fwd.cu")
+KERNEL_SOURCES = [os.path.join(ROOT, "exact_io_aware_102_b200", "csrc", f) for f in ("attn_fwd.cu", "sm100_ptx.cuh")]
 
 
 # ----------------------------------------------------------------- arithmetic
@@ -72,8 +72,12 @@ def load_peaks():
 
 
 def source_digest():
-    with open(KERNEL_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Digest of the forward kernel's sources (the kernel file and its PTX helper header)."""
+    h = hashlib.sha256()
+    for path in KERNEL_SOURCES:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic():

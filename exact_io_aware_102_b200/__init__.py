@@ -6,17 +6,17 @@ supplies device memory and the current stream.  There is no fallback: if the
 library is missing, every entry point raises.
 
 The C entry points keep their names here (``attn_fwd``, ``attn_fwd_strided``,
-``attn_fwd_block_sparse``, ``attn_status_string``, ``attn_check_device_status``,
+``attn_fwd_block_sparse``, ``attn_bwd``, ``attn_status_string``, ``attn_check_device_status``,
 ``attn_selftest_wait_timeout``, ``attn_version``); ``forward`` is the tensor
-convenience wrapper.
+convenience wrapper and ``backward`` its gradient counterpart.
 """
 import ctypes
 import math
 import os
 
 __all__ = [
-    "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_status_string", "attn_check_device_status",
-    "attn_selftest_wait_timeout", "attn_version", "forward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
+    "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_bwd", "attn_status_string", "attn_check_device_status",
+    "attn_selftest_wait_timeout", "attn_version", "forward", "backward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
 ]
 
@@ -53,6 +53,8 @@ def library():
         lib.attn_fwd_block_sparse.restype = i32
         lib.attn_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i64, i64, i64, i64,
                                               i64, vp, vp, ctypes.c_float, i32, vp]
+        lib.attn_bwd.restype = i32
+        lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, i32, vp]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_status_string.argtypes = [i32]
         lib.attn_check_device_status.restype = i32
@@ -90,6 +92,12 @@ def attn_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, qkv_strides, o_strides, s
     return library().attn_fwd_block_sparse(q, k, v, o, lse, int(B), int(H), int(N), int(d), sb, sh, sn, ob, oh,
                                            on, key_padding_mask, block_mask, float(scale), int(bool(causal)),
                                            stream)
+
+
+def attn_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, N, d, scale, causal, stream):
+    """Raw C call: device addresses as ints; returns the status."""
+    return library().attn_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, int(B), int(H), int(N), int(d),
+                              float(scale), int(bool(causal)), stream)
 
 
 def attn_status_string(status):
@@ -188,3 +196,34 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None, 
     if status != ATTN_OK:
         raise AttnError(status, what)
     return out, lse
+
+
+def backward(q, k, v, o, lse, dout, scale=None, causal=False, stream=None):
+    """Gradients of ``forward`` for the upstream gradient ``dout``.
+
+    q, k, v, o, dout: contiguous bf16 CUDA tensors [B, H, N, 64] (o and lse
+    from ``forward`` on the same q, k, v, scale and causal).  Returns
+    (dq fp32, dk bf16, dv bf16), each [B, H, N, 64].  Asynchronous on
+    ``stream`` (default: the current stream).
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("%s must be a contiguous bf16 CUDA tensor shaped like q" % name)
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    B, H, N, d = (int(x) for x in q.shape)
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor [B, H, N]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    delta = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    dq = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    dk = torch.empty_like(q)
+    dv = torch.empty_like(q)
+    status = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                      delta.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, scale, causal,
+                      _stream_handle(stream))
+    if status != ATTN_OK:
+        raise AttnError(status, "attn_bwd")
+    return dq, dk, dv

@@ -1,7 +1,7 @@
 """Build step for libattn.so (nvcc, sm_100a, in-tree).
 
-``python -m exact_io_aware_102_b200.build`` compiles ``csrc/attn_fwd.cu``
-into ``libattn.so`` next to this file.  The CUDA runtime is linked statically
+``python -m exact_io_aware_102_b200.build`` compiles ``csrc/attn_fwd.cu`` and
+``csrc/attn_bwd.cu`` into ``libattn.so`` next to this file.  The CUDA runtime is linked statically
 and the driver is reached through cudaGetDriverEntryPoint, so the library
 loads on machines without a GPU (its argument checks then still work).
 """
@@ -11,7 +11,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SRC = os.path.join(HERE, "csrc", "attn_fwd.cu")
+SRCS = [os.path.join(HERE, "csrc", f) for f in ("attn_fwd.cu", "attn_bwd.cu")]
 OUT = os.path.join(HERE, "libattn.so")
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -30,7 +30,7 @@ def nvcc():
 
 def build(verbose=False, extra=()):
     tmp = OUT + ".tmp%d" % os.getpid()
-    cmd = [nvcc()] + NVCC_FLAGS + list(extra) + ["-o", tmp, SRC]
+    cmd = [nvcc()] + NVCC_FLAGS + list(extra) + ["-o", tmp] + SRCS
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)

@@ -1,0 +1,707 @@
+// Exact attention backward for B200 (sm_100a), head size 64.
+//
+// What is computed (FlashAttention: Fast and Memory-Efficient Exact Attention
+// with IO-Awareness, wiki notes, section "Recomputation"): the forward kept
+// only O and one log-sum-exp per query row; the backward rebuilds the score
+// tiles S = scale Q K^T and the probabilities P = exp(S - LSE) tile by tile on
+// chip and never stores an N x N matrix.  For an upstream gradient dO:
+//
+//     dV = P^T dO,  dP = dO V^T,  dS = P o (dP - delta),  delta_i = dO_i . O_i,
+//     dQ = scale dS K,  dK = scale dS^T Q
+//
+// (delta_i = sum_j P_ij dP_ij, written through O = P V).
+//
+// How it maps to sm_100a:
+//   * a small kernel first writes delta = rowsum(dO o O) and clears the fp32
+//     dQ accumulator;
+//   * the main kernel runs a persistent grid, one CTA per SM; a work unit is
+//     one (batch, head, 128-key block).  dK and dV of the block accumulate in
+//     TMEM over the query tiles (128 rows each) the block interacts with;
+//   * warp 8 (one lane) loads K, V once per unit and Q_i, dO_i per query tile
+//     (two stages) by TMA; warp 9 (one lane) issues the tcgen05.mma:
+//     S^T = K Q_i^T and dP^T = V dO_i^T into TMEM, then dV += P^T dO_i,
+//     dK += dS^T Q_i and the dQ partial dS K_j;
+//   * warps 0-3 (one thread per key row) turn the S^T, dP^T rows into P^T and
+//     dS^T (bf16), written to shared memory in the 128-byte-swizzled layout
+//     the tensor core reads -- one dS^T tile serves dK (K-major) and, read
+//     transposed, dQ (M-major);
+//   * warps 4-7 (one thread per query row) read the dQ partial from TMEM and
+//     add it to the fp32 dQ accumulator in global memory with bulk
+//     asynchronous reductions (cp.reduce.async.bulk .add.f32), one 256-byte
+//     row per thread;
+//   * at the end of a unit warps 0-3 write dK (times scale) and dV in bf16.
+//   Every wait is bounded (see sm100_ptx.cuh) and no barrier spans warps
+//   other than mbarriers, so a timeout never leaves a thread blocked.
+//
+// TMEM columns: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
+// dQ [384,448).  Shared memory: K, V (16 KB each), two stages of Q and dO
+// (16 KB each), P^T and dS^T (32 KB each, two 64-column halves), dQ staging
+// rows, per-warp LSE / delta rows, barriers.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "attn.h"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+constexpr int kD = 64;            // head size handled here
+constexpr int kBK = 128;          // keys per unit (= TMEM lanes)
+constexpr int kBQ = 128;          // query rows per tile
+constexpr int kThreads = 320;     // warps 0-3 P/dS, 4-7 dQ, 8 load, 9 MMA
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
+constexpr float kLog2eB = 1.4426950408889634f;
+constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait
+constexpr unsigned long long kDrainNs = 100000000ull;   // 0.1 s per drain wait
+
+constexpr int kTile = kBQ * kD * 2;   // one bf16 [128 x 64] tile, 128-byte swizzle
+constexpr int kHalf = 128 * 64 * 2;   // one 64-column half of a [128 x 128] bf16 tile
+// shared-memory map (offsets from the 1 KB aligned base)
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kTile;
+constexpr int kOffQ = kOffV + kTile;          // [2] stages
+constexpr int kOffDO = kOffQ + 2 * kTile;     // [2] stages
+constexpr int kOffP = kOffDO + 2 * kTile;     // P^T, two halves
+constexpr int kOffDS = kOffP + 2 * kHalf;     // dS^T, two halves
+constexpr int kOffStage = kOffDS + 2 * kHalf; // dQ staging: 128 rows x 64 fp32, rows padded
+constexpr int kStageRowBytes = kD * 4 + 16;   // the padding spreads a warp's rows over all banks
+constexpr int kStageWarpBytes = 32 * kStageRowBytes;
+constexpr int kOffRow = kOffStage + 4 * kStageWarpBytes;  // per softmax warp: lse2[128], delta[128]
+constexpr int kRowWarpBytes = 2 * kBQ * 4;
+constexpr int kOffBar = kOffRow + 4 * kRowWarpBytes;
+constexpr int kSmemBytes = kOffBar + 256 + 1024;
+
+struct Bars {
+    static constexpr int kKVFull = 0, kKVEmpty = 8;
+    static constexpr int kQFull = 16;    // [2]
+    static constexpr int kQEmpty = 32;   // [2]
+    static constexpr int kSFull = 48, kSFree = 56;
+    static constexpr int kPFull = 64, kPFree = 72;
+    static constexpr int kDQFull = 80, kDQEmpty = 88;
+    static constexpr int kDKVFull = 96, kDKVEmpty = 104;
+    static constexpr int kDrain = 112;
+    static constexpr int kTmemSlot = 120, kAbort = 124;
+};
+
+struct BwdParams {
+    int BH, N, n_kb, n_qt, total_units, causal;
+    float scale, scale_log2;
+    const float* lse;     // [BH, N]
+    const float* delta;   // [BH, N]
+    float* dq;            // [BH, N, 64] fp32, accumulated
+    uint16_t* dk;         // [BH, N, 64] bf16
+    uint16_t* dv;
+    unsigned long long wait_ns;
+};
+
+struct BwdUnit {
+    int bh, kb, i0;  // head, key block, first query tile
+};
+
+// Units: (head, key block).  Non-causal: heads-major, so the CTAs running at
+// one time stream the same Q / dO tiles (L2 reuse).  Causal: key block kb
+// meets query tiles kb .. n_qt-1; the blocks with most tiles go first.
+__device__ __forceinline__ BwdUnit bwd_unit(int u, const BwdParams& p) {
+    BwdUnit w;
+    if (p.causal) {
+        w.kb = u / p.BH;
+        w.bh = u - w.kb * p.BH;
+        w.i0 = w.kb;
+    } else {
+        w.bh = u / p.n_kb;
+        w.kb = u - w.bh * p.n_kb;
+        w.i0 = 0;
+    }
+    return w;
+}
+
+struct Ctx {
+    uint32_t base, bar, tmem;
+    volatile uint32_t* abort_flag;
+    uint8_t* gbase;
+    BwdParams p;
+};
+
+__device__ __forceinline__ bool wait_b(const Ctx& c, uint32_t bar, uint32_t parity) {
+    return wait_bounded(bar, parity, c.abort_flag, c.p.wait_ns);
+}
+
+// ---------------------------------------------------------------- TMA producer
+__device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, const CUtensorMap* tk,
+                                          const CUtensorMap* tv, const CUtensorMap* tdo) {
+    const BwdParams& p = c.p;
+    uint32_t g = 0;      // query tiles issued
+    uint32_t units = 0;  // units whose K / V were issued
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        const BwdUnit w = bwd_unit(u, p);
+        if (!wait_b(c, c.bar + Bars::kKVEmpty, (units & 1) ^ 1)) {
+            ok = false;
+            break;
+        }
+        mbar_expect_tx(c.bar + Bars::kKVFull, 2 * kTile);
+        tma_load_4d(c.base + kOffK, tk, c.bar + Bars::kKVFull, 0, w.kb * kBK, w.bh, 0);
+        tma_load_4d(c.base + kOffV, tv, c.bar + Bars::kKVFull, 0, w.kb * kBK, w.bh, 0);
+        ++units;
+        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+            const uint32_t s = g & 1;
+            if (!wait_b(c, c.bar + Bars::kQEmpty + 8 * s, ((g >> 1) & 1) ^ 1)) {
+                ok = false;
+                break;
+            }
+            const uint32_t fb = c.bar + Bars::kQFull + 8 * s;
+            mbar_expect_tx(fb, 2 * kTile);
+            tma_load_4d(c.base + kOffQ + s * kTile, tq, fb, 0, i * kBQ, w.bh, 0);
+            tma_load_4d(c.base + kOffDO + s * kTile, tdo, fb, 0, i * kBQ, w.bh, 0);
+        }
+    }
+    if (!ok) {
+        // every issued copy lands before the CTA may exit
+        if (units > 0) wait_bounded(c.bar + Bars::kKVFull, (units - 1) & 1, nullptr, kDrainNs);
+        for (uint32_t k = (g > 2 ? g - 2 : 0); k < g; ++k)
+            wait_bounded(c.bar + Bars::kQFull + 8 * (k & 1), (k >> 1) & 1, nullptr, kDrainNs);
+    }
+}
+
+// ---------------------------------------------------------------- MMA issuing
+struct BwdMma {
+    static constexpr uint32_t kHi = sdesc_hi_sw128(1024);
+    // M = 128, N = 128, both operands K-major (S^T, dP^T)
+    static constexpr uint32_t kIdescNN = idesc_bf16_f32(128, 128, false);
+    // M = 128, N = 64, A K-major, B M/N-major (dV, dK)
+    static constexpr uint32_t kIdescKT = idesc_bf16_f32(128, 64, true);
+    // M = 128, N = 64, A and B M/N-major (dQ: A = dS read from the dS^T tile)
+    static constexpr uint32_t kIdescTT = idesc_bf16_f32(128, 64, true) | (1u << 15);
+
+    // D[128 x 128] = A[128 x 64] B[128 x 64]^T, both K-major tiles
+    __device__ __forceinline__ static void nt(uint32_t d, uint32_t a, uint32_t b) {
+        const uint32_t a0 = sdesc_lo(a, 16), b0 = sdesc_lo(b, 16);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+            mma_ss_lo(d, a0 + ((kk * 32) >> 4), b0 + ((kk * 32) >> 4), kHi, kIdescNN, kk > 0 ? 1u : 0u);
+    }
+    // D[128 x 64] (+)= A[128 x 128] B[128 x 64]: A K-major in two 64-column
+    // halves, B M/N-major (rows = the 128-long K dimension)
+    __device__ __forceinline__ static void kt(uint32_t d, uint32_t a, uint32_t b, bool acc) {
+        const uint32_t a0 = sdesc_lo(a, 16), b0 = sdesc_lo(b, kHalf);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+            mma_ss_lo(d, a0 + (((kk / 4) * kHalf + (kk % 4) * 32) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi,
+                      kIdescKT, (acc || kk > 0) ? 1u : 0u);
+    }
+    // D[128 x 64] = A[128 x 128] B[128 x 64] with A stored transposed (the
+    // dS^T tile: rows = K, two 64-wide halves of M), B M/N-major
+    __device__ __forceinline__ static void tt(uint32_t d, uint32_t a_t, uint32_t b) {
+        const uint32_t a0 = sdesc_lo(a_t, kHalf), b0 = sdesc_lo(b, kHalf);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+            mma_ss_lo(d, a0 + ((kk * 16 * 128) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi, kIdescTT,
+                      kk > 0 ? 1u : 0u);
+    }
+};
+
+__device__ __forceinline__ void role_mma(const Ctx& c) {
+    const BwdParams& p = c.p;
+    const uint32_t t = c.tmem;
+    bool ok = true;
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+        if (ok && !wait_b(c, bar, parity)) ok = false;
+        return ok;
+    };
+    uint32_t g = 0;       // query tiles of this CTA so far (S issued for tiles < g_s)
+    uint32_t units = 0;
+    // S^T and dP^T of tile g into TMEM, once the P/dS warps have loaded tile g-1
+    auto issue_s = [&](uint32_t gg) {
+        const uint32_t s = gg & 1;
+        if (!wait(c.bar + Bars::kQFull + 8 * s, (gg >> 1) & 1)) return;
+        if (gg > 0 && !wait(c.bar + Bars::kSFree, (gg - 1) & 1)) return;
+        tc_fence_after();
+        BwdMma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kTile);
+        BwdMma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kTile);
+        tc_commit(c.bar + Bars::kSFull);
+    };
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++units) {
+        const BwdUnit w = bwd_unit(u, p);
+        const int n = p.n_qt - w.i0;
+        if (!wait(c.bar + Bars::kKVFull, units & 1)) break;
+        issue_s(g);
+        for (int it = 0; ok && it < n; ++it, ++g) {
+            if (it + 1 < n) issue_s(g + 1);  // overlaps the P/dS work of tile g
+            if (!wait(c.bar + Bars::kPFull, g & 1)) break;
+            if (it == 0 && !wait(c.bar + Bars::kDKVEmpty, (units & 1) ^ 1)) break;
+            if (!wait(c.bar + Bars::kDQEmpty, (g & 1) ^ 1)) break;
+            tc_fence_after();
+            const uint32_t s = g & 1;
+            BwdMma::kt(t + kColDV, c.base + kOffP, c.base + kOffDO + s * kTile, it > 0);  // dV += P^T dO
+            BwdMma::kt(t + kColDK, c.base + kOffDS, c.base + kOffQ + s * kTile, it > 0);  // dK += dS^T Q
+            BwdMma::tt(t + kColDQ, c.base + kOffDS, c.base + kOffK);                        // dQ_j = dS K
+            tc_commit(c.bar + Bars::kPFree);
+            tc_commit(c.bar + Bars::kQEmpty + 8 * s);
+            tc_commit(c.bar + Bars::kDQFull);
+            if (it + 1 == n) {
+                tc_commit(c.bar + Bars::kDKVFull);
+                tc_commit(c.bar + Bars::kKVEmpty);
+            }
+        }
+    }
+    if (!ok) {
+        tc_commit(c.bar + Bars::kDrain);
+        wait_bounded(c.bar + Bars::kDrain, 0, nullptr, kDrainNs);
+    }
+}
+
+// Byte offset of element (row r, column col) of a [128 x 128] bf16 tile kept
+// as two 128-byte-swizzled 64-column halves (the layout TMA writes and the
+// tensor core reads): 16-byte chunk c of row r sits at chunk c ^ (r % 8).
+__device__ __forceinline__ uint32_t sw128_off(int r, int col) {
+    const int h = col >> 6, c16 = (col & 63) >> 3;
+    return static_cast<uint32_t>(h * kHalf + r * 128 + ((c16 ^ (r & 7)) << 4) + (col & 7) * 2);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c4, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c4), "r"(d)
+                 : "memory");
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
+// ---------------------------------------------------------- P / dS warps (0-3)
+// Thread = key row r of the unit's block = TMEM lane r.
+__device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
+    const BwdParams& p = c.p;
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_s = c.tmem + lane_off + kColS, t_dp = c.tmem + lane_off + kColDP;
+    const uint32_t t_dv = c.tmem + lane_off + kColDV, t_dk = c.tmem + lane_off + kColDK;
+    const uint32_t rows_smem = c.base + kOffRow + warp * kRowWarpBytes;  // lse2[128], delta[128]
+    const float sl2 = p.scale_log2;
+    uint32_t g = 0, units = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++units) {
+        const BwdUnit w = bwd_unit(u, p);
+        const int key = w.kb * kBK + r;
+        const bool key_ok = key < p.N;
+        const float* lse_h = p.lse + static_cast<size_t>(w.bh) * p.N;
+        const float* dl_h = p.delta + static_cast<size_t>(w.bh) * p.N;
+        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+            // this warp's copy of LSE * log2(e) and delta for the 128 query
+            // rows of tile i (rows past N: LSE = +inf, delta = 0, so P = dS = 0)
+            __syncwarp();
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int q = i * kBQ + lane * 4 + e;
+                const bool in = q < p.N;
+                const float l2 = in ? lse_h[q] * kLog2eB : INFINITY;
+                const float dl = in ? dl_h[q] : 0.f;
+                asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + (lane * 4 + e) * 4), "f"(l2) : "memory");
+                asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + 512 + (lane * 4 + e) * 4), "f"(dl)
+                             : "memory");
+            }
+            __syncwarp();
+            bool got = wait_b(c, c.bar + Bars::kSFull, g & 1);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // P^T / dS^T of the previous tile must have been consumed
+            if (g > 0) {
+                got = wait_b(c, c.bar + Bars::kPFree, (g - 1) & 1);
+                got = __all_sync(0xffffffffu, got);
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+            }
+            const bool diag = p.causal && i == w.kb;  // causal: query q sees key r iff q >= r
+#pragma unroll 1
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32(t_s + c4 * 32, sr);
+                tmem_ld32(t_dp + c4 * 32, dr);
+                tmem_wait_ld();
+                reg_fence32(sr);
+                reg_fence32(dr);
+                if (c4 == 3) {
+                    tc_fence_before();
+                    mbar_arrive(c.bar + Bars::kSFree);  // S^T / dP^T may be overwritten
+                }
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const float4 l2 = ld_shared_f4(rows_smem + (c4 * 32 + v * 4) * 4);
+                    const float4 dl = ld_shared_f4(rows_smem + 512 + (c4 * 32 + v * 4) * 4);
+                    const float lv[4] = {l2.x, l2.y, l2.z, l2.w};
+                    const float dv[4] = {dl.x, dl.y, dl.z, dl.w};
+                    float pp[4], ds[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = c4 * 32 + v * 4 + e;
+                        float x = ex2(fmaf(__uint_as_float(sr[v * 4 + e]), sl2, -lv[e]));
+                        if (!key_ok || (diag && q < r)) x = 0.f;
+                        pp[e] = x;
+                        ds[e] = x * (__uint_as_float(dr[v * 4 + e]) - dv[e]);
+                    }
+                    pk[v * 2] = pack_bf16x2(pp[0], pp[1]);
+                    pk[v * 2 + 1] = pack_bf16x2(pp[2], pp[3]);
+                    dk[v * 2] = pack_bf16x2(ds[0], ds[1]);
+                    dk[v * 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                }
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    const uint32_t off = sw128_off(r, c4 * 32 + q8 * 8);
+                    st_shared_v4(c.base + kOffP + off, pk[q8 * 4], pk[q8 * 4 + 1], pk[q8 * 4 + 2], pk[q8 * 4 + 3]);
+                    st_shared_v4(c.base + kOffDS + off, dk[q8 * 4], dk[q8 * 4 + 1], dk[q8 * 4 + 2], dk[q8 * 4 + 3]);
+                }
+            }
+            fence_proxy_async();  // the tensor core reads what the generic proxy wrote
+            mbar_arrive(c.bar + Bars::kPFull);
+        }
+        if (!ok) break;
+        // unit epilogue: dK (times scale) and dV of this key row
+        bool got = wait_b(c, c.bar + Bars::kDKVFull, units & 1);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        uint32_t a[2][32], b[2][32];
+        tmem_ld32(t_dv, a[0]);
+        tmem_ld32(t_dv + 32, a[1]);
+        tmem_ld32(t_dk, b[0]);
+        tmem_ld32(t_dk + 32, b[1]);
+        tmem_wait_ld();
+        reg_fence32(a[0]);
+        reg_fence32(a[1]);
+        reg_fence32(b[0]);
+        reg_fence32(b[1]);
+        tc_fence_before();
+        mbar_arrive(c.bar + Bars::kDKVEmpty);
+        if (key_ok) {
+            const size_t row = (static_cast<size_t>(w.bh) * p.N + key) * kD;
+            uint4* dvr = reinterpret_cast<uint4*>(p.dv + row);
+            uint4* dkr = reinterpret_cast<uint4*>(p.dk + row);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4) {
+                    uint32_t x[4], y[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int cc = v4 * 8 + e * 2;
+                        x[e] = pack_bf16x2(__uint_as_float(a[h][cc]), __uint_as_float(a[h][cc + 1]));
+                        y[e] = pack_bf16x2(__uint_as_float(b[h][cc]) * p.scale, __uint_as_float(b[h][cc + 1]) * p.scale);
+                    }
+                    dvr[h * 4 + v4] = make_uint4(x[0], x[1], x[2], x[3]);
+                    dkr[h * 4 + v4] = make_uint4(y[0], y[1], y[2], y[3]);
+                }
+        }
+    }
+}
+
+// ------------------------------------------------------------- dQ warps (4-7)
+// Thread = query row of the tile = TMEM lane; each thread stages its row
+// (scaled) in shared memory and adds it to dQ with one bulk reduction.
+__device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
+    const BwdParams& p = c.p;
+    const int quarter = warp & 3;
+    const uint32_t t_dq = c.tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColDQ;
+    const uint32_t my_row = c.base + kOffStage + quarter * kStageWarpBytes + lane * kStageRowBytes;
+    uint32_t g = 0;
+    bool pending = false;  // this thread's last bulk reduction may still read its staging row
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        const BwdUnit w = bwd_unit(u, p);
+        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+            bool got = wait_b(c, c.bar + Bars::kDQFull, g & 1);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t a[2][32];
+            tmem_ld32(t_dq, a[0]);
+            tmem_ld32(t_dq + 32, a[1]);
+            tmem_wait_ld();
+            reg_fence32(a[0]);
+            reg_fence32(a[1]);
+            tc_fence_before();
+            mbar_arrive(c.bar + Bars::kDQEmpty);
+            if (pending) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            pending = false;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int v4 = 0; v4 < 8; ++v4)
+                    st_shared_v4(my_row + (h * 8 + v4) * 16, __float_as_uint(__uint_as_float(a[h][v4 * 4]) * p.scale),
+                                 __float_as_uint(__uint_as_float(a[h][v4 * 4 + 1]) * p.scale),
+                                 __float_as_uint(__uint_as_float(a[h][v4 * 4 + 2]) * p.scale),
+                                 __float_as_uint(__uint_as_float(a[h][v4 * 4 + 3]) * p.scale));
+            fence_proxy_async();
+            const int row = i * kBQ + quarter * 32 + lane;
+            if (row < p.N) {
+                float* dst = p.dq + (static_cast<size_t>(w.bh) * p.N + row) * kD;
+                asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+                             "r"(my_row), "r"(static_cast<uint32_t>(kD * 4))
+                             : "memory");
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                pending = true;
+            }
+            __syncwarp();
+        }
+    }
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
+}
+
+// ------------------------------------------------------------------ kernels
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* const gbase = smem_raw + (base - raw);
+    const uint32_t bar = base + kOffBar;
+    volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + kOffBar + Bars::kAbort);
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + Bars::kTmemSlot);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(bar + Bars::kKVFull, 1);
+        mbar_init(bar + Bars::kKVEmpty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar + Bars::kQFull + 8 * s, 1);
+            mbar_init(bar + Bars::kQEmpty + 8 * s, 1);
+        }
+        mbar_init(bar + Bars::kSFull, 1);
+        mbar_init(bar + Bars::kSFree, kBK);
+        mbar_init(bar + Bars::kPFull, kBK);
+        mbar_init(bar + Bars::kPFree, 1);
+        mbar_init(bar + Bars::kDQFull, 1);
+        mbar_init(bar + Bars::kDQEmpty, kBQ);
+        mbar_init(bar + Bars::kDKVFull, 1);
+        mbar_init(bar + Bars::kDKVEmpty, kBK);
+        mbar_init(bar + Bars::kDrain, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+        fence_proxy_async();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const Ctx ctx{base, bar, *tmem_slot, abort_flag, gbase, p};
+    if (warp < 4) {
+        role_pds(ctx, warp, lane);
+    } else if (warp < 8) {
+        role_dq(ctx, warp, lane);
+    } else {
+        if (lane == 0) {
+            if (warp == kLoadWarp) role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do);
+            else if (warp == kMmaWarp) role_mma(ctx);
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(ctx.tmem, kTmemCols);
+    }
+}
+
+// delta[row] = sum_t dO[row, t] * O[row, t] (fp32), and the dQ accumulator
+// cleared; one thread per row.
+__global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                                     float* __restrict__ delta, float* __restrict__ dq, long long rows) {
+    for (long long row = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; row < rows;
+         row += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const uint4* a = reinterpret_cast<const uint4*>(o + row * kD);
+        const uint4* b = reinterpret_cast<const uint4*>(dout + row * kD);
+        float acc = 0.f;
+#pragma unroll
+        for (int v = 0; v < kD / 8; ++v) {
+            const uint4 x = a[v], y = b[v];
+            const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc = fmaf(__uint_as_float(xs[e] << 16), __uint_as_float(ys[e] << 16), acc);
+                acc = fmaf(__uint_as_float(xs[e] & 0xFFFF0000u), __uint_as_float(ys[e] & 0xFFFF0000u), acc);
+            }
+        }
+        delta[row] = acc;
+        float4* z = reinterpret_cast<float4*>(dq + row * kD);
+#pragma unroll
+        for (int v = 0; v < kD / 4; ++v) z[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+typedef CUresult (*AddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+struct BwdDriver {
+    EncodeTiledFn encode;
+    AddressRangeFn range;
+    bool ok;
+};
+
+// Driver entry points, looked up once (thread-safe static initialisation).
+const BwdDriver& bwd_driver() {
+    static const BwdDriver fns = [] {
+        BwdDriver f{nullptr, nullptr, false};
+        cudaDriverEntryPointQueryResult q1, q2;
+        void *f1 = nullptr, *f2 = nullptr;
+        f.ok = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+               q1 == cudaDriverEntryPointSuccess &&
+               cudaGetDriverEntryPoint("cuMemGetAddressRange", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+               q2 == cudaDriverEntryPointSuccess;
+        f.encode = reinterpret_cast<EncodeTiledFn>(f1);
+        f.range = reinterpret_cast<AddressRangeFn>(f2);
+        return f;
+    }();
+    return fns;
+}
+
+// bf16 [BH, N, 64] contiguous as a 4-D (64, N, BH, 1) map, box 64 x 128, 128-byte swizzle,
+// rows past N read as zeros.
+bool encode_map(EncodeTiledFn enc, CUtensorMap* map, const void* ptr, int BH, int N) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(N),
+                                static_cast<cuuint64_t>(BH), 1};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(N) * kD * 2,
+                                   static_cast<cuuint64_t>(BH) * N * kD * 2};
+    const cuuint32_t box[4] = {64, 128, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool span_ok(AddressRangeFn range, const void* ptr, size_t bytes, int device) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if ((a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) || a.device != device) return false;
+    CUdeviceptr lo = 0;
+    size_t size = 0;
+    if (range(&lo, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(ptr);
+    return x >= lo && bytes <= size && x - lo <= size - bytes;
+}
+
+bool disjoint(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x >= y + nb || y >= x + na;
+}
+
+}  // namespace
+
+// Status word of this translation unit (read and cleared by attn_check_device_status).
+int attn_bwd_take_device_status(int* status) {
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(status, g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, float* delta, float* dq, void* dk, void* dv, int B, int H, int N,
+                        int d, float scale, int causal, attn_stream_t stream) {
+    if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
+    if (d != kD) return ATTN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !o || !dout || !lse || !delta || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+    if (!isfinite(scale) || !(scale >= 1e-30f)) return ATTN_ERR_INVALID_ARG;
+    const long long BH = static_cast<long long>(B) * H;
+    if (BH > 0x7fffffffLL || N > 0x7fffffff - kBQ || BH * N > (1LL << 40) / kD) return ATTN_ERR_INVALID_ARG;
+    auto mis = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
+    if (mis(q, 16) || mis(k, 16) || mis(v, 16) || mis(o, 16) || mis(dout, 16) || mis(dk, 16) || mis(dv, 16) ||
+        mis(dq, 16) || mis(lse, 4) || mis(delta, 4))
+        return ATTN_ERR_INVALID_ARG;
+    const size_t rows = static_cast<size_t>(BH) * N;
+    const size_t tb = rows * kD * 2, qb = rows * kD * 4, lb = rows * 4;
+    // outputs must not overlap any input or each other
+    const void* ins[6] = {q, k, v, o, dout, lse};
+    const size_t in_b[6] = {tb, tb, tb, tb, tb, lb};
+    const void* outs[4] = {delta, dq, dk, dv};
+    const size_t out_b[4] = {lb, qb, tb, tb};
+    for (int a = 0; a < 4; ++a) {
+        for (int b = 0; b < 6; ++b)
+            if (!disjoint(outs[a], out_b[a], ins[b], in_b[b])) return ATTN_ERR_INVALID_ARG;
+        for (int b = a + 1; b < 4; ++b)
+            if (!disjoint(outs[a], out_b[a], outs[b], out_b[b])) return ATTN_ERR_INVALID_ARG;
+    }
+    const BwdDriver& drv = bwd_driver();
+    if (!drv.ok) return ATTN_ERR_CUDA;
+    const EncodeTiledFn enc = drv.encode;
+    const AddressRangeFn range = drv.range;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    for (int a = 0; a < 6; ++a)
+        if (!span_ok(range, ins[a], in_b[a], dev)) return ATTN_ERR_INVALID_ARG;
+    for (int a = 0; a < 4; ++a)
+        if (!span_ok(range, outs[a], out_b[a], dev)) return ATTN_ERR_INVALID_ARG;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return ATTN_ERR_CUDA;
+    alignas(64) CUtensorMap mq, mk, mv, mdo;
+    const int bh = static_cast<int>(BH);
+    if (!encode_map(enc, &mq, q, bh, N) || !encode_map(enc, &mk, k, bh, N) || !encode_map(enc, &mv, v, bh, N) ||
+        !encode_map(enc, &mdo, dout, bh, N))
+        return ATTN_ERR_CUDA;
+
+    BwdParams p;
+    p.BH = bh;
+    p.N = N;
+    p.n_kb = (N + kBK - 1) / kBK;
+    p.n_qt = (N + kBQ - 1) / kBQ;
+    const long long units = BH * p.n_kb;
+    if (units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    p.total_units = static_cast<int>(units);
+    p.causal = causal ? 1 : 0;
+    p.scale = scale;
+    p.scale_log2 = scale * kLog2eB;
+    p.lse = lse;
+    p.delta = delta;
+    p.dq = dq;
+    p.dk = static_cast<uint16_t*>(dk);
+    p.dv = static_cast<uint16_t*>(dv);
+    p.wait_ns = kWaitNs;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long long prep_blocks = (static_cast<long long>(rows) + 255) / 256;
+    attn_bwd_prep_kernel<<<static_cast<int>(prep_blocks < 4 * sms ? prep_blocks : 4 * sms), 256, 0, s>>>(
+        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), delta, dq, static_cast<long long>(rows));
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+        return ATTN_ERR_CUDA;
+    const int grid = static_cast<int>(units < sms ? units : sms);
+    attn_bwd_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}

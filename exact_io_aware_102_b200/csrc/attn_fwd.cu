@@ -43,6 +43,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "sm100_ptx.cuh"
 
 namespace {
 
@@ -123,268 +124,6 @@ struct Bars {
     static constexpr int kVFull = 272;     // [8] V ring (split layout)
     static constexpr int kVEmpty = 336;    // [8]
 };
-
-__device__ int g_attn_status = 0;   // 0 = fine; ATTN_ERR_TIMEOUT after a wait ran out
-
-// ---------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// The same test, but a thread whose phase is not complete is suspended (it
-// resumes as soon as the phase completes, or after at most hint_ns) instead
-// of spinning on the issue slots of its sub-partition.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-constexpr uint32_t kWaitSleepNs = 20000;
-
-// Wait until the phase with parity `parity` of barrier `bar` has completed.
-// Gives up after `limit_ns` (then raises the CTA abort flag and the device
-// status word) or as soon as another thread of the CTA has raised the abort
-// flag.  Returns false when it gave up.
-__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                       unsigned long long limit_ns) {
-    const uint64_t t0 = globaltimer_ns();
-    uint32_t n = 0;
-    while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
-        if ((++n & 3u) == 0) {
-            if (abort_flag != nullptr && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > limit_ns) {
-                if (abort_flag != nullptr) *abort_flag = 1u;
-                atomicExch(&g_attn_status, (int)ATTN_ERR_TIMEOUT);
-                return false;
-            }
-        }
-    }
-    return true;
-}
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
-                                             volatile uint32_t* abort_flag,
-                                             unsigned long long limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
-    return wait_slow(bar, parity, abort_flag, limit_ns);
-}
-
-__device__ __forceinline__ void fence_barrier_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
-}
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
-                                            int z, int w) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
-        : "memory");
-}
-
-// tcgen05 (5th-generation tensor core + tensor memory)
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     bar)
-                 : "memory");
-}
-// The same two MMAs with the shared-memory descriptors passed as 32-bit
-// halves: the high word is a per-operand constant and the low word is
-// (address >> 4) | (LBO >> 4) << 16, so stepping an operand is one add.
-__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
-                                          uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "mov.b64 da, {%1, %3};\n\t"
-        "mov.b64 db, {%2, %3};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
-                                          uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "mov.b64 db, {%2, %3};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// 32 lanes x 32 bits, 32 consecutive columns: thread i gets lane (base + i).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
-// Registers written by tcgen05.ld may only be read after tcgen05.wait::ld.
-// This empty volatile asm "redefines" them and is ordered after the wait, so
-// the compiler cannot hoist their uses above it.
-__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
-    asm volatile(""
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
-                   "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
-                   "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
-                   "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
-                   "+r"(r[31]));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-        "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
-// 16 bytes through the read-only path (every thread of a warpgroup reads the
-// same mask bytes: one broadcast transaction, then L1 hits).
-__device__ __forceinline__ uint4 ldg_nc16(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    uint32_t r;
-    // cvt packs its first source into the upper half
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
-template <int R>
-__device__ __forceinline__ void regs_increase() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
-}
-template <int R>
-__device__ __forceinline__ void regs_decrease() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-
-// 2^x for x <= 8 on the FMA/ALU pipes (no MUFU), two lanes at a time:
-// x = j + f with j = round(x) and f in [-1/2, 1/2]; 2^f from a degree-3
-// polynomial fitted for minimal relative error on [-1/2, 1/2]
-// (fit_exp2_poly.py; max relative error 7.6e-5, far below the bf16 rounding
-// that P gets); 2^j by adding j to the exponent field.  x is clamped at -126
-// so the exponent never wraps (2^-126 stands in for 0).
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
-    constexpr float kC0 = 0.99992824f, kC1 = 0.6932636f, kC2 = 0.2426099f, kC3 = 0.05515746f;
-    x.x = fmaxf(x.x, -126.0f);
-    x.y = fmaxf(x.y, -126.0f);
-    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-    const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
-    const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
-    float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-    q = __ffma2_rn(q, f, make_float2(kC1, kC1));
-    q = __ffma2_rn(q, f, make_float2(kC0, kC0));
-    // the low mantissa bits of t hold j (two's complement); t * 2^23 moves them
-    // to the exponent field, added to q in one integer multiply-add
-    uint32_t rx, ry;
-    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rx) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(q.x)));
-    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(ry) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(q.y)));
-    return make_float2(__uint_as_float(rx), __uint_as_float(ry));
-}
-
-// Shared-memory matrix descriptor for the 128-byte swizzle, as two 32-bit
-// words (tcgen05 format): low = start address >> 4 (bits 0-13) | leading
-// byte offset >> 4 (bits 16-29); high = stride byte offset >> 4 (bits 0-13),
-// version 1 (bit 14), layout type 2 = SWIZZLE_128B (bits 29-31).
-__host__ __device__ constexpr uint32_t sdesc_hi_sw128(uint32_t sbo_bytes) {
-    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
-}
-__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
-    return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
-}
-// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, A K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool b_mn_major) {
-    return (1u << 4)                        // D format f32
-           | (1u << 7)                      // A format bf16
-           | (1u << 10)                     // B format bf16
-           | ((b_mn_major ? 1u : 0u) << 16)  // B major
-           | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
-}
 
 // ------------------------------------------------------------- the scheduler
 // Which key tiles a work unit visits.  Full: all of them.  Causal: a Q tile
@@ -1437,6 +1176,9 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, 
 
 }  // namespace
 
+// The backward kernels keep their own status word (attn_bwd.cu).
+int attn_bwd_take_device_status(int* status);
+
 extern "C" {
 
 int attn_version(void) { return 100; }
@@ -1561,10 +1303,12 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
 
 int attn_check_device_status(attn_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
-    int status = 0;
+    int status = 0, bwd_status = 0;
     const int zero = 0;
     if (cudaMemcpyFromSymbol(&status, g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
     if (cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (attn_bwd_take_device_status(&bwd_status) != ATTN_OK) return ATTN_ERR_CUDA;
+    if (status == 0) status = bwd_status;
     return status == 0 ? ATTN_OK : status;
 }
 

@@ -12,7 +12,9 @@ the same shapes stand in):
   [B, H, N, d] and rounded to bf16 (round to nearest even);
 * the stability variant multiplies the bf16 Q by ``q_mult`` (4 is exact in bf16);
 * sampled query rows per (b, h): rows 0 and N-1 plus rows drawn from
-  ``torch.randperm(N)`` seeded with ``1000 + b*H + h``.
+  ``torch.randperm(N)`` seeded with ``1000 + b*H + h``;
+* the upstream gradient dO of the backward: float32 N(0, 1) [B, H, N, d]
+  from its own generator seeded with ``seed``, rounded to bf16.
 """
 import torch
 
@@ -27,6 +29,12 @@ def make_qkv(B, H, N, d, seed=0, q_mult=1.0):
     if q_mult != 1.0:
         q = (q * q_mult).to(torch.bfloat16)
     return q, k, v
+
+
+def make_dout(B, H, N, d, seed=1):
+    """Return a bf16 CPU tensor dO [B, H, N, d] contiguous."""
+    g = torch.Generator().manual_seed(int(seed))
+    return torch.randn((B, H, N, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
 
 
 def sample_rows(B, H, N, count=256):

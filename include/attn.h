@@ -129,6 +129,38 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
                           const unsigned char* block_mask,
                           float scale, int causal, attn_stream_t stream);
 
+/*
+ * attn_bwd -- exact attention backward by recomputation (FlashAttention:
+ * Fast and Memory-Efficient Exact Attention with IO-Awareness, wiki notes,
+ * section "Recomputation": S and P are rebuilt tile by tile from Q, K and the
+ * forward's statistics; no N x N matrix is stored).  Given the upstream
+ * gradient dO of O = softmax(scale Q K^T) V it writes
+ *
+ *     dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO,
+ *     dS = P o (dO V^T - delta),   delta_i = dO_i . O_i.
+ *
+ *   q, k, v, o, dout : bf16 [B, H, N, d], contiguous, 16-byte aligned, read
+ *                      only; o is the attn_fwd output for these q, k, v.
+ *   lse              : fp32 [B, H, N], the attn_fwd LSE, read only.
+ *   delta            : fp32 [B, H, N], written (delta_i above; a workspace
+ *                      the caller owns, useful to nobody else).
+ *   dq               : fp32 [B, H, N, d], written: dQ in fp32 (cleared, then
+ *                      accumulated over key blocks by the call itself).
+ *   dk, dv           : bf16 [B, H, N, d], written.
+ *   d                : 64 (other values return ATTN_ERR_UNSUPPORTED).
+ *   scale, causal, stream, B, H, N : as attn_fwd.
+ *
+ * Pointers must be device memory of the current device covering their
+ * tensors; no output may overlap an input or another output (checked on the
+ * host before anything is launched; ATTN_ERR_INVALID_ARG otherwise).  Two
+ * kernels are queued on `stream` (delta and the dQ clear, then the backward
+ * proper); the library allocates nothing.  Device-side timeouts are reported
+ * by attn_check_device_status().
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, float* delta, float* dq, void* dk, void* dv,
+             int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
+
 /* Human-readable name of an attn_status value (static string, never NULL). */
 const char* attn_status_string(int status);
 

@@ -27,7 +27,8 @@ def lib():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    assert {"attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_status_string", "attn_check_device_status",
+    assert {"attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_bwd", "attn_status_string",
+            "attn_check_device_status",
             "attn_selftest_wait_timeout", "attn_version"} <= set(names)
 
 
@@ -135,6 +136,30 @@ def test_block_mask_checked_on_host(lib):
     assert _sparse(65536, 6 * GIB) not in (pkg.ATTN_ERR_INVALID_ARG, pkg.ATTN_OK)
     # without a mask it is attn_fwd_strided
     assert _sparse(1000, None) not in (pkg.ATTN_ERR_INVALID_ARG, pkg.ATTN_OK)
+
+
+def _bwd(ptrs, N=1000, d=64, scale=0.125):
+    return pkg.attn_bwd(*ptrs, 1, 2, N, d, scale, 0, None)
+
+
+def test_bwd_arguments_checked_on_host(lib):
+    ok = [GIB * (i + 1) for i in range(10)]  # q k v o dout lse delta dq dk dv
+    assert _bwd(ok) not in (pkg.ATTN_ERR_INVALID_ARG, pkg.ATTN_OK)  # reaches the driver
+    assert _bwd(ok, d=128) == pkg.ATTN_ERR_UNSUPPORTED
+    assert _bwd(ok, scale=0.0) == pkg.ATTN_ERR_INVALID_ARG
+    for i in range(10):
+        bad = list(ok)
+        bad[i] = None
+        assert _bwd(bad) == pkg.ATTN_ERR_INVALID_ARG
+    bad = list(ok)
+    bad[7] = ok[0] + 64           # dq overlapping q
+    assert _bwd(bad) == pkg.ATTN_ERR_INVALID_ARG
+    bad = list(ok)
+    bad[9] = ok[8] + 128          # dv overlapping dk
+    assert _bwd(bad) == pkg.ATTN_ERR_INVALID_ARG
+    bad = list(ok)
+    bad[8] += 8                   # dk misaligned
+    assert _bwd(bad) == pkg.ATTN_ERR_INVALID_ARG
 
 
 def test_selftest_limit_validated(lib):

@@ -1,0 +1,108 @@
+"""Parity of the backward (through the C ABI) against the fp64 CPU oracle.
+
+The backward rebuilds P from the forward's LSE and forms dS, dV, dK and dQ
+from bf16 operands with fp32 accumulation (FlashAttention wiki notes, section
+"Recomputation").  Tolerance, per gradient tensor G in {dQ, dK, dV}:
+max|G - G_ref| <= 2e-2 * max|G_ref|, element by element, with G_ref the fp64
+oracle on the same bf16 Q, K, V, dO.  It comes from the arithmetic: P and dS
+enter the tensor core rounded to bf16 (relative 2^-9 each), delta is formed
+from the bf16 O, and dK, dV are returned in bf16 (relative 2^-9); the sums
+over up to N terms of mixed sign keep the error of an element a small
+multiple of 2^-9 of the largest element of its tensor.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_102_b200 as pkg
+import oracle
+from exact_io_aware_102_b200.inputs import make_dout, make_qkv, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 2e-2
+
+
+def run_bwd(B, H, N, causal, seed=0, scale=None):
+    d = 64
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dev = torch.device("cuda:0")
+    q, k, v = make_qkv(B, H, N, d, seed=seed)
+    do = make_dout(B, H, N, d, seed=seed + 100)
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
+    o, lse = pkg.forward(qd, kd, vd, scale=scale, causal=causal)
+    dq, dk, dv = pkg.backward(qd, kd, vd, o, lse, dod, scale=scale, causal=causal)
+    status = pkg.attn_check_device_status()
+    assert status == pkg.ATTN_OK, pkg.attn_status_string(status)
+    return (q, k, v, do), (dq.cpu().numpy(), dk.float().cpu().numpy(), dv.float().cpu().numpy()), scale
+
+
+def compare(got, ref, what):
+    err = np.abs(got - ref).max()
+    bound = REL_TOL * np.abs(ref).max()
+    assert np.isfinite(got).all(), what
+    assert err <= bound, "%s: max err %.3g > %.3g (max |ref| %.3g)" % (what, err, bound, np.abs(ref).max())
+    return err / max(np.abs(ref).max(), 1e-30)
+
+
+def check_full(B, H, N, causal, seed=0):
+    ins, (dq, dk, dv), scale = run_bwd(B, H, N, causal, seed)
+    rq, rk, rv = oracle.attention_bwd_rows(*ins, scale, causal)
+    shape = (B, H, N, 64)
+    return [compare(g, r.reshape(shape), n) for g, r, n in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV"))]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 2, 17, 127, 128, 129, 255, 256, 300, 700])
+def test_bwd_small_sizes_full(N, causal):
+    check_full(1, 2, N, causal, seed=N)
+
+
+def test_bwd_many_heads_and_batches_full():
+    check_full(2, 3, 333, False, seed=7)
+    check_full(2, 3, 333, True, seed=8)
+
+
+def test_bwd_more_units_than_sms_full():
+    # 2 x 40 heads x 8 key blocks = 640 units: every CTA walks several units
+    # and the two Q / dO stages wrap many times
+    check_full(2, 40, 1000, False, seed=9)
+    check_full(2, 40, 1000, True, seed=10)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_image_workload_sampled(causal):
+    # the 3 MP patch self-attention shape; dQ on 64 sampled query rows and
+    # dK, dV on 64 sampled key rows per head
+    B, H, N = 1, 16, 11616
+    ins, (dq, dk, dv), scale = run_bwd(B, H, N, causal, seed=3)
+    qs = sample_rows(B, H, N, 64).numpy()
+    ks = sample_rows(B, H, N, 64).numpy()[:, ::-1].copy()
+    rq, rk, rv = oracle.attention_bwd_rows(*ins, scale, causal, q_rows=qs, k_rows=ks)
+    flat = lambda x: x.reshape(B * H, N, 64)
+    compare(np.take_along_axis(flat(dq), qs[..., None], 1), rq, "dQ")
+    compare(np.take_along_axis(flat(dk), ks[..., None], 1), rk, "dK")
+    compare(np.take_along_axis(flat(dv), ks[..., None], 1), rv, "dV")
+
+
+def test_bwd_gradient_invariants_on_gpu_output():
+    # sum_j dK_j = 0 and <V, dV> = <O, dO> hold for the exact gradient; the
+    # kernel's must hold to within its rounding
+    B, H, N = 1, 4, 900
+    (q, k, v, do), (dq, dk, dv), scale = run_bwd(B, H, N, False, seed=12)
+    o, _ = oracle.attention_full(q.double().numpy(), k.double().numpy(), v.double().numpy(), scale)
+    sum_dk = np.abs(dk.sum(axis=2)).max()
+    assert sum_dk <= 2e-2 * np.abs(dk).max() * math.sqrt(N)
+    lhs = (v.double().numpy() * dv).sum(axis=(2, 3))
+    rhs = (o * do.double().numpy()).sum(axis=(2, 3))
+    assert np.abs(lhs - rhs).max() <= 1e-2 * np.abs(rhs).max() + 1e-3
+
+
+def test_bwd_deterministic_dk_dv():
+    # dK and dV come from one CTA each (no atomics): bit-identical reruns
+    _, (dq1, dk1, dv1), _ = run_bwd(1, 2, 640, True, seed=5)
+    _, (dq2, dk2, dv2), _ = run_bwd(1, 2, 640, True, seed=5)
+    assert np.array_equal(dk1, dk2) and np.array_equal(dv1, dv2)
+    np.testing.assert_allclose(dq1, dq2, rtol=0, atol=1e-5 * np.abs(dq1).max())
