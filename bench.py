@@ -13,7 +13,10 @@ With N > 1 (launched by torch.distributed.run) every rank runs its own
 replica of the workload on its own GPU (the path has no exchange step):
 value = FLOPs of all ranks / the slowest rank's time, scaling "weak".
 ``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample
-of the same workload.
+of the same workload.  ``--pass backward`` times the backward by
+recomputation (attn_bwd: dQ, dK, dV from Q, K, V, O, LSE and a seeded dO) on
+the same workload instead of the forward; it is a secondary line, not the
+headline metric.
 """
 import argparse
 import hashlib
@@ -333,6 +336,72 @@ def run_cuda(args, rank, world, dist):
     return line
 
 
+def bwd_flops(B, H, N, d, causal):
+    """10*B*H*N^2*d: five N x N x d products (S recomputed, dP, dV, dK, dQ), halved causal."""
+    f = 10.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def run_cuda_backward(args, rank, world, dist):
+    import torch
+    import exact_io_aware_102_b200 as pkg
+    from exact_io_aware_102_b200.inputs import make_dout, make_qkv
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    W = WORKLOAD
+    B, H, N, d, causal = W["B"], W["H"], W["N"], W["d"], W["causal"]
+    scale = 1.0 / math.sqrt(d)
+    q, k, v = (x.to(dev) for x in make_qkv(B, H, N, d, seed=0))
+    dout = make_dout(B, H, N, d, seed=1).to(dev)
+    o, lse = pkg.forward(q, k, v, scale=scale, causal=causal)
+    flops = bwd_flops(B, H, N, d, causal)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        pkg.backward(q, k, v, o, lse, dout, scale=scale, causal=causal)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            pkg.backward(q, k, v, o, lse, dout, scale=scale, causal=causal)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    st = pkg.attn_check_device_status()
+    if st != pkg.ATTN_OK:
+        raise RuntimeError("device status: " + pkg.attn_status_string(st))
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_local = sum(step_ms) / len(step_ms)
+    ms = reduce_max(ms_local, dist, dev)
+    peaks = load_peaks()
+    achieved = flops / (ms_local * 1e-3) / 1e12
+    return {
+        "metric": "attn bwd TFLOP/s at H16 N11616 d64 (dQ, dK, dV by recomputation)",
+        "value": round(flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: iid N(0,1) rounded to bf16, Q/K/V seed 0, dO seed 1",
+        "config": {"workload": "%s backward: B=%d H=%d N=%d d=%d %s, bf16 Q/K/V/O/dO/dK/dV, fp32 LSE/dQ" % (
+            W["name"], B, H, N, d, "causal" if causal else "non-causal"),
+            "B": B, "H": H, "N": N, "d": d, "causal": causal, "scale": scale,
+            "l2": "flushed before every timed step (256 MiB write, untimed)",
+            "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                     "peak_kind": "burst bf16 dense, %s" % peaks["source"]},
+        "cpu_baseline": None, "e2e": None, "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(), "step_ms_min": round(min(step_ms), 4), "step_ms_max": round(max(step_ms), 4),
+    }
+
+
 def run_reference(args, rank, world):
     """The fp64 CPU oracle timed on the host cores, each step a bounded sample."""
     from exact_io_aware_102_b200.inputs import make_qkv
@@ -374,6 +443,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
+                    help="time the forward (the headline) or the backward")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -400,7 +471,7 @@ def main(argv=None):
         tdist.init_process_group(backend="nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
     try:
-        line = run_cuda(args, rank, world, dist)
+        line = (run_cuda_backward if args.which == "backward" else run_cuda)(args, rank, world, dist)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
