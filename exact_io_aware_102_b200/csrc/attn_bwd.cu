@@ -17,26 +17,32 @@
 //   * the main kernel runs a persistent grid, one CTA per SM; a work unit is
 //     one (batch, head, 128-key block).  dK and dV of the block accumulate in
 //     TMEM over the query tiles (128 rows each) the block interacts with;
-//   * warp 8 (one lane) loads K, V once per unit and Q_i, dO_i per query tile
-//     (two stages) by TMA; warp 9 (one lane) issues the tcgen05.mma:
+//   * warp 12 (one lane) loads K, V once per unit and Q_i, dO_i per query tile
+//     (two stages) by TMA; warp 13 (one lane) issues the tcgen05.mma:
 //     S^T = K Q_i^T and dP^T = V dO_i^T into TMEM, then dV += P^T dO_i,
 //     dK += dS^T Q_i and the dQ partial dS K_j;
-//   * warps 0-3 (one thread per key row) turn the S^T, dP^T rows into P^T and
-//     dS^T (bf16), written to shared memory in the 128-byte-swizzled layout
-//     the tensor core reads -- one dS^T tile serves dK (K-major) and, read
-//     transposed, dQ (M-major);
-//   * warps 4-7 (one thread per query row) read the dQ partial from TMEM and
+//   * warps 0-7 (two threads per key row: warps 0-3 query columns 0-63, warps
+//     4-7 columns 64-127, so each SM sub-partition runs two of them) turn the
+//     S^T, dP^T rows into P^T (bf16, into TMEM: the A operand of dV) and dS^T
+//     (bf16, into one of two shared-memory buffers in the 128-byte-swizzled
+//     layout the tensor core reads -- one dS^T tile serves dK (K-major) and,
+//     read transposed, dQ (M-major)).  A tile's P^T and dS^T only wait for
+//     dV of the previous tile, so the products of tile i overlap the
+//     elementwise work of tile i+1;
+//   * warps 8-11 (one thread per query row) read the dQ partial from TMEM and
 //     add it to the fp32 dQ accumulator in global memory with bulk
 //     asynchronous reductions (cp.reduce.async.bulk .add.f32), one 256-byte
 //     row per thread;
-//   * at the end of a unit warps 0-3 write dK (times scale) and dV in bf16.
+//   * at the end of a unit warps 0-3 write dV and warps 4-7 dK (times scale)
+//     in bf16.
 //   Every wait is bounded (see sm100_ptx.cuh) and no barrier spans warps
 //   other than mbarriers, so a timeout never leaves a thread blocked.
 //
 // TMEM columns: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
-// dQ [384,448).  Shared memory: K, V (16 KB each), two stages of Q and dO
-// (16 KB each), P^T and dS^T (32 KB each, two 64-column halves), dQ staging
-// rows, per-warp LSE / delta rows, barriers.
+// dQ [384,448), P^T [448,512) (bf16 pairs).  Shared memory: K, V (16 KB
+// each), two stages of Q and dO (16 KB each), two dS^T buffers (32 KB each,
+// two 64-column halves), dQ staging rows, per-warp LSE / delta rows,
+// barriers.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -51,11 +57,14 @@ namespace {
 constexpr int kD = 64;            // head size handled here
 constexpr int kBK = 128;          // keys per unit (= TMEM lanes)
 constexpr int kBQ = 128;          // query rows per tile
-constexpr int kThreads = 320;     // warps 0-3 P/dS, 4-7 dQ, 8 load, 9 MMA
-constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kThreads = 448;     // warps 0-7 P/dS, 8-11 dQ, 12 load, 13 MMA
+constexpr int kPdsWarps = 8;      // two per SM sub-partition: query columns 0-63 and 64-127
+constexpr int kPdsThreads = kPdsWarps * 32;
+constexpr int kDqWarp0 = 8;
+constexpr int kLoadWarp = 12;
+constexpr int kMmaWarp = 13;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384, kColP = 448;
 constexpr float kLog2eB = 1.4426950408889634f;
 constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long kDrainNs = 100000000ull;   // 0.1 s per drain wait
@@ -67,14 +76,14 @@ constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kTile;
 constexpr int kOffQ = kOffV + kTile;          // [2] stages
 constexpr int kOffDO = kOffQ + 2 * kTile;     // [2] stages
-constexpr int kOffP = kOffDO + 2 * kTile;     // P^T, two halves
-constexpr int kOffDS = kOffP + 2 * kHalf;     // dS^T, two halves
-constexpr int kOffStage = kOffDS + 2 * kHalf; // dQ staging: 128 rows x 64 fp32, rows padded
+constexpr int kOffDS = kOffDO + 2 * kTile;    // [2] dS^T buffers, each two 64-column halves
+constexpr int kDsBytes = 2 * kHalf;
+constexpr int kOffStage = kOffDS + 2 * kDsBytes;  // dQ staging: 128 rows x 64 fp32, rows padded
 constexpr int kStageRowBytes = kD * 4 + 16;   // the padding spreads a warp's rows over all banks
 constexpr int kStageWarpBytes = 32 * kStageRowBytes;
-constexpr int kOffRow = kOffStage + 4 * kStageWarpBytes;  // per softmax warp: lse2[128], delta[128]
-constexpr int kRowWarpBytes = 2 * kBQ * 4;
-constexpr int kOffBar = kOffRow + 4 * kRowWarpBytes;
+constexpr int kOffRow = kOffStage + 4 * kStageWarpBytes;  // per P/dS warp: lse2[64], delta[64]
+constexpr int kRowWarpBytes = 2 * 64 * 4;
+constexpr int kOffBar = kOffRow + kPdsWarps * kRowWarpBytes;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
 
 struct Bars {
@@ -82,11 +91,13 @@ struct Bars {
     static constexpr int kQFull = 16;    // [2]
     static constexpr int kQEmpty = 32;   // [2]
     static constexpr int kSFull = 48, kSFree = 56;
-    static constexpr int kPFull = 64, kPFree = 72;
+    static constexpr int kPFull = 64;    // P^T (TMEM) and dS^T (SMEM) of a tile written
+    static constexpr int kPTFree = 72;   // dV of a tile retired: P^T's TMEM columns free
     static constexpr int kDQFull = 80, kDQEmpty = 88;
     static constexpr int kDKVFull = 96, kDKVEmpty = 104;
     static constexpr int kDrain = 112;
-    static constexpr int kTmemSlot = 120, kAbort = 124;
+    static constexpr int kDsFree = 120;  // [2] dK and dQ of a tile retired: its dS^T buffer free
+    static constexpr int kTmemSlot = 136, kAbort = 140;
 };
 
 struct BwdParams {
@@ -195,6 +206,14 @@ struct BwdMma {
             mma_ss_lo(d, a0 + (((kk / 4) * kHalf + (kk % 4) * 32) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi,
                       kIdescKT, (acc || kk > 0) ? 1u : 0u);
     }
+    // D[128 x 64] (+)= A[128 x 128] B[128 x 64]: A bf16 pairs in TMEM (P^T),
+    // B M/N-major
+    __device__ __forceinline__ static void ts(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
+        const uint32_t b0 = sdesc_lo(b, kHalf);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+            mma_ts_lo(d, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), kHi, kIdescKT, (acc || kk > 0) ? 1u : 0u);
+    }
     // D[128 x 64] = A[128 x 128] B[128 x 64] with A stored transposed (the
     // dS^T tile: rows = K, two 64-wide halves of M), B M/N-major
     __device__ __forceinline__ static void tt(uint32_t d, uint32_t a_t, uint32_t b) {
@@ -238,10 +257,12 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
             if (!wait(c.bar + Bars::kDQEmpty, (g & 1) ^ 1)) break;
             tc_fence_after();
             const uint32_t s = g & 1;
-            BwdMma::kt(t + kColDV, c.base + kOffP, c.base + kOffDO + s * kTile, it > 0);  // dV += P^T dO
-            BwdMma::kt(t + kColDK, c.base + kOffDS, c.base + kOffQ + s * kTile, it > 0);  // dK += dS^T Q
-            BwdMma::tt(t + kColDQ, c.base + kOffDS, c.base + kOffK);                        // dQ_j = dS K
-            tc_commit(c.bar + Bars::kPFree);
+            const uint32_t ds = c.base + kOffDS + s * kDsBytes;
+            BwdMma::ts(t + kColDV, t + kColP, c.base + kOffDO + s * kTile, it > 0);  // dV += P^T dO
+            tc_commit(c.bar + Bars::kPTFree);
+            BwdMma::kt(t + kColDK, ds, c.base + kOffQ + s * kTile, it > 0);          // dK += dS^T Q
+            BwdMma::tt(t + kColDQ, ds, c.base + kOffK);                               // dQ_j = dS K
+            tc_commit(c.bar + Bars::kDsFree + 8 * s);
             tc_commit(c.bar + Bars::kQEmpty + 8 * s);
             tc_commit(c.bar + Bars::kDQFull);
             if (it + 1 == n) {
@@ -264,6 +285,16 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int col) {
     return static_cast<uint32_t>(h * kHalf + r * 128 + ((c16 ^ (r & 7)) << 4) + (col & 7) * 2);
 }
 
+// 32 lanes x 16 consecutive 32-bit TMEM columns from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c4, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c4), "r"(d)
                  : "memory");
@@ -274,15 +305,19 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
     return v;
 }
 
-// ---------------------------------------------------------- P / dS warps (0-3)
-// Thread = key row r of the unit's block = TMEM lane r.
+// ---------------------------------------------------------- P / dS warps (0-7)
+// Thread = key row r of the unit's block (TMEM lane r) and one half of the
+// 128 query columns of a tile.
 __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
     const BwdParams& p = c.p;
-    const int r = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_s = c.tmem + lane_off + kColS, t_dp = c.tmem + lane_off + kColDP;
-    const uint32_t t_dv = c.tmem + lane_off + kColDV, t_dk = c.tmem + lane_off + kColDK;
-    const uint32_t rows_smem = c.base + kOffRow + warp * kRowWarpBytes;  // lse2[128], delta[128]
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const int col0 = half * 64;  // first query column of this thread
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_s = c.tmem + lane_off + kColS + col0, t_dp = c.tmem + lane_off + kColDP + col0;
+    const uint32_t t_acc = c.tmem + lane_off + (half == 0 ? kColDV : kColDK);
+    const uint32_t t_p = c.tmem + lane_off + kColP + col0 / 2;  // bf16 pairs
+    const uint32_t rows_smem = c.base + kOffRow + warp * kRowWarpBytes;  // lse2[64], delta[64]
     const float sl2 = p.scale_log2;
     uint32_t g = 0, units = 0;
     bool ok = true;
@@ -292,21 +327,29 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
         const bool key_ok = key < p.N;
         const float* lse_h = p.lse + static_cast<size_t>(w.bh) * p.N;
         const float* dl_h = p.delta + static_cast<size_t>(w.bh) * p.N;
-        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
-            // this warp's copy of LSE * log2(e) and delta for the 128 query
-            // rows of tile i (rows past N: LSE = +inf, delta = 0, so P = dS = 0)
-            __syncwarp();
+        // LSE * log2(e) and delta of this lane's two query rows of tile i
+        // (rows past N: LSE = +inf and delta = 0, so P = dS = 0), fetched one
+        // tile ahead
+        float pre_l[2], pre_d[2];
+        auto fetch = [&](int i) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int q = i * kBQ + lane * 4 + e;
+            for (int e = 0; e < 2; ++e) {
+                const int q = i * kBQ + col0 + lane * 2 + e;
                 const bool in = q < p.N;
-                const float l2 = in ? lse_h[q] * kLog2eB : INFINITY;
-                const float dl = in ? dl_h[q] : 0.f;
-                asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + (lane * 4 + e) * 4), "f"(l2) : "memory");
-                asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + 512 + (lane * 4 + e) * 4), "f"(dl)
-                             : "memory");
+                pre_l[e] = in ? lse_h[q] * kLog2eB : INFINITY;
+                pre_d[e] = in ? dl_h[q] : 0.f;
             }
+        };
+        fetch(w.i0);
+        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
             __syncwarp();
+            asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(rows_smem + lane * 8), "f"(pre_l[0]), "f"(pre_l[1])
+                         : "memory");
+            asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(rows_smem + 256 + lane * 8), "f"(pre_d[0]),
+                         "f"(pre_d[1])
+                         : "memory");
+            __syncwarp();
+            if (i + 1 < p.n_qt) fetch(i + 1);
             bool got = wait_b(c, c.bar + Bars::kSFull, g & 1);
             got = __all_sync(0xffffffffu, got);
             if (!got) {
@@ -314,61 +357,81 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
                 break;
             }
             tc_fence_after();
-            // P^T / dS^T of the previous tile must have been consumed
-            if (g > 0) {
-                got = wait_b(c, c.bar + Bars::kPFree, (g - 1) & 1);
-                got = __all_sync(0xffffffffu, got);
-                if (!got) {
-                    ok = false;
-                    break;
-                }
-            }
             const bool diag = p.causal && i == w.kb;  // causal: query q sees key r iff q >= r
+            // a warp-uniform fast path when no element of the warp's rows is masked
+            const bool masked = __any_sync(0xffffffffu, !key_ok || diag);
+            const uint32_t ds_buf = c.base + kOffDS + (g & 1) * kDsBytes;
 #pragma unroll 1
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 uint32_t sr[32], dr[32];
                 tmem_ld32(t_s + c4 * 32, sr);
                 tmem_ld32(t_dp + c4 * 32, dr);
                 tmem_wait_ld();
                 reg_fence32(sr);
                 reg_fence32(dr);
-                if (c4 == 3) {
+                if (c4 == 1) {
                     tc_fence_before();
                     mbar_arrive(c.bar + Bars::kSFree);  // S^T / dP^T may be overwritten
                 }
                 uint32_t pk[16], dk[16];
+                const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
                 for (int v = 0; v < 8; ++v) {
                     const float4 l2 = ld_shared_f4(rows_smem + (c4 * 32 + v * 4) * 4);
-                    const float4 dl = ld_shared_f4(rows_smem + 512 + (c4 * 32 + v * 4) * 4);
-                    const float lv[4] = {l2.x, l2.y, l2.z, l2.w};
-                    const float dv[4] = {dl.x, dl.y, dl.z, dl.w};
-                    float pp[4], ds[4];
+                    const float4 dl = ld_shared_f4(rows_smem + 256 + (c4 * 32 + v * 4) * 4);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int q = c4 * 32 + v * 4 + e;
-                        float x = ex2(fmaf(__uint_as_float(sr[v * 4 + e]), sl2, -lv[e]));
-                        if (!key_ok || (diag && q < r)) x = 0.f;
-                        pp[e] = x;
-                        ds[e] = x * (__uint_as_float(dr[v * 4 + e]) - dv[e]);
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int e = v * 4 + e2 * 2;
+                        const float2 nl = e2 == 0 ? make_float2(-l2.x, -l2.y) : make_float2(-l2.z, -l2.w);
+                        const float2 nd = e2 == 0 ? make_float2(-dl.x, -dl.y) : make_float2(-dl.z, -dl.w);
+                        float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sl2x2, nl);
+                        x.x = ex2(x.x);
+                        x.y = ex2(x.y);
+                        if (masked) {
+                            const int q = col0 + c4 * 32 + e;
+                            if (!key_ok || (diag && q < r)) x.x = 0.f;
+                            if (!key_ok || (diag && q + 1 < r)) x.y = 0.f;
+                        }
+                        const float2 dsv = __fmul2_rn(
+                            x, __fadd2_rn(make_float2(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), nd));
+                        pk[e >> 1] = pack_bf16x2(x.x, x.y);
+                        dk[e >> 1] = pack_bf16x2(dsv.x, dsv.y);
                     }
-                    pk[v * 2] = pack_bf16x2(pp[0], pp[1]);
-                    pk[v * 2 + 1] = pack_bf16x2(pp[2], pp[3]);
-                    dk[v * 2] = pack_bf16x2(ds[0], ds[1]);
-                    dk[v * 2 + 1] = pack_bf16x2(ds[2], ds[3]);
                 }
+                if (c4 == 0 && g > 0) {
+                    // P^T's TMEM columns: dV of the previous tile must have retired
+                    bool free = wait_b(c, c.bar + Bars::kPTFree, (g - 1) & 1);
+                    free = __all_sync(0xffffffffu, free);
+                    if (!free) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                if (c4 == 0 && g > 1) {
+                    // this dS^T buffer: dK and dQ of tile g-2 must have retired
+                    bool free = wait_b(c, c.bar + Bars::kDsFree + 8 * (g & 1), ((g >> 1) & 1) ^ 1);
+                    free = __all_sync(0xffffffffu, free);
+                    if (!free) {
+                        ok = false;
+                        break;
+                    }
+                }
+                tmem_st16(t_p + c4 * 16, pk);
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
-                    const uint32_t off = sw128_off(r, c4 * 32 + q8 * 8);
-                    st_shared_v4(c.base + kOffP + off, pk[q8 * 4], pk[q8 * 4 + 1], pk[q8 * 4 + 2], pk[q8 * 4 + 3]);
-                    st_shared_v4(c.base + kOffDS + off, dk[q8 * 4], dk[q8 * 4 + 1], dk[q8 * 4 + 2], dk[q8 * 4 + 3]);
+                    const uint32_t off = sw128_off(r, col0 + c4 * 32 + q8 * 8);
+                    st_shared_v4(ds_buf + off, dk[q8 * 4], dk[q8 * 4 + 1], dk[q8 * 4 + 2], dk[q8 * 4 + 3]);
                 }
             }
+            if (!ok) break;
+            tmem_wait_st();
+            tc_fence_before();
             fence_proxy_async();  // the tensor core reads what the generic proxy wrote
             mbar_arrive(c.bar + Bars::kPFull);
         }
         if (!ok) break;
-        // unit epilogue: dK (times scale) and dV of this key row
+        // unit epilogue: dV (warps 0-3) or dK times scale (warps 4-7) of this key row
         bool got = wait_b(c, c.bar + Bars::kDKVFull, units & 1);
         got = __all_sync(0xffffffffu, got);
         if (!got) {
@@ -376,41 +439,35 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             break;
         }
         tc_fence_after();
-        uint32_t a[2][32], b[2][32];
-        tmem_ld32(t_dv, a[0]);
-        tmem_ld32(t_dv + 32, a[1]);
-        tmem_ld32(t_dk, b[0]);
-        tmem_ld32(t_dk + 32, b[1]);
+        uint32_t a[2][32];
+        tmem_ld32(t_acc, a[0]);
+        tmem_ld32(t_acc + 32, a[1]);
         tmem_wait_ld();
         reg_fence32(a[0]);
         reg_fence32(a[1]);
-        reg_fence32(b[0]);
-        reg_fence32(b[1]);
         tc_fence_before();
         mbar_arrive(c.bar + Bars::kDKVEmpty);
         if (key_ok) {
-            const size_t row = (static_cast<size_t>(w.bh) * p.N + key) * kD;
-            uint4* dvr = reinterpret_cast<uint4*>(p.dv + row);
-            uint4* dkr = reinterpret_cast<uint4*>(p.dk + row);
+            const float f = half == 0 ? 1.f : p.scale;
+            uint4* dst = reinterpret_cast<uint4*>((half == 0 ? p.dv : p.dk) +
+                                                  (static_cast<size_t>(w.bh) * p.N + key) * kD);
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int v4 = 0; v4 < 4; ++v4) {
-                    uint32_t x[4], y[4];
+                    uint32_t x[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int cc = v4 * 8 + e * 2;
-                        x[e] = pack_bf16x2(__uint_as_float(a[h][cc]), __uint_as_float(a[h][cc + 1]));
-                        y[e] = pack_bf16x2(__uint_as_float(b[h][cc]) * p.scale, __uint_as_float(b[h][cc + 1]) * p.scale);
+                        x[e] = pack_bf16x2(__uint_as_float(a[h][cc]) * f, __uint_as_float(a[h][cc + 1]) * f);
                     }
-                    dvr[h * 4 + v4] = make_uint4(x[0], x[1], x[2], x[3]);
-                    dkr[h * 4 + v4] = make_uint4(y[0], y[1], y[2], y[3]);
+                    dst[h * 4 + v4] = make_uint4(x[0], x[1], x[2], x[3]);
                 }
         }
     }
 }
 
-// ------------------------------------------------------------- dQ warps (4-7)
+// ------------------------------------------------------------- dQ warps (8-11)
 // Thread = query row of the tile = TMEM lane; each thread stages its row
 // (scaled) in shared memory and adds it to dQ with one bulk reduction.
 __device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
@@ -487,13 +544,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(bar + Bars::kQEmpty + 8 * s, 1);
         }
         mbar_init(bar + Bars::kSFull, 1);
-        mbar_init(bar + Bars::kSFree, kBK);
-        mbar_init(bar + Bars::kPFull, kBK);
-        mbar_init(bar + Bars::kPFree, 1);
+        mbar_init(bar + Bars::kSFree, kPdsThreads);
+        mbar_init(bar + Bars::kPFull, kPdsThreads);
+        mbar_init(bar + Bars::kPTFree, 1);
+        mbar_init(bar + Bars::kDsFree, 1);
+        mbar_init(bar + Bars::kDsFree + 8, 1);
         mbar_init(bar + Bars::kDQFull, 1);
         mbar_init(bar + Bars::kDQEmpty, kBQ);
         mbar_init(bar + Bars::kDKVFull, 1);
-        mbar_init(bar + Bars::kDKVEmpty, kBK);
+        mbar_init(bar + Bars::kDKVEmpty, kPdsThreads);
         mbar_init(bar + Bars::kDrain, 1);
         *abort_flag = 0u;
         fence_barrier_init();
@@ -513,9 +572,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const Ctx ctx{base, bar, *tmem_slot, abort_flag, gbase, p};
-    if (warp < 4) {
+    if (warp < kPdsWarps) {
         role_pds(ctx, warp, lane);
-    } else if (warp < 8) {
+    } else if (warp < kDqWarp0 + 4) {
         role_dq(ctx, warp, lane);
     } else {
         if (lane == 0) {
