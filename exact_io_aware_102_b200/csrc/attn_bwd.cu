@@ -57,7 +57,13 @@ namespace {
 constexpr int kD = 64;            // head size handled here
 constexpr int kBK = 128;          // keys per unit (= TMEM lanes)
 constexpr int kBQ = 128;          // query rows per tile
-constexpr int kThreads = 448;     // warps 0-7 P/dS, 8-11 dQ, 12 load, 13 MMA
+constexpr int kThreads = 512;     // warps 0-7 P/dS, 8-11 dQ, 12 load, 13 MMA, 14-15 idle
+// Register split (setmaxnreg): the block launches with 512 x 128 registers;
+// the two P/dS warpgroups take 160 each, the dQ and load/MMA warpgroups keep
+// 96 (256 x 160 + 256 x 96 = 512 x 128).
+constexpr int kPdsRegs = 160;
+constexpr int kOtherRegs = 96;
+static_assert(256 * kPdsRegs + 256 * kOtherRegs == kThreads * 128, "setmaxnreg split must equal the launch budget");
 constexpr int kPdsWarps = 8;      // two per SM sub-partition: query columns 0-63 and 64-127
 constexpr int kPdsThreads = kPdsWarps * 32;
 constexpr int kDqWarp0 = 8;
@@ -573,10 +579,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const Ctx ctx{base, bar, *tmem_slot, abort_flag, gbase, p};
     if (warp < kPdsWarps) {
+        regs_increase<kPdsRegs>();
         role_pds(ctx, warp, lane);
     } else if (warp < kDqWarp0 + 4) {
+        regs_decrease<kOtherRegs>();
         role_dq(ctx, warp, lane);
     } else {
+        regs_decrease<kOtherRegs>();
         if (lane == 0) {
             if (warp == kLoadWarp) role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do);
             else if (warp == kMmaWarp) role_mma(ctx);
