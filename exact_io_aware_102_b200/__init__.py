@@ -6,7 +6,7 @@ supplies device memory and the current stream.  There is no fallback: if the
 library is missing, every entry point raises.
 
 The C entry points keep their names here (``attn_fwd``, ``attn_fwd_strided``,
-``attn_fwd_block_sparse``, ``attn_bwd``, ``attn_status_string``, ``attn_check_device_status``,
+``attn_fwd_block_sparse``, ``attn_bwd``, ``attn_bwd_noalloc``, ``attn_status_string``, ``attn_check_device_status``,
 ``attn_selftest_wait_timeout``, ``attn_version``); ``forward`` is the tensor
 convenience wrapper and ``backward`` its gradient counterpart.
 """
@@ -15,7 +15,7 @@ import math
 import os
 
 __all__ = [
-    "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_bwd", "attn_status_string", "attn_check_device_status",
+    "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_bwd", "attn_bwd_noalloc", "attn_status_string", "attn_check_device_status",
     "attn_selftest_wait_timeout", "attn_version", "forward", "backward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
 ]
@@ -55,6 +55,8 @@ def library():
                                               i64, vp, vp, ctypes.c_float, i32, vp]
         lib.attn_bwd.restype = i32
         lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, i32, vp]
+        lib.attn_bwd_noalloc.restype = i32
+        lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, i32, vp]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_status_string.argtypes = [i32]
         lib.attn_check_device_status.restype = i32
@@ -98,6 +100,12 @@ def attn_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, N, d, scale, causal
     """Raw C call: device addresses as ints; returns the status."""
     return library().attn_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, int(B), int(H), int(N), int(d),
                               float(scale), int(bool(causal)), stream)
+
+
+def attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, stream):
+    """Raw C call: attn_bwd with delta in the library's static device array (no allocation)."""
+    return library().attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, int(B), int(H), int(N), int(d),
+                                      float(scale), int(bool(causal)), stream)
 
 
 def attn_status_string(status):

@@ -49,6 +49,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "attn.h"
 #include "sm100_ptx.cuh"
 
@@ -698,9 +700,61 @@ int attn_bwd_take_device_status(int* status) {
     return ATTN_OK;
 }
 
+namespace {
+
+// attn_bwd_noalloc's delta rows live here: file-scope static device memory,
+// part of the module image, so that entry point allocates nothing.
+constexpr long long kNoAllocDeltaRows = 1LL << 20;  // B*H*N at most (4 MiB of fp32)
+__device__ __align__(256) float g_noalloc_delta[kNoAllocDeltaRows];
+constexpr int kMaxDevices = 64;
+
+// Device address of g_noalloc_delta on the current device, resolved once
+// per device (cudaGetSymbolAddress); nullptr on failure.
+float* noalloc_delta() {
+    static std::mutex m;
+    static float* addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(m);
+    if (addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_delta) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = static_cast<float*>(ptr);
+    }
+    return addr[dev];
+}
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+             float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+             attn_stream_t stream);
+
+}  // namespace
+
 extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                         const float* lse, float* delta, float* dq, void* dk, void* dv, int B, int H, int N,
                         int d, float scale, int causal, attn_stream_t stream) {
+    return bwd_impl(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, N, d, scale, causal, stream);
+}
+
+extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                const float* lse, float* dq, void* dk, void* dv, int B, int H, int N, int d,
+                                float scale, int causal, attn_stream_t stream) {
+    if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
+    if (static_cast<long long>(B) * H * N > kNoAllocDeltaRows) return ATTN_ERR_INVALID_ARG;
+    if (d != kD) return ATTN_ERR_UNSUPPORTED;
+    float* delta = noalloc_delta();
+    if (delta == nullptr) return ATTN_ERR_CUDA;
+    return bwd_impl(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, N, d, scale, causal, stream);
+}
+
+namespace {
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+             float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+             attn_stream_t stream) {
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
     if (d != kD) return ATTN_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o || !dout || !lse || !delta || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
@@ -773,3 +827,5 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     attn_bwd_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, mdo, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
+
+}  // namespace

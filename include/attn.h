@@ -161,6 +161,25 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              const float* lse, float* delta, float* dq, void* dk, void* dv,
              int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
 
+/*
+ * attn_bwd_noalloc -- attn_bwd without the delta workspace argument: the
+ * call allocates nothing and needs no caller scratch.  The pages have no
+ * counterpart; it exists for callers that may not allocate (for example
+ * inside a captured CUDA graph).
+ *
+ * delta is kept in a static device array of the library (1 << 20 fp32 rows,
+ * 4 MiB, part of the module image), so B*H*N must be at most 1048576
+ * (otherwise ATTN_ERR_INVALID_ARG, checked before anything runs).  Its
+ * address is looked up once per device (cudaGetSymbolAddress) on the first
+ * call on that device: make that first call outside stream capture.  The
+ * array is shared by every call on a device, so calls whose executions may
+ * overlap (different streams without ordering between them) race on it:
+ * order them on one stream or by events.  Everything else as attn_bwd.
+ */
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, float* dq, void* dk, void* dv,
+                     int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
+
 /* Human-readable name of an attn_status value (static string, never NULL). */
 const char* attn_status_string(int status);
 
