@@ -61,10 +61,10 @@ constexpr int kBK = 128;          // keys per unit (= TMEM lanes)
 constexpr int kBQ = 128;          // query rows per tile
 constexpr int kThreads = 512;     // warps 0-7 P/dS, 8-11 dQ, 12 load, 13 MMA, 14-15 idle
 // Register split (setmaxnreg): the block launches with 512 x 128 registers;
-// the two P/dS warpgroups take 160 each, the dQ and load/MMA warpgroups keep
-// 96 (256 x 160 + 256 x 96 = 512 x 128).
-constexpr int kPdsRegs = 160;
-constexpr int kOtherRegs = 96;
+// the two P/dS warpgroups take 176 each, the dQ and load/MMA warpgroups keep
+// 80 (256 x 176 + 256 x 80 = 512 x 128).
+constexpr int kPdsRegs = 176;
+constexpr int kOtherRegs = 80;
 static_assert(256 * kPdsRegs + 256 * kOtherRegs == kThreads * 128, "setmaxnreg split must equal the launch budget");
 constexpr int kPdsWarps = 8;      // two per SM sub-partition: query columns 0-63 and 64-127
 constexpr int kPdsThreads = kPdsWarps * 32;
@@ -369,18 +369,22 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             // a warp-uniform fast path when no element of the warp's rows is masked
             const bool masked = __any_sync(0xffffffffu, !key_ok || diag);
             const uint32_t ds_buf = c.base + kOffDS + (g & 1) * kDsBytes;
-#pragma unroll 1
+            // both 32-column chunks of this thread's S^T and dP^T row, then
+            // release them at once: the next tile's products start now
+            uint32_t sr[2][32], dr[2][32];
+            tmem_ld32(t_s, sr[0]);
+            tmem_ld32(t_s + 32, sr[1]);
+            tmem_ld32(t_dp, dr[0]);
+            tmem_ld32(t_dp + 32, dr[1]);
+            tmem_wait_ld();
+            reg_fence32(sr[0]);
+            reg_fence32(sr[1]);
+            reg_fence32(dr[0]);
+            reg_fence32(dr[1]);
+            tc_fence_before();
+            mbar_arrive(c.bar + Bars::kSFree);  // S^T / dP^T may be overwritten
+#pragma unroll
             for (int c4 = 0; c4 < 2; ++c4) {
-                uint32_t sr[32], dr[32];
-                tmem_ld32(t_s + c4 * 32, sr);
-                tmem_ld32(t_dp + c4 * 32, dr);
-                tmem_wait_ld();
-                reg_fence32(sr);
-                reg_fence32(dr);
-                if (c4 == 1) {
-                    tc_fence_before();
-                    mbar_arrive(c.bar + Bars::kSFree);  // S^T / dP^T may be overwritten
-                }
                 uint32_t pk[16], dk[16];
                 const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
@@ -392,7 +396,8 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
                         const int e = v * 4 + e2 * 2;
                         const float2 nl = e2 == 0 ? make_float2(-l2.x, -l2.y) : make_float2(-l2.z, -l2.w);
                         const float2 nd = e2 == 0 ? make_float2(-dl.x, -dl.y) : make_float2(-dl.z, -dl.w);
-                        float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sl2x2, nl);
+                        float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[c4][e]), __uint_as_float(sr[c4][e + 1])),
+                                              sl2x2, nl);
                         x.x = ex2(x.x);
                         x.y = ex2(x.y);
                         if (masked) {
@@ -401,7 +406,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
                             if (!key_ok || (diag && q + 1 < r)) x.y = 0.f;
                         }
                         const float2 dsv = __fmul2_rn(
-                            x, __fadd2_rn(make_float2(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), nd));
+                            x, __fadd2_rn(make_float2(__uint_as_float(dr[c4][e]), __uint_as_float(dr[c4][e + 1])), nd));
                         pk[e >> 1] = pack_bf16x2(x.x, x.y);
                         dk[e >> 1] = pack_bf16x2(dsv.x, dsv.y);
                     }
@@ -496,24 +501,25 @@ __device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
                 break;
             }
             tc_fence_after();
-            uint32_t a[2][32];
-            tmem_ld32(t_dq, a[0]);
-            tmem_ld32(t_dq + 32, a[1]);
-            tmem_wait_ld();
-            reg_fence32(a[0]);
-            reg_fence32(a[1]);
-            tc_fence_before();
-            mbar_arrive(c.bar + Bars::kDQEmpty);
             if (pending) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             pending = false;
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int h = 0; h < 2; ++h) {
+                uint32_t a[32];
+                tmem_ld32(t_dq + h * 32, a);
+                tmem_wait_ld();
+                reg_fence32(a);
+                if (h == 1) {
+                    tc_fence_before();
+                    mbar_arrive(c.bar + Bars::kDQEmpty);
+                }
 #pragma unroll
                 for (int v4 = 0; v4 < 8; ++v4)
-                    st_shared_v4(my_row + (h * 8 + v4) * 16, __float_as_uint(__uint_as_float(a[h][v4 * 4]) * p.scale),
-                                 __float_as_uint(__uint_as_float(a[h][v4 * 4 + 1]) * p.scale),
-                                 __float_as_uint(__uint_as_float(a[h][v4 * 4 + 2]) * p.scale),
-                                 __float_as_uint(__uint_as_float(a[h][v4 * 4 + 3]) * p.scale));
+                    st_shared_v4(my_row + (h * 8 + v4) * 16, __float_as_uint(__uint_as_float(a[v4 * 4]) * p.scale),
+                                 __float_as_uint(__uint_as_float(a[v4 * 4 + 1]) * p.scale),
+                                 __float_as_uint(__uint_as_float(a[v4 * 4 + 2]) * p.scale),
+                                 __float_as_uint(__uint_as_float(a[v4 * 4 + 3]) * p.scale));
+            }
             fence_proxy_async();
             const int row = i * kBQ + quarter * 32 + lane;
             if (row < p.N) {
