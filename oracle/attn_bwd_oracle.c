@@ -22,8 +22,12 @@
  *     dQ_i  = scale * sum_j dS_ij k_j              (S = scale Q K^T)
  *     dK_j  = scale * sum_i dS_ij q_i
  *
- * Causal: key j is visible to query i iff j <= i.  Rows with no visible key
- * cannot occur (no padding here).  bf16 inputs are widened exactly to fp64.
+ * Causal: key j is visible to query i iff j <= i.  Key padding (the forward
+ * oracle's convention, from flash-attnの代役がVRAMを18GB溶かしていたので87%削った話,
+ * §3 and §6): key_pad NULL or [B, N] bytes, nonzero = padded key, invisible to
+ * every row.  A row with no visible key has O = 0 whatever Q, K, V are, so
+ * its dQ is 0 and it adds nothing to dK, dV.  bf16 inputs are widened
+ * exactly to fp64.
  *
  * Parity status: pinned by the CPU tests (central finite differences, the
  * invariants sum_j dK_j = 0, <Q, dQ> = <K, dK> and <V, dV> = <O, dO>, and a
@@ -49,7 +53,7 @@ static double widen(uint16_t bits) {
  * k_sel likewise for dK and dV.  dq: [n_q, d]; dk, dv: [n_k, d].
  */
 static int bwd_head(const double* qh, const double* kh, const double* vh, const double* doh, int N,
-                    int d, double scale, int causal, const int32_t* q_sel, int n_q,
+                    int d, double scale, int causal, const unsigned char* pad, const int32_t* q_sel, int n_q,
                     const int32_t* k_sel, int n_k, double* dq, double* dk, double* dv, int n_threads) {
     /* position of each row in the selections (-1: not selected) */
     int* q_pos = (int*)malloc(sizeof(int) * (size_t)N);
@@ -87,20 +91,23 @@ static int bwd_head(const double* qh, const double* kh, const double* vh, const 
                 const int visible = causal ? i + 1 : N;
                 const double* qi = qh + (size_t)i * d;
                 const double* doi = doh + (size_t)i * d;
-                /* scores and the softmax row */
+                /* scores and the softmax row (padded keys: P = 0) */
                 double m = -INFINITY;
+                int any = 0;
                 for (int j = 0; j < visible; ++j) {
+                    if (pad && pad[j]) continue;
                     double acc = 0.0;
                     for (int t = 0; t < d; ++t) acc += qi[t] * kh[(size_t)j * d + t];
                     s[j] = scale * acc;
-                    if (s[j] > m) m = s[j];
+                    if (!any || s[j] > m) m = s[j];
+                    any = 1;
                 }
                 double sum = 0.0;
                 for (int j = 0; j < visible; ++j) {
-                    p[j] = exp(s[j] - m);
+                    p[j] = (pad && pad[j]) ? 0.0 : exp(s[j] - m);
                     sum += p[j];
                 }
-                for (int j = 0; j < visible; ++j) p[j] /= sum;
+                for (int j = 0; j < visible; ++j) p[j] = any ? p[j] / sum : 0.0;
                 /* dP and the row term sum_k P_ik dP_ik */
                 double row = 0.0;
                 for (int j = 0; j < visible; ++j) {
@@ -153,14 +160,16 @@ static int sel_ok(const int32_t* sel, long count, int N) {
 
 /*
  * bf16 inputs (raw 16-bit patterns) Q, K, V, dO, layout [B, H, N, d]
- * contiguous.  q_rows: NULL (all rows, n_q must equal N) or int32
+ * contiguous.  key_pad: NULL or [B, N] bytes, nonzero = padded key.
+ * q_rows: NULL (all rows, n_q must equal N) or int32
  * [B*H, n_q], distinct rows per head; k_rows likewise for dK / dV.
  * dq: fp64 [B*H, n_q, d]; dk, dv: fp64 [B*H, n_k, d].
  * Returns 0, -1 on bad arguments, -2 when out of memory.
  */
 int attn_oracle_bwd_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                          const uint16_t* dout, int B, int H, int N, int d, double scale,
-                         int causal, const int32_t* q_rows, int n_q, const int32_t* k_rows,
+                         int causal, const unsigned char* key_pad, const int32_t* q_rows, int n_q,
+                         const int32_t* k_rows,
                          int n_k, double* dq, double* dk, double* dv, int n_threads) {
     if (B < 1 || H < 1 || N < 1 || d < 1 || n_q < 0 || n_k < 0) return -1;
     if ((!q_rows && n_q != N) || (!k_rows && n_k != N)) return -1;
@@ -177,7 +186,8 @@ int attn_oracle_bwd_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v
             vh[e] = widen(v[bh * head + e]);
             doh[e] = widen(dout[bh * head + e]);
         }
-        rc = bwd_head(qh, kh, vh, doh, N, d, scale, causal, q_rows ? q_rows + bh * n_q : NULL, n_q,
+        const unsigned char* pad = key_pad ? key_pad + (size_t)(bh / H) * N : NULL;
+        rc = bwd_head(qh, kh, vh, doh, N, d, scale, causal, pad, q_rows ? q_rows + bh * n_q : NULL, n_q,
                       k_rows ? k_rows + bh * n_k : NULL, n_k, dq + (size_t)bh * n_q * d,
                       dk + (size_t)bh * n_k * d, dv + (size_t)bh * n_k * d, n_threads);
     }
@@ -188,7 +198,8 @@ int attn_oracle_bwd_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v
 /* fp64 inputs, otherwise as attn_oracle_bwd_bf16. */
 int attn_oracle_bwd_f64(const double* q, const double* k, const double* v, const double* dout,
                         int B, int H, int N, int d, double scale, int causal,
-                        const int32_t* q_rows, int n_q, const int32_t* k_rows, int n_k,
+                        const unsigned char* key_pad, const int32_t* q_rows, int n_q,
+                        const int32_t* k_rows, int n_k,
                         double* dq, double* dk, double* dv, int n_threads) {
     if (B < 1 || H < 1 || N < 1 || d < 1 || n_q < 0 || n_k < 0) return -1;
     if ((!q_rows && n_q != N) || (!k_rows && n_k != N)) return -1;
@@ -197,7 +208,8 @@ int attn_oracle_bwd_f64(const double* q, const double* k, const double* v, const
     int rc = 0;
     for (long bh = 0; rc == 0 && bh < (long)B * H; ++bh)
         rc = bwd_head(q + bh * head, k + bh * head, v + bh * head, dout + bh * head, N, d, scale,
-                      causal, q_rows ? q_rows + bh * n_q : NULL, n_q,
+                      causal, key_pad ? key_pad + (size_t)(bh / H) * N : NULL,
+                      q_rows ? q_rows + bh * n_q : NULL, n_q,
                       k_rows ? k_rows + bh * n_k : NULL, n_k, dq + (size_t)bh * n_q * d,
                       dk + (size_t)bh * n_k * d, dv + (size_t)bh * n_k * d, n_threads);
     return rc;

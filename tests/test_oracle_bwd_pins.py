@@ -132,3 +132,80 @@ def test_bwd_oracle_rejects_bad_rows():
         oracle.attention_bwd_rows(q, q, q, q, 1.0, q_rows=np.array([0, 4]))
     with pytest.raises(ValueError):
         oracle.attention_bwd_rows(q, q, q, q, 1.0, k_rows=np.array([1, 1]))
+
+
+# ---- key padding (nonzero = padded key; flash-attnの代役がVRAMを18GB溶かしていたので87%削った話, §3 and §6)
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_padded_finite_differences(causal):
+    N, d, scale = 7, 3, 0.8
+    q, k, v, do = (RNG.normal(size=(2, 1, N, d)) for _ in range(4))
+    pad = np.zeros((2, N), dtype=np.uint8)
+    pad[0, [1, 4]] = 1
+    pad[1, :3] = 1                      # causal: rows 0-2 of batch 1 see nothing
+    dq, dk, dv = (g.reshape(2, 1, N, d) for g in oracle.attention_bwd_rows(q, k, v, do, scale, causal, key_pad=pad))
+
+    def loss():
+        o, _ = oracle.attention_full(q, k, v, scale, causal, key_pad=pad)
+        return float((o * do).sum())
+
+    h = 1e-6
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = x[idx]
+            x[idx] = old + h
+            up = loss()
+            x[idx] = old - h
+            dn = loss()
+            x[idx] = old
+            num[idx] = (up - dn) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=0, atol=2e-8)
+
+
+def test_padded_keys_get_zero_gradients_and_drop_out():
+    # padded keys get dK = dV = 0, and the rest equals the backward of the
+    # problem with the padded keys removed (queries kept)
+    B, H, N, d, scale = 1, 2, 13, 4, 0.6
+    q, k, v, do = (RNG.normal(size=(B, H, N, d)) for _ in range(4))
+    pad = np.zeros((B, N), dtype=np.uint8)
+    pad[0, [0, 5, 6, 12]] = 1
+    keep = np.nonzero(pad[0] == 0)[0]
+    dq, dk, dv = (g.reshape(B, H, N, d) for g in oracle.attention_bwd_rows(q, k, v, do, scale, key_pad=pad))
+    assert (dk[:, :, pad[0] == 1] == 0).all() and (dv[:, :, pad[0] == 1] == 0).all()
+    # the reduced problem: all N queries against the kept keys, through autograd
+    tq = torch.tensor(q, requires_grad=True)
+    tk = torch.tensor(k[:, :, keep], requires_grad=True)
+    tv = torch.tensor(v[:, :, keep], requires_grad=True)
+    o = torch.softmax(scale * tq @ tk.transpose(-1, -2), dim=-1) @ tv
+    o.backward(torch.tensor(do))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk[:, :, keep], tk.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv[:, :, keep], tv.grad.numpy(), rtol=0, atol=1e-12)
+
+
+def test_fully_padded_batch_has_zero_gradients():
+    q, k, v, do = (RNG.normal(size=(2, 2, 9, 3)) for _ in range(4))
+    pad = np.zeros((2, 9), dtype=np.uint8)
+    pad[1] = 1
+    grads = oracle.attention_bwd_rows(q, k, v, do, 0.5, key_pad=pad)
+    for g in grads:
+        assert (g.reshape(2, 2, 9, 3)[1] == 0).all()
+    ref = oracle.attention_bwd_rows(q[:1], k[:1], v[:1], do[:1], 0.5)
+    for g, r in zip(grads, ref):
+        # equal up to the order in which OpenMP threads add their dK, dV parts
+        np.testing.assert_allclose(g.reshape(2, 2, 9, 3)[0], r.reshape(1, 2, 9, 3)[0], rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_padded_c_oracle_matches_numpy_twin(causal):
+    q, k, v = make_qkv(2, 2, 60, 16, seed=51)
+    do = make_qkv(2, 2, 60, 16, seed=52)[0]
+    pad = (np.random.default_rng(3).random((2, 60)) < 0.3).astype(np.uint8)
+    pad[1, :20] = 1
+    got = oracle.attention_bwd_rows(q, k, v, do, 0.25, causal, key_pad=pad)
+    tw = oracle.attention_bwd_full(*(x.double().numpy() for x in (q, k, v, do)), 0.25, causal, key_pad=pad)
+    for a, b in zip(got, tw):
+        np.testing.assert_allclose(a.reshape(b.shape), b, rtol=0, atol=1e-12)
