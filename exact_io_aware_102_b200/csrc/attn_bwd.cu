@@ -109,7 +109,8 @@ struct Bars {
 };
 
 struct BwdParams {
-    int BH, N, n_kb, n_qt, total_units, causal;
+    int BH, H, N, n_kb, n_qt, total_units, causal;
+    const uint8_t* key_pad;  // [B, N] (nonzero = padded key) or null
     float scale, scale_log2;
     const float* lse;     // [BH, N]
     const float* delta;   // [BH, N]
@@ -332,19 +333,21 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++units) {
         const BwdUnit w = bwd_unit(u, p);
         const int key = w.kb * kBK + r;
-        const bool key_ok = key < p.N;
+        // padded keys (and rows past N) take no part: P = dS = 0 on their rows
+        const bool key_ok = key < p.N && (p.key_pad == nullptr || p.key_pad[static_cast<size_t>(w.bh / p.H) * p.N + key] == 0);
         const float* lse_h = p.lse + static_cast<size_t>(w.bh) * p.N;
         const float* dl_h = p.delta + static_cast<size_t>(w.bh) * p.N;
         // LSE * log2(e) and delta of this lane's two query rows of tile i
-        // (rows past N: LSE = +inf and delta = 0, so P = dS = 0), fetched one
-        // tile ahead
+        // (rows past N, and rows that saw no key (LSE = -inf, O = 0): +inf and
+        // delta = 0, so P = dS = 0), fetched one tile ahead
         float pre_l[2], pre_d[2];
         auto fetch = [&](int i) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int q = i * kBQ + col0 + lane * 2 + e;
-                const bool in = q < p.N;
-                pre_l[e] = in ? lse_h[q] * kLog2eB : INFINITY;
+                const float l = q < p.N ? lse_h[q] : -INFINITY;
+                const bool in = l > -INFINITY;
+                pre_l[e] = in ? l * kLog2eB : INFINITY;
                 pre_d[e] = in ? dl_h[q] : 0.f;
             }
         };
@@ -460,7 +463,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
         reg_fence32(a[1]);
         tc_fence_before();
         mbar_arrive(c.bar + Bars::kDKVEmpty);
-        if (key_ok) {
+        if (key < p.N) {  // padded keys store their (zero) rows too
             const float f = half == 0 ? 1.f : p.scale;
             uint4* dst = reinterpret_cast<uint4*>((half == 0 ? p.dv : p.dk) +
                                                   (static_cast<size_t>(w.bh) * p.N + key) * kD);
@@ -734,33 +737,35 @@ float* noalloc_delta() {
 }
 
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-             float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
-             attn_stream_t stream);
+             const unsigned char* key_pad, float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d,
+             float scale, int causal, attn_stream_t stream);
 
 }  // namespace
 
 extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                        const float* lse, float* delta, float* dq, void* dk, void* dv, int B, int H, int N,
-                        int d, float scale, int causal, attn_stream_t stream) {
-    return bwd_impl(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, N, d, scale, causal, stream);
+                        const float* lse, const unsigned char* key_padding_mask, float* delta, float* dq, void* dk,
+                        void* dv, int B, int H, int N, int d, float scale, int causal, attn_stream_t stream) {
+    return bwd_impl(q, k, v, o, dout, lse, key_padding_mask, delta, dq, dk, dv, B, H, N, d, scale, causal, stream);
 }
 
 extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                                const float* lse, float* dq, void* dk, void* dv, int B, int H, int N, int d,
-                                float scale, int causal, attn_stream_t stream) {
+                                const float* lse, const unsigned char* key_padding_mask, float* dq, void* dk,
+                                void* dv, int B, int H, int N, int d, float scale, int causal,
+                                attn_stream_t stream) {
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
     if (static_cast<long long>(B) * H * N > kNoAllocDeltaRows) return ATTN_ERR_INVALID_ARG;
     if (d != kD) return ATTN_ERR_UNSUPPORTED;
     float* delta = noalloc_delta();
     if (delta == nullptr) return ATTN_ERR_CUDA;
-    return bwd_impl(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, N, d, scale, causal, stream);
+    return bwd_impl(q, k, v, o, dout, lse, key_padding_mask, delta, dq, dk, dv, B, H, N, d, scale, causal,
+                    stream);
 }
 
 namespace {
 
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-             float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
-             attn_stream_t stream) {
+             const unsigned char* key_pad, float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d,
+             float scale, int causal, attn_stream_t stream) {
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
     if (d != kD) return ATTN_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o || !dout || !lse || !delta || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
@@ -778,11 +783,13 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     const size_t in_b[6] = {tb, tb, tb, tb, tb, lb};
     const void* outs[4] = {delta, dq, dk, dv};
     const size_t out_b[4] = {lb, qb, tb, tb};
+    const size_t pad_b = static_cast<size_t>(B) * N;
     for (int a = 0; a < 4; ++a) {
         for (int b = 0; b < 6; ++b)
             if (!disjoint(outs[a], out_b[a], ins[b], in_b[b])) return ATTN_ERR_INVALID_ARG;
         for (int b = a + 1; b < 4; ++b)
             if (!disjoint(outs[a], out_b[a], outs[b], out_b[b])) return ATTN_ERR_INVALID_ARG;
+        if (key_pad && !disjoint(outs[a], out_b[a], key_pad, pad_b)) return ATTN_ERR_INVALID_ARG;
     }
     const BwdDriver& drv = bwd_driver();
     if (!drv.ok) return ATTN_ERR_CUDA;
@@ -794,6 +801,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
         if (!span_ok(range, ins[a], in_b[a], dev)) return ATTN_ERR_INVALID_ARG;
     for (int a = 0; a < 4; ++a)
         if (!span_ok(range, outs[a], out_b[a], dev)) return ATTN_ERR_INVALID_ARG;
+    if (key_pad && !span_ok(range, key_pad, pad_b, dev)) return ATTN_ERR_INVALID_ARG;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         return ATTN_ERR_CUDA;
@@ -805,7 +813,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
 
     BwdParams p;
     p.BH = bh;
+    p.H = H;
     p.N = N;
+    p.key_pad = key_pad;
     p.n_kb = (N + kBK - 1) / kBK;
     p.n_qt = (N + kBQ - 1) / kBQ;
     const long long units = BH * p.n_kb;

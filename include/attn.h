@@ -142,6 +142,10 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
  *   q, k, v, o, dout : bf16 [B, H, N, d], contiguous, 16-byte aligned, read
  *                      only; o is the attn_fwd output for these q, k, v.
  *   lse              : fp32 [B, H, N], the attn_fwd LSE, read only.
+ *   key_padding_mask : NULL, or the [B, N] byte mask the forward used
+ *                      (nonzero = padded key): padded keys get dK = dV = 0
+ *                      and no query row attends to them; a row that saw no
+ *                      key (LSE = -inf, O = 0) gets dQ = 0.
  *   delta            : fp32 [B, H, N], written (delta_i above; a workspace
  *                      the caller owns, useful to nobody else).
  *   dq               : fp32 [B, H, N, d], written: dQ in fp32 (cleared, then
@@ -158,7 +162,8 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
  * by attn_check_device_status().
  */
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-             const float* lse, float* delta, float* dq, void* dk, void* dv,
+             const float* lse, const unsigned char* key_padding_mask,
+             float* delta, float* dq, void* dk, void* dv,
              int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
 
 /*
@@ -177,7 +182,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
  * order them on one stream or by events.  Everything else as attn_bwd.
  */
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                     const float* lse, float* dq, void* dk, void* dv,
+                     const float* lse, const unsigned char* key_padding_mask,
+                     float* dq, void* dk, void* dv,
                      int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
 
 /* Human-readable name of an attn_status value (static string, never NULL). */

@@ -138,8 +138,8 @@ def test_block_mask_checked_on_host(lib):
     assert _sparse(1000, None) not in (pkg.ATTN_ERR_INVALID_ARG, pkg.ATTN_OK)
 
 
-def _bwd(ptrs, N=1000, d=64, scale=0.125):
-    return pkg.attn_bwd(*ptrs, 1, 2, N, d, scale, 0, None)
+def _bwd(ptrs, N=1000, d=64, scale=0.125, pad=None):
+    return pkg.attn_bwd(*ptrs, 1, 2, N, d, scale, 0, None, key_padding_mask=pad)
 
 
 def test_bwd_arguments_checked_on_host(lib):
@@ -160,6 +160,8 @@ def test_bwd_arguments_checked_on_host(lib):
     bad = list(ok)
     bad[8] += 8                   # dk misaligned
     assert _bwd(bad) == pkg.ATTN_ERR_INVALID_ARG
+    assert _bwd(ok, pad=ok[7] + 16) == pkg.ATTN_ERR_INVALID_ARG   # mask overlapping dq
+    assert _bwd(ok, pad=GIB * 11) not in (pkg.ATTN_ERR_INVALID_ARG, pkg.ATTN_OK)
 
 
 def test_selftest_limit_validated(lib):

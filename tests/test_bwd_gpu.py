@@ -106,3 +106,36 @@ def test_bwd_deterministic_dk_dv():
     _, (dq2, dk2, dv2), _ = run_bwd(1, 2, 640, True, seed=5)
     assert np.array_equal(dk1, dk2) and np.array_equal(dv1, dv2)
     np.testing.assert_allclose(dq1, dq2, rtol=0, atol=1e-5 * np.abs(dq1).max())
+
+
+# ---- key padding (the forward's mask, nonzero = padded key)
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [300, 700])
+def test_bwd_key_padding_full(N, causal):
+    B, H, d = 4, 2, 64
+    scale = 1.0 / 8
+    dev = torch.device("cuda:0")
+    rng = np.random.default_rng(N)
+    pad = np.zeros((B, N), dtype=bool)
+    pad[0, N - 37:] = True                 # trailing
+    pad[1] = rng.random(N) < 0.3           # scattered
+    pad[2, : N // 2] = True                # leading: causal rows < N/2 see nothing
+    pad[3] = True                          # fully padded batch
+    q, k, v = make_qkv(B, H, N, d, seed=N + 1)
+    do = make_dout(B, H, N, d, seed=N + 2)
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
+    pad_t = torch.as_tensor(pad).to(dev)
+    o, lse = pkg.forward(qd, kd, vd, scale=scale, causal=causal, key_padding_mask=pad_t)
+    dq, dk, dv = pkg.backward(qd, kd, vd, o, lse, dod, scale=scale, causal=causal, key_padding_mask=pad_t)
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    refs = oracle.attention_bwd_rows(q, k, v, do, scale, causal, key_pad=pad.astype(np.uint8))
+    shape = (B, H, N, d)
+    for g, r, name in zip((dq, dk, dv), refs, ("dQ", "dK", "dV")):
+        g = g.float().cpu().numpy()
+        assert np.isfinite(g).all(), name
+        compare(g, r.reshape(shape), name)
+    # padded keys: exactly zero dK, dV; the fully padded batch: all zero
+    dk_n, dv_n = dk.float().cpu().numpy(), dv.float().cpu().numpy()
+    assert (dk_n[:, :, :][np.broadcast_to(pad[:, None, :], (B, H, N))] == 0).all()
+    assert (dv_n[np.broadcast_to(pad[:, None, :], (B, H, N))] == 0).all()
+    assert (dq[3] == 0).all()
