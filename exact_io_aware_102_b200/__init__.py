@@ -211,10 +211,10 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None, 
 def backward(q, k, v, o, lse, dout, scale=None, causal=False, stream=None, key_padding_mask=None):
     """Gradients of ``forward`` for the upstream gradient ``dout``.
 
-    q, k, v, o, dout: contiguous bf16 CUDA tensors [B, H, N, 64] (o and lse
+    q, k, v, o, dout: contiguous bf16 CUDA tensors [B, H, N, d], d = 64 or 128 (o and lse
     from ``forward`` on the same q, k, v, scale, causal and
     ``key_padding_mask``, a bool / uint8 CUDA tensor [B, N] or None).  Returns
-    (dq fp32, dk bf16, dv bf16), each [B, H, N, 64].  Asynchronous on
+    (dq fp32, dk bf16, dv bf16), each [B, H, N, d].  Asynchronous on
     ``stream`` (default: the current stream).
     """
     import torch

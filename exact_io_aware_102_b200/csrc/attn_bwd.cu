@@ -1,4 +1,4 @@
-// Exact attention backward for B200 (sm_100a), head size 64.
+// Exact attention backward for B200 (sm_100a), head sizes 64 and 128.
 //
 // What is computed (FlashAttention: Fast and Memory-Efficient Exact Attention
 // with IO-Awareness, wiki notes, section "Recomputation"): the forward kept
@@ -612,16 +612,17 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 }
 
 // delta[row] = sum_t dO[row, t] * O[row, t] (fp32), and the dQ accumulator
-// cleared; one thread per row.
+// cleared; one thread per row of D elements.
+template <int D>
 __global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                      float* __restrict__ delta, float* __restrict__ dq, long long rows) {
     for (long long row = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; row < rows;
          row += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const uint4* a = reinterpret_cast<const uint4*>(o + row * kD);
-        const uint4* b = reinterpret_cast<const uint4*>(dout + row * kD);
+        const uint4* a = reinterpret_cast<const uint4*>(o + row * D);
+        const uint4* b = reinterpret_cast<const uint4*>(dout + row * D);
         float acc = 0.f;
 #pragma unroll
-        for (int v = 0; v < kD / 8; ++v) {
+        for (int v = 0; v < D / 8; ++v) {
             const uint4 x = a[v], y = b[v];
             const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
@@ -631,11 +632,473 @@ __global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint1
             }
         }
         delta[row] = acc;
-        float4* z = reinterpret_cast<float4*>(dq + row * kD);
+        float4* z = reinterpret_cast<float4*>(dq + row * D);
 #pragma unroll
-        for (int v = 0; v < kD / 4; ++v) z[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int v = 0; v < D / 4; ++v) z[v] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
+
+// ============================================================== head size 128
+// The same backward at d = 128 with 64-row query tiles, so that TMEM holds
+// dV and dK (128 columns each): S^T [0,64), dP^T [64,128), dV [128,256),
+// dK [256,384), dQ^T [384,448), P^T [448,480).  dQ is formed transposed,
+// dQ^T = K^T dS^T (M = 128 over the head dimension), because a 64-row dQ tile
+// would need the M = 64 accumulator shape; warps 8-11 (one thread per head
+// column) write it transposed into a [64 x 128] fp32 staging tile, which one
+// bulk reduction (32 KB, contiguous in dQ) adds to the accumulator.
+namespace b128 {
+
+constexpr int kD = 128;
+constexpr int kBQ = 64;                     // query rows per tile
+constexpr uint32_t kColS = 0, kColDP = 64, kColDV = 128, kColDK = 256, kColDQ = 384, kColP = 448;
+constexpr int kKHalf = 128 * 64 * 2;        // a [128 x 64] bf16 half of the K or V tile
+constexpr int kQHalf = 64 * 64 * 2;         // a [64 x 64] bf16 half of a Q or dO tile
+constexpr int kKTile = 2 * kKHalf;
+constexpr int kQTile = 2 * kQHalf;
+constexpr int kDsTile = 128 * 64 * 2;       // dS^T [128 keys x 64 queries], one 128-byte-swizzled half
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kKTile;
+constexpr int kOffQ = kOffV + kKTile;       // [2] stages
+constexpr int kOffDO = kOffQ + 2 * kQTile;  // [2] stages
+constexpr int kOffDS = kOffDO + 2 * kQTile; // [2] dS^T buffers
+constexpr int kOffStage = kOffDS + 2 * kDsTile;  // dQ staging: [64 rows x 128] fp32, row-major
+constexpr int kStageBytes = kBQ * kD * 4;
+constexpr int kOffRow = kOffStage + kStageBytes;  // per P/dS warp: lse2[32], delta[32]
+constexpr int kRowWarpBytes = 2 * 32 * 4;
+constexpr int kOffBar = kOffRow + kPdsWarps * kRowWarpBytes;
+constexpr int kSmemBytes = kOffBar + 256 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+struct Bars {
+    static constexpr int kKVFull = 0, kKVEmpty = 8;
+    static constexpr int kQFull = 16, kQEmpty = 32;  // [2] each
+    static constexpr int kSFull = 48, kSFree = 56;
+    static constexpr int kPFull = 64, kPTFree = 72;
+    static constexpr int kDQFull = 80, kDQEmpty = 88;
+    static constexpr int kDKVFull = 96, kDKVEmpty = 104;
+    static constexpr int kDrain = 112;
+    static constexpr int kDsFree = 120;              // [2]
+    static constexpr int kStageFull = 136;           // 128 dQ threads wrote the staging tile
+    static constexpr int kStageFree = 144;           // its bulk reduction has read it
+    static constexpr int kTmemSlot = 152, kAbort = 156;
+};
+
+// Causal: key block kb (keys 128 kb ..) meets 64-row query tiles 2 kb ..
+__device__ __forceinline__ BwdUnit unit(int u, const BwdParams& p) {
+    BwdUnit w = bwd_unit(u, p);
+    if (p.causal) w.i0 = 2 * w.kb;
+    return w;
+}
+
+__device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, const CUtensorMap* tk,
+                                          const CUtensorMap* tv, const CUtensorMap* tdo) {
+    const BwdParams& p = c.p;
+    uint32_t g = 0, units = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        const BwdUnit w = unit(u, p);
+        if (!wait_b(c, c.bar + Bars::kKVEmpty, (units & 1) ^ 1)) {
+            ok = false;
+            break;
+        }
+        mbar_expect_tx(c.bar + Bars::kKVFull, 2 * kKTile);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(c.base + kOffK + x * kKHalf, tk, c.bar + Bars::kKVFull, x * 64, w.kb * 128, w.bh, 0);
+            tma_load_4d(c.base + kOffV + x * kKHalf, tv, c.bar + Bars::kKVFull, x * 64, w.kb * 128, w.bh, 0);
+        }
+        ++units;
+        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+            const uint32_t s = g & 1;
+            if (!wait_b(c, c.bar + Bars::kQEmpty + 8 * s, ((g >> 1) & 1) ^ 1)) {
+                ok = false;
+                break;
+            }
+            const uint32_t fb = c.bar + Bars::kQFull + 8 * s;
+            mbar_expect_tx(fb, 2 * kQTile);
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                tma_load_4d(c.base + kOffQ + s * kQTile + x * kQHalf, tq, fb, x * 64, i * kBQ, w.bh, 0);
+                tma_load_4d(c.base + kOffDO + s * kQTile + x * kQHalf, tdo, fb, x * 64, i * kBQ, w.bh, 0);
+            }
+        }
+    }
+    if (!ok) {
+        if (units > 0) wait_bounded(c.bar + Bars::kKVFull, (units - 1) & 1, nullptr, kDrainNs);
+        for (uint32_t k = (g > 2 ? g - 2 : 0); k < g; ++k)
+            wait_bounded(c.bar + Bars::kQFull + 8 * (k & 1), (k >> 1) & 1, nullptr, kDrainNs);
+    }
+}
+
+struct Mma {
+    static constexpr uint32_t kHi = sdesc_hi_sw128(1024);
+    static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, false);                 // S^T, dP^T
+    static constexpr uint32_t kIdescKV = idesc_bf16_f32(128, 128, true);                // dV, dK
+    static constexpr uint32_t kIdescQ = idesc_bf16_f32(128, 64, true) | (1u << 15);     // dQ^T
+    // D[128 x 64] = A[128 x 128] B[64 x 128]^T: A a K / V tile, B a Q / dO tile,
+    // both K-major in two 64-column halves
+    __device__ __forceinline__ static void nt(uint32_t d, uint32_t a, uint32_t b) {
+        const uint32_t a0 = sdesc_lo(a, 16), b0 = sdesc_lo(b, 16);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+            mma_ss_lo(d, a0 + (((kk / 4) * kKHalf + (kk % 4) * 32) >> 4),
+                      b0 + (((kk / 4) * kQHalf + (kk % 4) * 32) >> 4), kHi, kIdescS, kk > 0 ? 1u : 0u);
+    }
+    // dV (+)= P^T dO: A = P^T bf16 pairs in TMEM (K = 64 queries), B = the dO
+    // tile M/N-major (N = 128 over two 64-column halves)
+    __device__ __forceinline__ static void pv(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
+        const uint32_t b0 = sdesc_lo(b, kQHalf);
+#pragma unroll
+        for (int kk = 0; kk < kBQ / 16; ++kk)
+            mma_ts_lo(d, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), kHi, kIdescKV, (acc || kk > 0) ? 1u : 0u);
+    }
+    // dK (+)= dS^T Q: A = dS^T K-major (one 64-wide half), B = the Q tile M/N-major
+    __device__ __forceinline__ static void dsq(uint32_t d, uint32_t a, uint32_t b, bool acc) {
+        const uint32_t a0 = sdesc_lo(a, 16), b0 = sdesc_lo(b, kQHalf);
+#pragma unroll
+        for (int kk = 0; kk < kBQ / 16; ++kk)
+            mma_ss_lo(d, a0 + ((kk * 32) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi, kIdescKV, (acc || kk > 0) ? 1u : 0u);
+    }
+    // dQ^T = K^T dS^T: A = the K tile read M-major (M = 128 head columns over two
+    // halves, K = 128 keys), B = dS^T M/N-major (N = 64 queries)
+    __device__ __forceinline__ static void kds(uint32_t d, uint32_t a, uint32_t b) {
+        const uint32_t a0 = sdesc_lo(a, kKHalf), b0 = sdesc_lo(b, kDsTile);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+            mma_ss_lo(d, a0 + ((kk * 16 * 128) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi, kIdescQ, kk > 0 ? 1u : 0u);
+    }
+};
+
+__device__ __forceinline__ void role_mma(const Ctx& c) {
+    const BwdParams& p = c.p;
+    const uint32_t t = c.tmem;
+    bool ok = true;
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+        if (ok && !wait_b(c, bar, parity)) ok = false;
+        return ok;
+    };
+    uint32_t g = 0, units = 0;
+    auto issue_s = [&](uint32_t gg) {
+        const uint32_t s = gg & 1;
+        if (!wait(c.bar + Bars::kQFull + 8 * s, (gg >> 1) & 1)) return;
+        if (gg > 0 && !wait(c.bar + Bars::kSFree, (gg - 1) & 1)) return;
+        tc_fence_after();
+        Mma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kQTile);
+        Mma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kQTile);
+        tc_commit(c.bar + Bars::kSFull);
+    };
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++units) {
+        const BwdUnit w = unit(u, p);
+        const int n = p.n_qt - w.i0;
+        if (!wait(c.bar + Bars::kKVFull, units & 1)) break;
+        issue_s(g);
+        for (int it = 0; ok && it < n; ++it, ++g) {
+            if (it + 1 < n) issue_s(g + 1);
+            if (!wait(c.bar + Bars::kPFull, g & 1)) break;
+            if (it == 0 && !wait(c.bar + Bars::kDKVEmpty, (units & 1) ^ 1)) break;
+            tc_fence_after();
+            const uint32_t s = g & 1, ds = c.base + kOffDS + s * kDsTile;
+            Mma::pv(t + kColDV, t + kColP, c.base + kOffDO + s * kQTile, it > 0);   // dV += P^T dO
+            tc_commit(c.bar + Bars::kPTFree);
+            Mma::dsq(t + kColDK, ds, c.base + kOffQ + s * kQTile, it > 0);         // dK += dS^T Q
+            if (!wait(c.bar + Bars::kDQEmpty, (g & 1) ^ 1)) break;
+            tc_fence_after();
+            Mma::kds(t + kColDQ, c.base + kOffK, ds);                                // dQ^T = K^T dS^T
+            tc_commit(c.bar + Bars::kDsFree + 8 * s);
+            tc_commit(c.bar + Bars::kQEmpty + 8 * s);
+            tc_commit(c.bar + Bars::kDQFull);
+            if (it + 1 == n) {
+                tc_commit(c.bar + Bars::kDKVFull);
+                tc_commit(c.bar + Bars::kKVEmpty);
+            }
+        }
+    }
+    if (!ok) {
+        tc_commit(c.bar + Bars::kDrain);
+        wait_bounded(c.bar + Bars::kDrain, 0, nullptr, kDrainNs);
+    }
+}
+
+// Thread = key row r (TMEM lane) and 32 of the tile's 64 query columns.
+__device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
+    const BwdParams& p = c.p;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const int col0 = half * 32;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_s = c.tmem + lane_off + kColS + col0, t_dp = c.tmem + lane_off + kColDP + col0;
+    const uint32_t t_p = c.tmem + lane_off + kColP + col0 / 2;
+    const uint32_t t_acc = c.tmem + lane_off + (half == 0 ? kColDV : kColDK);
+    const uint32_t rows_smem = c.base + kOffRow + warp * kRowWarpBytes;  // lse2[32], delta[32]
+    const float sl2 = p.scale_log2;
+    uint32_t g = 0, units = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++units) {
+        const BwdUnit w = unit(u, p);
+        const int key = w.kb * 128 + r;
+        const bool key_ok = key < p.N && (p.key_pad == nullptr || p.key_pad[static_cast<size_t>(w.bh / p.H) * p.N + key] == 0);
+        const float* lse_h = p.lse + static_cast<size_t>(w.bh) * p.N;
+        const float* dl_h = p.delta + static_cast<size_t>(w.bh) * p.N;
+        float pre_l, pre_d;
+        auto fetch = [&](int i) {
+            const int q = i * kBQ + col0 + lane;
+            const float l = q < p.N ? lse_h[q] : -INFINITY;
+            const bool in = l > -INFINITY;
+            pre_l = in ? l * kLog2eB : INFINITY;
+            pre_d = in ? dl_h[q] : 0.f;
+        };
+        fetch(w.i0);
+        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+            __syncwarp();
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + lane * 4), "f"(pre_l) : "memory");
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + 128 + lane * 4), "f"(pre_d) : "memory");
+            __syncwarp();
+            if (i + 1 < p.n_qt) fetch(i + 1);
+            bool got = wait_b(c, c.bar + Bars::kSFull, g & 1);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sr[32], dr[32];
+            tmem_ld32(t_s, sr);
+            tmem_ld32(t_dp, dr);
+            tmem_wait_ld();
+            reg_fence32(sr);
+            reg_fence32(dr);
+            tc_fence_before();
+            mbar_arrive(c.bar + Bars::kSFree);
+            // causal: query 64 i + col sees key 128 kb + r iff it is not smaller
+            const bool diag = p.causal && (i >> 1) == w.kb;
+            const bool masked = __any_sync(0xffffffffu, !key_ok || diag);
+            const int qbase = i * kBQ + col0 - w.kb * 128;  // query minus key block start
+            uint32_t pk[16], dk[16];
+            const float2 sl2x2 = make_float2(sl2, sl2);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const float4 l2 = ld_shared_f4(rows_smem + v * 16);
+                const float4 dl = ld_shared_f4(rows_smem + 128 + v * 16);
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const int e = v * 4 + e2 * 2;
+                    const float2 nl = e2 == 0 ? make_float2(-l2.x, -l2.y) : make_float2(-l2.z, -l2.w);
+                    const float2 nd = e2 == 0 ? make_float2(-dl.x, -dl.y) : make_float2(-dl.z, -dl.w);
+                    float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sl2x2, nl);
+                    x.x = ex2(x.x);
+                    x.y = ex2(x.y);
+                    if (masked) {
+                        if (!key_ok || (diag && qbase + e < r)) x.x = 0.f;
+                        if (!key_ok || (diag && qbase + e + 1 < r)) x.y = 0.f;
+                    }
+                    const float2 dsv =
+                        __fmul2_rn(x, __fadd2_rn(make_float2(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), nd));
+                    pk[e >> 1] = pack_bf16x2(x.x, x.y);
+                    dk[e >> 1] = pack_bf16x2(dsv.x, dsv.y);
+                }
+            }
+            if (g > 0) {
+                bool free = wait_b(c, c.bar + Bars::kPTFree, (g - 1) & 1);
+                free = __all_sync(0xffffffffu, free);
+                if (!free) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            if (g > 1) {
+                bool free = wait_b(c, c.bar + Bars::kDsFree + 8 * (g & 1), ((g >> 1) & 1) ^ 1);
+                free = __all_sync(0xffffffffu, free);
+                if (!free) {
+                    ok = false;
+                    break;
+                }
+            }
+            tmem_st16(t_p, pk);
+            const uint32_t ds_buf = c.base + kOffDS + (g & 1) * kDsTile;
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+                const uint32_t off = sw128_off(r, col0 + q8 * 8);
+                st_shared_v4(ds_buf + off, dk[q8 * 4], dk[q8 * 4 + 1], dk[q8 * 4 + 2], dk[q8 * 4 + 3]);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            fence_proxy_async();
+            mbar_arrive(c.bar + Bars::kPFull);
+        }
+        if (!ok) break;
+        // unit epilogue: dV (warps 0-3) or dK times scale (warps 4-7), 32 columns at a time
+        bool got = wait_b(c, c.bar + Bars::kDKVFull, units & 1);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        const float f = half == 0 ? 1.f : p.scale;
+        uint4* dst = reinterpret_cast<uint4*>((half == 0 ? p.dv : p.dk) + (static_cast<size_t>(w.bh) * p.N + key) * kD);
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t a[32];
+            tmem_ld32(t_acc + c4 * 32, a);
+            tmem_wait_ld();
+            reg_fence32(a);
+            if (c4 == 3) {
+                tc_fence_before();
+                mbar_arrive(c.bar + Bars::kDKVEmpty);
+            }
+            if (key < p.N) {
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4) {
+                    uint32_t x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        x[e] = pack_bf16x2(__uint_as_float(a[v4 * 8 + e * 2]) * f, __uint_as_float(a[v4 * 8 + e * 2 + 1]) * f);
+                    dst[c4 * 4 + v4] = make_uint4(x[0], x[1], x[2], x[3]);
+                }
+            }
+        }
+    }
+}
+
+// Thread = head column t (TMEM lane) of dQ^T; writes column t of the [64 x 128]
+// staging tile; one thread adds the tile to dQ with one bulk reduction.
+__device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
+    const BwdParams& p = c.p;
+    const int quarter = warp & 3;
+    const int col = quarter * 32 + lane;
+    const uint32_t t_dq = c.tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColDQ;
+    const uint32_t stage = c.base + kOffStage;
+    const bool issuer = warp == kDqWarp0 && lane == 0;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        const BwdUnit w = unit(u, p);
+        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+            bool got = wait_b(c, c.bar + Bars::kDQFull, g & 1);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            got = wait_b(c, c.bar + Bars::kStageFree, (g & 1) ^ 1);  // the previous reduction has read it
+            got = __all_sync(0xffffffffu, got);
+            if (!got) {
+                ok = false;
+                break;
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t a[32];
+                tmem_ld32(t_dq + h * 32, a);
+                tmem_wait_ld();
+                reg_fence32(a);
+                if (h == 1) {
+                    tc_fence_before();
+                    mbar_arrive(c.bar + Bars::kDQEmpty);
+                }
+#pragma unroll
+                for (int q = 0; q < 32; ++q)
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(stage + (h * 32 + q) * (kD * 4) + col * 4),
+                                 "f"(__uint_as_float(a[q]) * p.scale)
+                                 : "memory");
+            }
+            fence_proxy_async();
+            mbar_arrive(c.bar + Bars::kStageFull);
+            if (issuer) {
+                if (wait_b(c, c.bar + Bars::kStageFull, g & 1)) {
+                    const int rows = min(kBQ, p.N - i * kBQ);
+                    float* dst = p.dq + (static_cast<size_t>(w.bh) * p.N + static_cast<size_t>(i) * kBQ) * kD;
+                    asm volatile(
+                        "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+                        "r"(stage), "r"(static_cast<uint32_t>(rows * kD * 4))
+                        : "memory");
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    mbar_arrive(c.bar + Bars::kStageFree);
+                } else {
+                    ok = false;
+                }
+            }
+            ok = __all_sync(0xffffffffu, ok);
+        }
+    }
+    if (issuer) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* const gbase = smem_raw + (base - raw);
+    const uint32_t bar = base + kOffBar;
+    volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + kOffBar + Bars::kAbort);
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + Bars::kTmemSlot);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(bar + Bars::kKVFull, 1);
+        mbar_init(bar + Bars::kKVEmpty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar + Bars::kQFull + 8 * s, 1);
+            mbar_init(bar + Bars::kQEmpty + 8 * s, 1);
+            mbar_init(bar + Bars::kDsFree + 8 * s, 1);
+        }
+        mbar_init(bar + Bars::kSFull, 1);
+        mbar_init(bar + Bars::kSFree, kPdsThreads);
+        mbar_init(bar + Bars::kPFull, kPdsThreads);
+        mbar_init(bar + Bars::kPTFree, 1);
+        mbar_init(bar + Bars::kDQFull, 1);
+        mbar_init(bar + Bars::kDQEmpty, 128);
+        mbar_init(bar + Bars::kDKVFull, 1);
+        mbar_init(bar + Bars::kDKVEmpty, kPdsThreads);
+        mbar_init(bar + Bars::kDrain, 1);
+        mbar_init(bar + Bars::kStageFull, 128);
+        mbar_init(bar + Bars::kStageFree, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+        fence_proxy_async();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const Ctx ctx{base, bar, *tmem_slot, abort_flag, gbase, p};
+    if (warp < kPdsWarps) {
+        regs_increase<kPdsRegs>();
+        b128::role_pds(ctx, warp, lane);
+    } else if (warp < kDqWarp0 + 4) {
+        regs_decrease<kOtherRegs>();
+        b128::role_dq(ctx, warp, lane);
+    } else {
+        regs_decrease<kOtherRegs>();
+        if (lane == 0) {
+            if (warp == kLoadWarp) b128::role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do);
+            else if (warp == kMmaWarp) b128::role_mma(ctx);
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(ctx.tmem, kTmemCols);
+    }
+}
+
+}  // namespace b128
 
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -666,14 +1129,14 @@ const BwdDriver& bwd_driver() {
     return fns;
 }
 
-// bf16 [BH, N, 64] contiguous as a 4-D (64, N, BH, 1) map, box 64 x 128, 128-byte swizzle,
-// rows past N read as zeros.
-bool encode_map(EncodeTiledFn enc, CUtensorMap* map, const void* ptr, int BH, int N) {
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(N),
+// bf16 [BH, N, d] contiguous as a 4-D (d, N, BH, 1) map, box 64 columns x
+// box_rows rows, 128-byte swizzle, rows past N read as zeros.
+bool encode_map(EncodeTiledFn enc, CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_rows) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                                 static_cast<cuuint64_t>(BH), 1};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(N) * kD * 2,
-                                   static_cast<cuuint64_t>(BH) * N * kD * 2};
-    const cuuint32_t box[4] = {64, 128, 1, 1};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2,
+                                   static_cast<cuuint64_t>(BH) * N * d * 2};
+    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -754,7 +1217,7 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
                                 attn_stream_t stream) {
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
     if (static_cast<long long>(B) * H * N > kNoAllocDeltaRows) return ATTN_ERR_INVALID_ARG;
-    if (d != kD) return ATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     float* delta = noalloc_delta();
     if (delta == nullptr) return ATTN_ERR_CUDA;
     return bwd_impl(q, k, v, o, dout, lse, key_padding_mask, delta, dq, dk, dv, B, H, N, d, scale, causal,
@@ -767,17 +1230,17 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
              const unsigned char* key_pad, float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d,
              float scale, int causal, attn_stream_t stream) {
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
-    if (d != kD) return ATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o || !dout || !lse || !delta || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
     if (!isfinite(scale) || !(scale >= 1e-30f)) return ATTN_ERR_INVALID_ARG;
     const long long BH = static_cast<long long>(B) * H;
-    if (BH > 0x7fffffffLL || N > 0x7fffffff - kBQ || BH * N > (1LL << 40) / kD) return ATTN_ERR_INVALID_ARG;
+    if (BH > 0x7fffffffLL || N > 0x7fffffff - 128 || BH * N > (1LL << 40) / d) return ATTN_ERR_INVALID_ARG;
     auto mis = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
     if (mis(q, 16) || mis(k, 16) || mis(v, 16) || mis(o, 16) || mis(dout, 16) || mis(dk, 16) || mis(dv, 16) ||
         mis(dq, 16) || mis(lse, 4) || mis(delta, 4))
         return ATTN_ERR_INVALID_ARG;
     const size_t rows = static_cast<size_t>(BH) * N;
-    const size_t tb = rows * kD * 2, qb = rows * kD * 4, lb = rows * 4;
+    const size_t tb = rows * d * 2, qb = rows * d * 4, lb = rows * 4;
     // outputs must not overlap any input or each other
     const void* ins[6] = {q, k, v, o, dout, lse};
     const size_t in_b[6] = {tb, tb, tb, tb, tb, lb};
@@ -807,8 +1270,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
         return ATTN_ERR_CUDA;
     alignas(64) CUtensorMap mq, mk, mv, mdo;
     const int bh = static_cast<int>(BH);
-    if (!encode_map(enc, &mq, q, bh, N) || !encode_map(enc, &mk, k, bh, N) || !encode_map(enc, &mv, v, bh, N) ||
-        !encode_map(enc, &mdo, dout, bh, N))
+    const int q_rows = d == 64 ? kBQ : b128::kBQ;  // query rows per tile (the Q / dO box)
+    if (!encode_map(enc, &mq, q, bh, N, d, q_rows) || !encode_map(enc, &mk, k, bh, N, d, kBK) ||
+        !encode_map(enc, &mv, v, bh, N, d, kBK) || !encode_map(enc, &mdo, dout, bh, N, d, q_rows))
         return ATTN_ERR_CUDA;
 
     BwdParams p;
@@ -817,7 +1281,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     p.N = N;
     p.key_pad = key_pad;
     p.n_kb = (N + kBK - 1) / kBK;
-    p.n_qt = (N + kBQ - 1) / kBQ;
+    p.n_qt = (N + q_rows - 1) / q_rows;
     const long long units = BH * p.n_kb;
     if (units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     p.total_units = static_cast<int>(units);
@@ -833,14 +1297,20 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const long long prep_blocks = (static_cast<long long>(rows) + 255) / 256;
-    attn_bwd_prep_kernel<<<static_cast<int>(prep_blocks < 4 * sms ? prep_blocks : 4 * sms), 256, 0, s>>>(
-        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), delta, dq, static_cast<long long>(rows));
+    const int prep_grid = static_cast<int>(prep_blocks < 4 * sms ? prep_blocks : 4 * sms);
+    const uint16_t* o16 = static_cast<const uint16_t*>(o);
+    const uint16_t* do16 = static_cast<const uint16_t*>(dout);
+    if (d == 64)
+        attn_bwd_prep_kernel<64><<<prep_grid, 256, 0, s>>>(o16, do16, delta, dq, static_cast<long long>(rows));
+    else
+        attn_bwd_prep_kernel<128><<<prep_grid, 256, 0, s>>>(o16, do16, delta, dq, static_cast<long long>(rows));
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-        cudaSuccess)
+    auto kern = d == 64 ? attn_bwd_kernel : b128::kernel;
+    const int smem = d == 64 ? kSmemBytes : b128::kSmemBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return ATTN_ERR_CUDA;
     const int grid = static_cast<int>(units < sms ? units : sms);
-    attn_bwd_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mdo, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -151,7 +151,7 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
  *   dq               : fp32 [B, H, N, d], written: dQ in fp32 (cleared, then
  *                      accumulated over key blocks by the call itself).
  *   dk, dv           : bf16 [B, H, N, d], written.
- *   d                : 64 (other values return ATTN_ERR_UNSUPPORTED).
+ *   d                : 64 or 128 (other values return ATTN_ERR_UNSUPPORTED).
  *   scale, causal, stream, B, H, N : as attn_fwd.
  *
  * Pointers must be device memory of the current device covering their

@@ -3,8 +3,10 @@
 The backward rebuilds P from the forward's LSE and forms dS, dV, dK and dQ
 from bf16 operands with fp32 accumulation (FlashAttention wiki notes, section
 "Recomputation").  Tolerance, per gradient tensor G in {dQ, dK, dV}:
-max|G - G_ref| <= 2e-2 * max|G_ref|, element by element, with G_ref the fp64
-oracle on the same bf16 Q, K, V, dO.  It comes from the arithmetic: P and dS
+max|G - G_ref| <= 2e-2 * max|G_ref| + 1e-5, element by element, with G_ref
+the fp64 oracle on the same bf16 Q, K, V, dO.  The absolute 1e-5 covers
+references that cancel exactly (one key: dS = dP - delta = 0), where the
+kernel is left with fp32 rounding of dP - delta.  It comes from the arithmetic: P and dS
 enter the tensor core rounded to bf16 (relative 2^-9 each), delta is formed
 from the bf16 O, and dK, dV are returned in bf16 (relative 2^-9); the sums
 over up to N terms of mixed sign keep the error of an element a small
@@ -23,10 +25,10 @@ from exact_io_aware_102_b200.inputs import make_dout, make_qkv, sample_rows
 pytestmark = pytest.mark.gpu
 
 REL_TOL = 2e-2
+ABS_FLOOR = 1e-5
 
 
-def run_bwd(B, H, N, causal, seed=0, scale=None):
-    d = 64
+def run_bwd(B, H, N, causal, seed=0, scale=None, d=64):
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dev = torch.device("cuda:0")
     q, k, v = make_qkv(B, H, N, d, seed=seed)
@@ -41,16 +43,16 @@ def run_bwd(B, H, N, causal, seed=0, scale=None):
 
 def compare(got, ref, what):
     err = np.abs(got - ref).max()
-    bound = REL_TOL * np.abs(ref).max()
+    bound = REL_TOL * np.abs(ref).max() + ABS_FLOOR
     assert np.isfinite(got).all(), what
     assert err <= bound, "%s: max err %.3g > %.3g (max |ref| %.3g)" % (what, err, bound, np.abs(ref).max())
     return err / max(np.abs(ref).max(), 1e-30)
 
 
-def check_full(B, H, N, causal, seed=0):
-    ins, (dq, dk, dv), scale = run_bwd(B, H, N, causal, seed)
+def check_full(B, H, N, causal, seed=0, d=64):
+    ins, (dq, dk, dv), scale = run_bwd(B, H, N, causal, seed, d=d)
     rq, rk, rv = oracle.attention_bwd_rows(*ins, scale, causal)
-    shape = (B, H, N, 64)
+    shape = (B, H, N, d)
     return [compare(g, r.reshape(shape), n) for g, r, n in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV"))]
 
 
@@ -109,11 +111,12 @@ def test_bwd_deterministic_dk_dv():
 
 
 # ---- key padding (the forward's mask, nonzero = padded key)
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [300, 700])
-def test_bwd_key_padding_full(N, causal):
-    B, H, d = 4, 2, 64
-    scale = 1.0 / 8
+def test_bwd_key_padding_full(N, causal, d):
+    B, H = 4, 2
+    scale = 1.0 / math.sqrt(d)
     dev = torch.device("cuda:0")
     rng = np.random.default_rng(N)
     pad = np.zeros((B, N), dtype=bool)
@@ -139,3 +142,28 @@ def test_bwd_key_padding_full(N, causal):
     assert (dk_n[:, :, :][np.broadcast_to(pad[:, None, :], (B, H, N))] == 0).all()
     assert (dv_n[np.broadcast_to(pad[:, None, :], (B, H, N))] == 0).all()
     assert (dq[3] == 0).all()
+
+
+# ---- head size 128 (64-row query tiles, dQ formed transposed)
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 17, 63, 64, 65, 127, 128, 129, 255, 300, 700])
+def test_bwd_d128_small_sizes_full(N, causal):
+    check_full(1, 2, N, causal, seed=N + 7, d=128)
+
+
+def test_bwd_d128_more_units_than_sms_full():
+    check_full(2, 40, 1000, False, seed=19, d=128)
+    check_full(2, 40, 1000, True, seed=20, d=128)
+
+
+def test_bwd_d128_long_causal_sampled():
+    # the causal decoder shape of the forward (d = 128) at N = 8192, 2 heads
+    B, H, N, d = 1, 2, 8192, 128
+    ins, (dq, dk, dv), scale = run_bwd(B, H, N, True, seed=23, d=d)
+    qs = sample_rows(B, H, N, 64).numpy()
+    ks = sample_rows(B, H, N, 64).numpy()[:, ::-1].copy()
+    rq, rk, rv = oracle.attention_bwd_rows(*ins, scale, True, q_rows=qs, k_rows=ks)
+    flat = lambda x: x.reshape(B * H, N, d)
+    compare(np.take_along_axis(flat(dq), qs[..., None], 1), rq, "dQ")
+    compare(np.take_along_axis(flat(dk), ks[..., None], 1), rk, "dK")
+    compare(np.take_along_axis(flat(dv), ks[..., None], 1), rv, "dV")

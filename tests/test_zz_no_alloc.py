@@ -24,7 +24,7 @@ def test_noalloc_rejects_oversize_on_host():
     # B*H*N = 2^20 + 64 rows: larger than the static array
     assert pkg.attn_bwd_noalloc(*dense, 1, 1, CAPACITY + 64, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
     assert pkg.attn_bwd_noalloc(*dense, 0, 1, 128, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
-    assert pkg.attn_bwd_noalloc(*dense, 1, 1, 128, 128, 0.125, 0, None) == pkg.ATTN_ERR_UNSUPPORTED
+    assert pkg.attn_bwd_noalloc(*dense, 1, 1, 128, 96, 0.125, 0, None) == pkg.ATTN_ERR_UNSUPPORTED
 
 
 def _buffers(B, H, N, d, seed, causal):
