@@ -8,7 +8,9 @@ library is missing, every entry point raises.
 The C entry points keep their names here (``attn_fwd``, ``attn_fwd_strided``,
 ``attn_fwd_block_sparse``, ``attn_bwd``, ``attn_bwd_noalloc``, ``attn_status_string``, ``attn_check_device_status``,
 ``attn_selftest_wait_timeout``, ``attn_version``); ``forward`` is the tensor
-convenience wrapper and ``backward`` its gradient counterpart.
+convenience wrapper, ``forward_host`` the same on host tensors with the
+transfers overlapped with the kernel, and ``backward`` the gradient
+counterpart.
 """
 import ctypes
 import math
@@ -16,7 +18,7 @@ import os
 
 __all__ = [
     "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_bwd", "attn_bwd_noalloc", "attn_status_string", "attn_check_device_status",
-    "attn_selftest_wait_timeout", "attn_version", "forward", "backward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
+    "attn_selftest_wait_timeout", "attn_version", "forward", "forward_host", "backward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
 ]
 
@@ -244,3 +246,67 @@ def backward(q, k, v, o, lse, dout, scale=None, causal=False, stream=None, key_p
     if status != ATTN_OK:
         raise AttnError(status, "attn_bwd")
     return dq, dk, dv
+
+
+def forward_host(q, k, v, scale=None, causal=False, chunks=4, out=None, lse=None, workspace=None,
+                 device=None):
+    """Attention on host tensors, with transfers overlapped with the kernel.
+
+    q, k, v: contiguous bf16 CPU tensors [B, H, N, d] (pinned, for
+    asynchronous copies).  The B*H heads are split into ``chunks`` groups;
+    group c+1 is copied to the device while the kernel runs on group c and
+    the outputs of group c-1 are copied back, on three CUDA streams.  Returns
+    host tensors (o bf16 [B, H, N, d], lse fp32 [B, H, N]), written into
+    ``out`` / ``lse`` when given (pinned host tensors).  ``workspace``: None
+    or a tuple of device tensors (q, k, v, o, lse) shaped like the inputs and
+    outputs, reused across calls.  On return every copy has been queued; the
+    current stream of ``device`` is ordered after all of them (synchronize it
+    before reading the outputs).
+    """
+    import torch
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one shape [B, H, N, d]")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous bf16 host tensor" % name)
+    B, H, N, d = (int(x) for x in q.shape)
+    BH = B * H
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    if workspace is None:
+        workspace = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                     torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                     torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                     torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                     torch.empty((B, H, N), dtype=torch.float32, device=dev))
+    qd, kd, vd, od, ld = (w.view(BH, *w.shape[2:]) for w in workspace)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    for w in workspace:  # used on the copy streams too: keep the allocator from reusing it early
+        w.record_stream(s_in)
+        w.record_stream(s_out)
+    qh, kh, vh, oh, lh = (t.view(BH, *t.shape[2:]) for t in (q, k, v, out, lse))
+    chunks = max(1, min(int(chunks), BH))
+    bounds = [BH * c // chunks for c in range(chunks + 1)]
+    compute = torch.cuda.current_stream(dev)
+    s_in.wait_stream(compute)  # the workspace is free once earlier work on it is done
+    s_out.wait_stream(compute)
+    for c in range(chunks):
+        h0, h1 = bounds[c], bounds[c + 1]
+        if h1 == h0:
+            continue
+        with torch.cuda.stream(s_in):
+            for dst, src in ((qd, qh), (kd, kh), (vd, vh)):
+                dst[h0:h1].copy_(src[h0:h1], non_blocking=True)
+        compute.wait_stream(s_in)
+        view = lambda t: t[h0:h1].view(1, h1 - h0, *t.shape[1:])
+        forward(view(qd), view(kd), view(vd), scale=scale, causal=causal, out=view(od), lse=view(ld),
+                stream=compute)
+        s_out.wait_stream(compute)
+        with torch.cuda.stream(s_out):
+            oh[h0:h1].copy_(od[h0:h1], non_blocking=True)
+            lh[h0:h1].copy_(ld[h0:h1], non_blocking=True)
+    compute.wait_stream(s_out)
+    return out, lse

@@ -355,3 +355,17 @@ def test_block_sparse_largest_mask_d128_sampled():
     bm = random_block_mask(512, 0.05, 9)
     np.fill_diagonal(bm, True)
     sparse_check(1, 2, N, 128, True, bm, rows=64)
+
+
+# ---- host-memory entry point: chunked transfers overlapping the kernel
+@pytest.mark.parametrize("chunks", [1, 3, 8])
+def test_forward_host_equals_device_forward(chunks):
+    dev = torch.device("cuda:0")
+    for (B, H, N, d, causal) in ((2, 3, 500, 64, True), (1, 16, 1944, 64, False), (1, 4, 700, 128, True)):
+        q, k, v = make_qkv(B, H, N, d, seed=N + chunks)
+        qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+        oh, lh = pkg.forward_host(qh, kh, vh, causal=causal, chunks=chunks)
+        torch.cuda.synchronize()
+        o, lse = pkg.forward(q.to(dev), k.to(dev), v.to(dev), causal=causal)
+        assert pkg.attn_check_device_status() == pkg.ATTN_OK
+        assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu())
