@@ -16,7 +16,10 @@ value = FLOPs of all ranks / the slowest rank's time, scaling "weak".
 of the same workload.  ``--pass backward`` times the backward by
 recomputation (attn_bwd: dQ, dK, dV from Q, K, V, O, LSE and a seeded dO) on
 the same workload instead of the forward; it is a secondary line, not the
-headline metric.
+headline metric.  ``--sweep`` prints one line per patch count of the pages'
+image sweep (N = 1944, 3952, 7776, 11616, 38400; B=1, H=16, d=64): TFLOP/s
+and the call's peak extra device bytes next to one materialised H x N x N
+bf16 score table.
 """
 import argparse
 import hashlib
@@ -405,6 +408,52 @@ def run_cuda_backward(args, rank, world, dist):
     }
 
 
+def run_sweep(args):
+    """TFLOP/s and peak extra device bytes over the image sweep (one JSON line each)."""
+    import torch
+    import exact_io_aware_102_b200 as pkg
+    from exact_io_aware_102_b200.inputs import make_qkv
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peaks = load_peaks()
+    lines = []
+    for N in (1944, 3952, 7776, 11616, 38400):
+        B, H, d = 1, 16, 64
+        q, k, v = (x.to(dev) for x in make_qkv(B, H, N, d, seed=0))
+        pkg.forward(q, k, v)
+        torch.cuda.synchronize()
+        base = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
+        o, lse = pkg.forward(q, k, v)
+        torch.cuda.synchronize()
+        extra = torch.cuda.max_memory_allocated() - base
+        steps = max(5, min(args.steps, 50))
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            pkg.forward(q, k, v, out=o, lse=lse)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record()
+            pkg.forward(q, k, v, out=o, lse=lse)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        st = pkg.attn_check_device_status()
+        if st != pkg.ATTN_OK:
+            raise RuntimeError("device status: " + pkg.attn_status_string(st))
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        tf = attn_flops(B, H, N, d, False) / (ms * 1e-3) / 1e12
+        lines.append({"sweep": "patch self-attention", "B": B, "H": H, "N": N, "d": d, "causal": False,
+                      "tflops": round(tf, 2), "pct_of_peak": round(100 * tf / peaks["bf16_tflops"], 2),
+                      "ms": round(ms, 4), "peak_extra_bytes": int(extra),
+                      "o_plus_lse_bytes": output_bytes(B, H, N, d),
+                      "materialised_copy_bf16": materialised_bytes(H, N, 2)})
+        del q, k, v, o, lse
+    return lines
+
+
 def run_reference(args, rank, world):
     """The fp64 CPU oracle timed on the host cores, each step a bounded sample."""
     from exact_io_aware_102_b200.inputs import make_qkv
@@ -448,6 +497,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
                     help="time the forward (the headline) or the backward")
+    ap.add_argument("--sweep", action="store_true", help="TFLOP/s and peak extra bytes over the image sweep")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -458,6 +508,13 @@ def main(argv=None):
     rank = int(os.environ.get("RANK", "0"))
     if world != args.gpus:
         ap.error("--gpus %d but WORLD_SIZE=%d: launch N>1 with torch.distributed.run" % (args.gpus, world))
+
+    if args.sweep:
+        if world != 1:
+            ap.error("--sweep runs on one GPU")
+        for line in run_sweep(args):
+            print(json.dumps(line), flush=True)
+        return 0
 
     if args.impl == "reference":
         if rank != 0:
