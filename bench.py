@@ -37,6 +37,15 @@ if ROOT not in sys.path:
 
 METRIC = "attn fwd TFLOP/s (% bf16 TC peak) at H16 N11616 d64; peak extra HBM bytes"
 WORKLOAD = {"name": "patch self-attention 3 MP", "B": 1, "H": 16, "N": 11616, "d": 64, "causal": False}
+# the other workloads of the pages (--config); the default line is WORKLOAD
+CONFIGS = {
+    "headline": WORKLOAD,
+    "tiny": {"name": "tiny exact attention", "B": 1, "H": 2, "N": 128, "d": 64, "causal": False},
+    "half_mp": {"name": "patch self-attention 0.5 MP", "B": 1, "H": 16, "N": 1944, "d": 64, "causal": False},
+    "eight_mp": {"name": "patch self-attention 8 MP", "B": 1, "H": 16, "N": 38400, "d": 64, "causal": False},
+    "causal_decoder": {"name": "causal decoder", "B": 8, "H": 12, "N": 1024, "d": 64, "causal": True},
+    "causal_d128": {"name": "causal decoder d=128", "B": 1, "H": 16, "N": 16384, "d": 128, "causal": True},
+}
 DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
@@ -211,6 +220,17 @@ def time_oracle(q, k, v, scale, causal, budget_s, max_rows=None):
 
 
 # -------------------------------------------------------------------- arms
+def workload(args):
+    return CONFIGS[args.config]
+
+
+def metric_name(W, what="fwd"):
+    if W is WORKLOAD and what == "fwd":
+        return METRIC
+    return "attn %s TFLOP/s at B%d H%d N%d d%d%s" % (what, W["B"], W["H"], W["N"], W["d"],
+                                                     " causal" if W["causal"] else "")
+
+
 def run_cuda(args, rank, world, dist):
     import torch
     import exact_io_aware_102_b200 as pkg
@@ -219,7 +239,7 @@ def run_cuda(args, rank, world, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    W = WORKLOAD
+    W = workload(args)
     B, H, N, d, causal = W["B"], W["H"], W["N"], W["d"], W["causal"]
     scale = 1.0 / math.sqrt(d)
     q_cpu, k_cpu, v_cpu = make_qkv(B, H, N, d, seed=0)
@@ -271,7 +291,8 @@ def run_cuda(args, rank, world, dist):
     achieved = flops / (ms_local * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": profiled_traffic(), "peak_kind": "burst bf16 dense, %s" % peaks["source"],
+                "traffic": profiled_traffic() if W is WORKLOAD else None,
+                "peak_kind": "burst bf16 dense, %s" % peaks["source"],
                 "algorithmic_bytes": algorithmic_bytes(B, H, N, d),
                 "frac_of_datasheet_2250": round(achieved / DATASHEET_BF16_TFLOPS, 4)}
 
@@ -322,7 +343,7 @@ def run_cuda(args, rank, world, dist):
                                                                         r["seconds"])}
 
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "metric": metric_name(W), "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic: iid N(0,1) rounded to bf16, seed 0",
         "config": {"workload": "%s: B=%d H=%d N=%d d=%d %s, bf16 Q/K/V/O, fp32 LSE" % (
@@ -356,7 +377,7 @@ def run_cuda_backward(args, rank, world, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    W = WORKLOAD
+    W = workload(args)
     B, H, N, d, causal = W["B"], W["H"], W["N"], W["d"], W["causal"]
     scale = 1.0 / math.sqrt(d)
     q, k, v = (x.to(dev) for x in make_qkv(B, H, N, d, seed=0))
@@ -390,7 +411,7 @@ def run_cuda_backward(args, rank, world, dist):
     peaks = load_peaks()
     achieved = flops / (ms_local * 1e-3) / 1e12
     return {
-        "metric": "attn bwd TFLOP/s at H16 N11616 d64 (dQ, dK, dV by recomputation)",
+        "metric": metric_name(W, "bwd") + " (dQ, dK, dV by recomputation)",
         "value": round(flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -457,7 +478,7 @@ def run_sweep(args):
 def run_reference(args, rank, world):
     """The fp64 CPU oracle timed on the host cores, each step a bounded sample."""
     from exact_io_aware_102_b200.inputs import make_qkv
-    W = WORKLOAD
+    W = workload(args)
     B, H, N, d, causal = W["B"], W["H"], W["N"], W["d"], W["causal"]
     scale = 1.0 / math.sqrt(d)
     q, k, v = make_qkv(B, H, N, d, seed=0)
@@ -474,7 +495,7 @@ def run_reference(args, rank, world):
     value = flop / secs / 1e12
     sample = ("%d of %d query rows per head x %d heads per step (seeded), fp64 C oracle" % (rows, N, B * H))
     return {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "impl": "reference", "metric": metric_name(W), "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic: iid N(0,1) rounded to bf16, seed 0",
@@ -498,6 +519,8 @@ def main(argv=None):
     ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
                     help="time the forward (the headline) or the backward")
     ap.add_argument("--sweep", action="store_true", help="TFLOP/s and peak extra bytes over the image sweep")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default="headline",
+                    help="workload (default: the headline patch self-attention 3 MP)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

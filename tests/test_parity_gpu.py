@@ -369,3 +369,37 @@ def test_forward_host_equals_device_forward(chunks):
         o, lse = pkg.forward(q.to(dev), k.to(dev), v.to(dev), causal=causal)
         assert pkg.attn_check_device_status() == pkg.ATTN_OK
         assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu())
+
+
+# ---- everything at once: packed-projection strides, key padding and a block mask
+@pytest.mark.parametrize("d,causal", [(64, False), (64, True), (128, False), (128, True)])
+def test_strided_padded_block_sparse_together(d, causal):
+    dev = torch.device("cuda:0")
+    B, H, N = 2, 3, 600
+    T = (N + 127) // 128
+    g = torch.Generator().manual_seed(31 + d)
+    packed = torch.randn(B, N, 3, H, d, generator=g).to(torch.bfloat16).to(dev)
+    q, k, v = (packed[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    rng = np.random.default_rng(d + int(causal))
+    pad = rng.random((B, N)) < 0.2
+    pad[1, N - 100:] = True
+    bm = random_block_mask(T, 0.6, 77 + d)
+    o_buf = torch.zeros((B, N, H, d), dtype=torch.bfloat16, device=dev)
+    o, lse = pkg.forward(q, k, v, causal=causal, out=o_buf.permute(0, 2, 1, 3),
+                         key_padding_mask=torch.as_tensor(pad).to(dev), block_mask=torch.as_tensor(bm).to(dev))
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    qc, kc, vc = (x.contiguous().cpu() for x in (q, k, v))
+    o_ref, lse_ref = oracle.attention_rows(qc, kc, vc, 1.0 / math.sqrt(d), causal, key_pad=pad.astype(np.uint8),
+                                           block_mask=bm.astype(np.uint8))
+    o_n = o.float().cpu().numpy().reshape(o_ref.shape)
+    lse_n = lse.cpu().numpy().reshape(lse_ref.shape)
+    assert np.abs(o_n - o_ref).max() <= TOL_O
+    empty = np.isneginf(lse_ref)
+    assert (np.isneginf(lse_n) == empty).all()
+    assert np.abs(lse_n[~empty] - lse_ref[~empty]).max() <= TOL_LSE
+
+
+def test_many_small_heads_full():
+    # 1024 (batch, head) pairs of 200 rows: 1024 work units over 148 CTAs
+    check(64, 16, 200, 64, False, seed=41)
+    check(64, 16, 200, 64, True, seed=42)
