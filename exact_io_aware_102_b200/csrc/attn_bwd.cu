@@ -30,9 +30,9 @@
 //     dV of the previous tile, so the products of tile i overlap the
 //     elementwise work of tile i+1;
 //   * warps 8-11 (one thread per query row) read the dQ partial from TMEM and
-//     add it to the fp32 dQ accumulator in global memory with bulk
-//     asynchronous reductions (cp.reduce.async.bulk .add.f32), one 256-byte
-//     row per thread;
+//     add it to the fp32 dQ accumulator in global memory with tensor
+//     reductions (cp.reduce.async.bulk.tensor .add), two [32 x 32] boxes per
+//     warp;
 //   * at the end of a unit warps 0-3 write dV and warps 4-7 dK (times scale)
 //     in bf16.
 //   Every wait is bounded (see sm100_ptx.cuh) and no barrier spans warps
@@ -86,9 +86,9 @@ constexpr int kOffQ = kOffV + kTile;          // [2] stages
 constexpr int kOffDO = kOffQ + 2 * kTile;     // [2] stages
 constexpr int kOffDS = kOffDO + 2 * kTile;    // [2] dS^T buffers, each two 64-column halves
 constexpr int kDsBytes = 2 * kHalf;
-constexpr int kOffStage = kOffDS + 2 * kDsBytes;  // dQ staging: 128 rows x 64 fp32, rows padded
-constexpr int kStageRowBytes = kD * 4 + 16;   // the padding spreads a warp's rows over all banks
-constexpr int kStageWarpBytes = 32 * kStageRowBytes;
+constexpr int kOffStage = kOffDS + 2 * kDsBytes;  // dQ staging: per dQ warp two [32 x 32] fp32 boxes
+constexpr int kStageBoxBytes = 32 * 32 * 4;   // 128-byte-swizzled, as the tensor reduction reads them
+constexpr int kStageWarpBytes = 2 * kStageBoxBytes;
 constexpr int kOffRow = kOffStage + 4 * kStageWarpBytes;  // per P/dS warp: lse2[64], delta[64]
 constexpr int kRowWarpBytes = 2 * 64 * 4;
 constexpr int kOffBar = kOffRow + kPdsWarps * kRowWarpBytes;
@@ -484,15 +484,17 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
 }
 
 // ------------------------------------------------------------- dQ warps (8-11)
-// Thread = query row of the tile = TMEM lane; each thread stages its row
-// (scaled) in shared memory and adds it to dQ with one bulk reduction.
-__device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
+// Thread = query row of the tile = TMEM lane.  Each warp stages its 32 rows
+// as two [32 x 32] fp32 boxes in the 128-byte-swizzled layout and adds them
+// to dQ with two tensor reductions (cp.reduce.async.bulk.tensor .add); the
+// tensor map clips rows past N.
+__device__ __forceinline__ void role_dq(const Ctx& c, const CUtensorMap* tm_dq, int warp, int lane) {
     const BwdParams& p = c.p;
     const int quarter = warp & 3;
     const uint32_t t_dq = c.tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColDQ;
-    const uint32_t my_row = c.base + kOffStage + quarter * kStageWarpBytes + lane * kStageRowBytes;
+    const uint32_t stage = c.base + kOffStage + quarter * kStageWarpBytes;
     uint32_t g = 0;
-    bool pending = false;  // this thread's last bulk reduction may still read its staging row
+    bool pending = false;  // lane 0: this warp's last reductions may still read the staging boxes
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
@@ -504,8 +506,9 @@ __device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
                 break;
             }
             tc_fence_after();
-            if (pending) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            if (lane == 0 && pending) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             pending = false;
+            __syncwarp();
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t a[32];
@@ -516,27 +519,32 @@ __device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
                     tc_fence_before();
                     mbar_arrive(c.bar + Bars::kDQEmpty);
                 }
+                // row `lane` of box h: 16-byte chunk v4 at chunk v4 ^ (lane % 8)
 #pragma unroll
                 for (int v4 = 0; v4 < 8; ++v4)
-                    st_shared_v4(my_row + (h * 8 + v4) * 16, __float_as_uint(__uint_as_float(a[v4 * 4]) * p.scale),
+                    st_shared_v4(stage + h * kStageBoxBytes + lane * 128 + ((v4 ^ (lane & 7)) << 4),
+                                 __float_as_uint(__uint_as_float(a[v4 * 4]) * p.scale),
                                  __float_as_uint(__uint_as_float(a[v4 * 4 + 1]) * p.scale),
                                  __float_as_uint(__uint_as_float(a[v4 * 4 + 2]) * p.scale),
                                  __float_as_uint(__uint_as_float(a[v4 * 4 + 3]) * p.scale));
             }
             fence_proxy_async();
-            const int row = i * kBQ + quarter * 32 + lane;
-            if (row < p.N) {
-                float* dst = p.dq + (static_cast<size_t>(w.bh) * p.N + row) * kD;
-                asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
-                             "r"(my_row), "r"(static_cast<uint32_t>(kD * 4))
-                             : "memory");
+            __syncwarp();
+            const int row0 = i * kBQ + quarter * 32;
+            if (lane == 0 && row0 < p.N) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    asm volatile(
+                        "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
+                        ::"l"(reinterpret_cast<uint64_t>(tm_dq)), "r"(h * 32), "r"(row0), "r"(w.bh),
+                        "r"(stage + h * kStageBoxBytes)
+                        : "memory");
                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 pending = true;
             }
-            __syncwarp();
         }
     }
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     __syncwarp();
 }
 
@@ -544,7 +552,7 @@ __device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const BwdParams p) {
+                const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -580,6 +588,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_do);
+        prefetch_tmap(&tm_dq);
     }
     if (warp == 0) {
         tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -594,7 +603,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         role_pds(ctx, warp, lane);
     } else if (warp < kDqWarp0 + 4) {
         regs_decrease<kOtherRegs>();
-        role_dq(ctx, warp, lane);
+        role_dq(ctx, &tm_dq, warp, lane);
     } else {
         regs_decrease<kOtherRegs>();
         if (lane == 0) {
@@ -1030,7 +1039,8 @@ __device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
 
 __global__ void __launch_bounds__(kThreads, 1)
 kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+       const __grid_constant__ CUtensorMap /*tm_dq: d = 128 adds whole tiles untiled*/, const BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -1140,6 +1150,18 @@ bool encode_map(EncodeTiledFn enc, CUtensorMap* map, const void* ptr, int BH, in
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 dQ [BH, N, 64] as a 3-D (64, N, BH) map, box 32 x 32, 128-byte swizzle
+// (the tensor reductions of the d = 64 kernel; rows past N are clipped).
+bool encode_dq_map(EncodeTiledFn enc, CUtensorMap* map, void* ptr, int BH, int N) {
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {64 * 4, static_cast<cuuint64_t>(N) * 64 * 4};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1268,12 +1290,17 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         return ATTN_ERR_CUDA;
-    alignas(64) CUtensorMap mq, mk, mv, mdo;
+    alignas(64) CUtensorMap mq, mk, mv, mdo, mdq;
     const int bh = static_cast<int>(BH);
     const int q_rows = d == 64 ? kBQ : b128::kBQ;  // query rows per tile (the Q / dO box)
     if (!encode_map(enc, &mq, q, bh, N, d, q_rows) || !encode_map(enc, &mk, k, bh, N, d, kBK) ||
         !encode_map(enc, &mv, v, bh, N, d, kBK) || !encode_map(enc, &mdo, dout, bh, N, d, q_rows))
         return ATTN_ERR_CUDA;
+    if (d == 64) {
+        if (!encode_dq_map(enc, &mdq, dq, bh, N)) return ATTN_ERR_CUDA;
+    } else {
+        mdq = mq;  // unused at d = 128
+    }
 
     BwdParams p;
     p.BH = bh;
@@ -1310,7 +1337,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return ATTN_ERR_CUDA;
     const int grid = static_cast<int>(units < sms ? units : sms);
-    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mdo, p);
+    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mdo, mdq, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
