@@ -98,3 +98,28 @@ def test_reference_arm_other_ranks_exit_quietly():
 def test_warmup_below_three_rejected():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_backward_flops_and_configs():
+    # five N x N x d products in the backward (S recomputed, dP, dV, dK, dQ)
+    assert bench.bwd_flops(1, 16, 11616, 64, False) == 10 * 16 * 11616 ** 2 * 64
+    assert bench.bwd_flops(1, 16, 16384, 128, True) == 5 * 16 * 16384 ** 2 * 128
+    # every workload of the pages is reachable by name, the default is the headline
+    assert bench.CONFIGS["headline"] is bench.WORKLOAD
+    assert {c["N"] for c in bench.CONFIGS.values()} >= {128, 1944, 11616, 38400, 1024, 16384}
+    args = type("A", (), {"config": "causal_d128"})()
+    w = bench.workload(args)
+    assert (w["B"], w["H"], w["N"], w["d"], w["causal"]) == (1, 16, 16384, 128, True)
+    # the headline keeps the metric name it is quoted on; others name their shape
+    assert bench.metric_name(bench.WORKLOAD) == bench.METRIC
+    assert bench.metric_name(w) == "attn fwd TFLOP/s at B1 H16 N16384 d128 causal"
+    assert bench.metric_name(bench.WORKLOAD, "bwd").startswith("attn bwd TFLOP/s at B1 H16 N11616 d64")
+
+
+def test_reference_arm_other_config():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                          "--steps", "1", "--warmup", "3", "--cpu-budget", "1"],
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["config"]["N"] == 128 and line["metric"].endswith("N128 d64")
