@@ -26,8 +26,11 @@
  * oracle's convention, from flash-attnの代役がVRAMを18GB溶かしていたので87%削った話,
  * §3 and §6): key_pad NULL or [B, N] bytes, nonzero = padded key, invisible to
  * every row.  A row with no visible key has O = 0 whatever Q, K, V are, so
- * its dQ is 0 and it adds nothing to dK, dV.  bf16 inputs are widened
- * exactly to fp64.
+ * its dQ is 0 and it adds nothing to dK, dV.  Block mask (the forward
+ * oracle's convention, FlashAttention wiki notes, section "Block-sparse
+ * FlashAttention"): NULL or [ceil(N/br), ceil(N/bc)] bytes; key j is visible
+ * to query i only if entry (i / br, j / bc) is nonzero.  bf16 inputs are
+ * widened exactly to fp64.
  *
  * Parity status: pinned by the CPU tests (central finite differences, the
  * invariants sum_j dK_j = 0, <Q, dQ> = <K, dK> and <V, dV> = <O, dO>, and a
@@ -53,7 +56,8 @@ static double widen(uint16_t bits) {
  * k_sel likewise for dK and dV.  dq: [n_q, d]; dk, dv: [n_k, d].
  */
 static int bwd_head(const double* qh, const double* kh, const double* vh, const double* doh, int N,
-                    int d, double scale, int causal, const unsigned char* pad, const int32_t* q_sel, int n_q,
+                    int d, double scale, int causal, const unsigned char* pad,
+                    const unsigned char* block_mask, int br, int bc, const int32_t* q_sel, int n_q,
                     const int32_t* k_sel, int n_k, double* dq, double* dk, double* dv, int n_threads) {
     /* position of each row in the selections (-1: not selected) */
     int* q_pos = (int*)malloc(sizeof(int) * (size_t)N);
@@ -90,12 +94,14 @@ static int bwd_head(const double* qh, const double* kh, const double* vh, const 
             for (int i = 0; i < N; ++i) {
                 const int visible = causal ? i + 1 : N;
                 const double* qi = qh + (size_t)i * d;
+                const int tc = bc > 0 ? (N + bc - 1) / bc : 0;
+                const unsigned char* brow = block_mask ? block_mask + (size_t)(i / br) * tc : NULL;
                 const double* doi = doh + (size_t)i * d;
                 /* scores and the softmax row (padded keys: P = 0) */
                 double m = -INFINITY;
                 int any = 0;
                 for (int j = 0; j < visible; ++j) {
-                    if (pad && pad[j]) continue;
+                    if ((pad && pad[j]) || (brow && !brow[j / bc])) continue;
                     double acc = 0.0;
                     for (int t = 0; t < d; ++t) acc += qi[t] * kh[(size_t)j * d + t];
                     s[j] = scale * acc;
@@ -104,7 +110,7 @@ static int bwd_head(const double* qh, const double* kh, const double* vh, const 
                 }
                 double sum = 0.0;
                 for (int j = 0; j < visible; ++j) {
-                    p[j] = (pad && pad[j]) ? 0.0 : exp(s[j] - m);
+                    p[j] = ((pad && pad[j]) || (brow && !brow[j / bc])) ? 0.0 : exp(s[j] - m);
                     sum += p[j];
                 }
                 for (int j = 0; j < visible; ++j) p[j] = any ? p[j] / sum : 0.0;
@@ -161,6 +167,7 @@ static int sel_ok(const int32_t* sel, long count, int N) {
 /*
  * bf16 inputs (raw 16-bit patterns) Q, K, V, dO, layout [B, H, N, d]
  * contiguous.  key_pad: NULL or [B, N] bytes, nonzero = padded key.
+ * block_mask: NULL or [ceil(N / br), ceil(N / bc)] bytes, nonzero = computed.
  * q_rows: NULL (all rows, n_q must equal N) or int32
  * [B*H, n_q], distinct rows per head; k_rows likewise for dK / dV.
  * dq: fp64 [B*H, n_q, d]; dk, dv: fp64 [B*H, n_k, d].
@@ -168,12 +175,13 @@ static int sel_ok(const int32_t* sel, long count, int N) {
  */
 int attn_oracle_bwd_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                          const uint16_t* dout, int B, int H, int N, int d, double scale,
-                         int causal, const unsigned char* key_pad, const int32_t* q_rows, int n_q,
-                         const int32_t* k_rows,
+                         int causal, const unsigned char* key_pad, const unsigned char* block_mask,
+                         int br, int bc, const int32_t* q_rows, int n_q, const int32_t* k_rows,
                          int n_k, double* dq, double* dk, double* dv, int n_threads) {
     if (B < 1 || H < 1 || N < 1 || d < 1 || n_q < 0 || n_k < 0) return -1;
     if ((!q_rows && n_q != N) || (!k_rows && n_k != N)) return -1;
     if (!sel_ok(q_rows, (long)B * H * n_q, N) || !sel_ok(k_rows, (long)B * H * n_k, N)) return -1;
+    if (block_mask && (br < 1 || bc < 1)) return -1;
     const size_t head = (size_t)N * d;
     double* buf = (double*)malloc(sizeof(double) * head * 4);
     if (!buf) return -2;
@@ -187,7 +195,8 @@ int attn_oracle_bwd_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v
             doh[e] = widen(dout[bh * head + e]);
         }
         const unsigned char* pad = key_pad ? key_pad + (size_t)(bh / H) * N : NULL;
-        rc = bwd_head(qh, kh, vh, doh, N, d, scale, causal, pad, q_rows ? q_rows + bh * n_q : NULL, n_q,
+        rc = bwd_head(qh, kh, vh, doh, N, d, scale, causal, pad, block_mask, br, bc,
+                      q_rows ? q_rows + bh * n_q : NULL, n_q,
                       k_rows ? k_rows + bh * n_k : NULL, n_k, dq + (size_t)bh * n_q * d,
                       dk + (size_t)bh * n_k * d, dv + (size_t)bh * n_k * d, n_threads);
     }
@@ -198,17 +207,18 @@ int attn_oracle_bwd_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v
 /* fp64 inputs, otherwise as attn_oracle_bwd_bf16. */
 int attn_oracle_bwd_f64(const double* q, const double* k, const double* v, const double* dout,
                         int B, int H, int N, int d, double scale, int causal,
-                        const unsigned char* key_pad, const int32_t* q_rows, int n_q,
-                        const int32_t* k_rows, int n_k,
+                        const unsigned char* key_pad, const unsigned char* block_mask, int br,
+                        int bc, const int32_t* q_rows, int n_q, const int32_t* k_rows, int n_k,
                         double* dq, double* dk, double* dv, int n_threads) {
     if (B < 1 || H < 1 || N < 1 || d < 1 || n_q < 0 || n_k < 0) return -1;
     if ((!q_rows && n_q != N) || (!k_rows && n_k != N)) return -1;
     if (!sel_ok(q_rows, (long)B * H * n_q, N) || !sel_ok(k_rows, (long)B * H * n_k, N)) return -1;
+    if (block_mask && (br < 1 || bc < 1)) return -1;
     const size_t head = (size_t)N * d;
     int rc = 0;
     for (long bh = 0; rc == 0 && bh < (long)B * H; ++bh)
         rc = bwd_head(q + bh * head, k + bh * head, v + bh * head, dout + bh * head, N, d, scale,
-                      causal, key_pad ? key_pad + (size_t)(bh / H) * N : NULL,
+                      causal, key_pad ? key_pad + (size_t)(bh / H) * N : NULL, block_mask, br, bc,
                       q_rows ? q_rows + bh * n_q : NULL, n_q,
                       k_rows ? k_rows + bh * n_k : NULL, n_k, dq + (size_t)bh * n_q * d,
                       dk + (size_t)bh * n_k * d, dv + (size_t)bh * n_k * d, n_threads);

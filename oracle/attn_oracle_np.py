@@ -47,13 +47,14 @@ def attention_full(q, k, v, scale, causal=False, return_probs=False, key_pad=Non
     return o, lse
 
 
-def attention_bwd_full(q, k, v, do, scale, causal=False, key_pad=None):
+def attention_bwd_full(q, k, v, do, scale, causal=False, key_pad=None, block_mask=None, block=(128, 128)):
     """Gradients (dQ, dK, dV) [B,H,N,d] of O = softmax(scale Q K^T) V for the
     upstream gradient dO, whole matrices at once: the chain rule through
     O = P V, the row softmax and S = scale Q K^T (FlashAttention wiki notes,
     section "Recomputation": the backward rebuilds S and P)."""
     q, k, v, do = (np.asarray(x, dtype=np.float64) for x in (q, k, v, do))
-    _, _, p = attention_full(q, k, v, scale, causal, return_probs=True, key_pad=key_pad)
+    _, _, p = attention_full(q, k, v, scale, causal, return_probs=True, key_pad=key_pad, block_mask=block_mask,
+                             block=block)
     dv = np.matmul(np.swapaxes(p, -1, -2), do)
     dp = np.matmul(do, np.swapaxes(v, -1, -2))
     ds = p * (dp - (p * dp).sum(axis=-1, keepdims=True))

@@ -44,8 +44,8 @@ def _load():
             fn = getattr(lib, name)
             fn.restype = ctypes.c_int
             fn.argtypes = [ptr, ptr, ptr, ptr, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                           ctypes.c_double, ctypes.c_int, ptr, ptr, ctypes.c_int, ptr, ctypes.c_int, ptr, ptr,
-                           ptr, ctypes.c_int]
+                           ctypes.c_double, ctypes.c_int, ptr, ptr, ctypes.c_int, ctypes.c_int, ptr, ctypes.c_int,
+                           ptr, ctypes.c_int, ptr, ptr, ptr, ctypes.c_int]
         lib.attn_oracle_max_threads.restype = ctypes.c_int
         lib.attn_oracle_max_threads.argtypes = []
         _lib = lib
@@ -129,13 +129,15 @@ def _select(rows, B, H, N):
     return a.shape[1], a, a.ctypes.data
 
 
-def attention_bwd_rows(q, k, v, do, scale, causal=False, q_rows=None, k_rows=None, n_threads=0, key_pad=None):
+def attention_bwd_rows(q, k, v, do, scale, causal=False, q_rows=None, k_rows=None, n_threads=0, key_pad=None,
+                       block_mask=None, block=(128, 128)):
     """Exact gradients of O = softmax(scale Q K^T) V for the upstream gradient dO.
 
     q, k, v, do: [B, H, N, d], bf16 torch tensors (widened exactly) or float64
     arrays.  q_rows / k_rows: None (all rows) or int arrays [B*H, R] (or [R],
     shared by every head) of distinct rows: dQ is evaluated at q_rows, dK and
     dV at k_rows.  key_pad: None or a [B, N] array, nonzero = padded key.
+    block_mask: None or a [ceil(N / Br), ceil(N / Bc)] array, (Br, Bc) = block.
     Returns (dQ [B*H, Rq, d], dK [B*H, Rk, d], dV [B*H, Rk, d]) as float64
     numpy arrays.
     """
@@ -161,10 +163,19 @@ def attention_bwd_rows(q, k, v, do, scale, causal=False, q_rows=None, k_rows=Non
     if key_pad is not None:
         pad_a = np.ascontiguousarray(np.asarray(key_pad).astype(np.uint8).reshape(B, N))
         pad_p = pad_a.ctypes.data
+    bm_p = None
+    br, bc = (int(x) for x in block)
+    if block_mask is not None:
+        if br < 1 or bc < 1:
+            raise ValueError("block sizes must be >= 1")
+        bm_a = np.ascontiguousarray(np.asarray(block_mask).astype(np.uint8).reshape((N + br - 1) // br,
+                                                                                     (N + bc - 1) // bc))
+        bm_p = bm_a.ctypes.data
     dq = np.empty((B * H, n_q, d), dtype=np.float64)
     dk = np.empty((B * H, n_k, d), dtype=np.float64)
     dv = np.empty((B * H, n_k, d), dtype=np.float64)
-    rc = fn(*(a.ctypes.data for a in arrs), B, H, N, d, float(scale), int(bool(causal)), pad_p, qp, n_q, kp, n_k,
+    rc = fn(*(a.ctypes.data for a in arrs), B, H, N, d, float(scale), int(bool(causal)), pad_p, bm_p, br, bc, qp,
+            n_q, kp, n_k,
             dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, int(n_threads))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (code %d)" % rc)

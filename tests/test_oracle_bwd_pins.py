@@ -209,3 +209,55 @@ def test_padded_c_oracle_matches_numpy_twin(causal):
     tw = oracle.attention_bwd_full(*(x.double().numpy() for x in (q, k, v, do)), 0.25, causal, key_pad=pad)
     for a, b in zip(got, tw):
         np.testing.assert_allclose(a.reshape(b.shape), b, rtol=0, atol=1e-12)
+
+
+# ---- block mask (FlashAttention wiki notes, "Block-sparse FlashAttention")
+
+def test_block_mask_finite_differences_and_autograd():
+    # Br = 3, Bc = 2 on N = 7 (ragged last blocks): finite differences, and
+    # autograd of the plain formula with the same visibility as a -inf mask
+    N, d, scale = 7, 3, 0.9
+    q, k, v, do = (RNG.normal(size=(1, 2, N, d)) for _ in range(4))
+    M = np.array([[1, 0, 1, 0], [0, 1, 1, 1], [1, 0, 0, 1]], dtype=np.uint8)
+    grads = [g.reshape(1, 2, N, d) for g in oracle.attention_bwd_rows(q, k, v, do, scale, block_mask=M, block=(3, 2))]
+    vis = M[(np.arange(N) // 3)[:, None], (np.arange(N) // 2)[None, :]].astype(bool)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    s = (scale * tq @ tk.transpose(-1, -2)).masked_fill(torch.tensor(~vis), float("-inf"))
+    (torch.softmax(s, dim=-1) @ tv).backward(torch.tensor(do))
+    for g, t in zip(grads, (tq, tk, tv)):
+        np.testing.assert_allclose(g, t.grad.numpy(), rtol=0, atol=1e-12)
+
+    def loss():
+        o, _ = oracle.attention_full(q, k, v, scale, block_mask=M, block=(3, 2))
+        return float((o * do).sum())
+
+    h = 1e-6
+    for x, g in zip((q, k, v), grads):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = x[idx]
+            x[idx] = old + h
+            up = loss()
+            x[idx] = old - h
+            dn = loss()
+            x[idx] = old
+            num[idx] = (up - dn) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=0, atol=2e-8)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_mask_c_oracle_matches_numpy_twin(causal):
+    q, k, v = make_qkv(1, 2, 300, 16, seed=61)
+    do = make_qkv(1, 2, 300, 16, seed=62)[0]
+    M = (np.random.default_rng(8).random((3, 3)) < 0.6).astype(np.uint8)
+    M[1, :] = 0
+    pad = (np.random.default_rng(9).random((1, 300)) < 0.2).astype(np.uint8)
+    got = oracle.attention_bwd_rows(q, k, v, do, 0.25, causal, key_pad=pad, block_mask=M)
+    tw = oracle.attention_bwd_full(*(x.double().numpy() for x in (q, k, v, do)), 0.25, causal, key_pad=pad,
+                                   block_mask=M)
+    for a, b in zip(got, tw):
+        np.testing.assert_allclose(a.reshape(b.shape), b, rtol=0, atol=1e-12)
+    # query block 1 sees nothing: its dQ rows are zero
+    assert (got[0].reshape(1, 2, 300, 16)[:, :, 128:256] == 0).all()
