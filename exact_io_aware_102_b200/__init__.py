@@ -56,11 +56,11 @@ def library():
         lib.attn_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i64, i64, i64, i64,
                                               i64, vp, vp, ctypes.c_float, i32, vp]
         lib.attn_bwd.restype = i32
-        lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, i32,
-                                 vp]
+        lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
+                                 i32, vp]
         lib.attn_bwd_noalloc.restype = i32
-        lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
-                                         i32, vp]
+        lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                         ctypes.c_float, i32, vp]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_status_string.argtypes = [i32]
         lib.attn_check_device_status.restype = i32
@@ -100,16 +100,18 @@ def attn_fwd_block_sparse(q, k, v, o, lse, B, H, N, d, qkv_strides, o_strides, s
                                            stream)
 
 
-def attn_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, N, d, scale, causal, stream, key_padding_mask=None):
+def attn_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, N, d, scale, causal, stream, key_padding_mask=None,
+             block_mask=None):
     """Raw C call: device addresses as ints; returns the status."""
-    return library().attn_bwd(q, k, v, o, dout, lse, key_padding_mask, delta, dq, dk, dv, int(B), int(H), int(N),
-                              int(d), float(scale), int(bool(causal)), stream)
+    return library().attn_bwd(q, k, v, o, dout, lse, key_padding_mask, block_mask, delta, dq, dk, dv, int(B), int(H),
+                              int(N), int(d), float(scale), int(bool(causal)), stream)
 
 
-def attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, stream, key_padding_mask=None):
+def attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, stream, key_padding_mask=None,
+                     block_mask=None):
     """Raw C call: attn_bwd with delta in the library's static device array (no allocation)."""
-    return library().attn_bwd_noalloc(q, k, v, o, dout, lse, key_padding_mask, dq, dk, dv, int(B), int(H), int(N),
-                                      int(d), float(scale), int(bool(causal)), stream)
+    return library().attn_bwd_noalloc(q, k, v, o, dout, lse, key_padding_mask, block_mask, dq, dk, dv, int(B), int(H),
+                                      int(N), int(d), float(scale), int(bool(causal)), stream)
 
 
 def attn_status_string(status):
@@ -210,12 +212,13 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None, stream=None, 
     return out, lse
 
 
-def backward(q, k, v, o, lse, dout, scale=None, causal=False, stream=None, key_padding_mask=None):
+def backward(q, k, v, o, lse, dout, scale=None, causal=False, stream=None, key_padding_mask=None, block_mask=None):
     """Gradients of ``forward`` for the upstream gradient ``dout``.
 
     q, k, v, o, dout: contiguous bf16 CUDA tensors [B, H, N, d], d = 64 or 128 (o and lse
     from ``forward`` on the same q, k, v, scale, causal and
-    ``key_padding_mask``, a bool / uint8 CUDA tensor [B, N] or None).  Returns
+    ``key_padding_mask``, a bool / uint8 CUDA tensor [B, N] or None, and
+    ``block_mask``, as in ``forward``).  Returns
     (dq fp32, dk bf16, dv bf16), each [B, H, N, d].  Asynchronous on
     ``stream`` (default: the current stream).
     """
@@ -236,13 +239,20 @@ def backward(q, k, v, o, lse, dout, scale=None, causal=False, stream=None, key_p
                 or not key_padding_mask.is_cuda or not key_padding_mask.is_contiguous()):
             raise ValueError("key_padding_mask must be a contiguous bool/uint8 CUDA tensor [B, N]")
         pad_ptr = key_padding_mask.data_ptr()
+    bm_ptr = None
+    if block_mask is not None:
+        T = (N + BLOCK - 1) // BLOCK
+        if (block_mask.shape != (T, T) or block_mask.dtype not in (torch.bool, torch.uint8)
+                or not block_mask.is_cuda or not block_mask.is_contiguous()):
+            raise ValueError("block_mask must be a contiguous bool/uint8 CUDA tensor [ceil(N/128), ceil(N/128)]")
+        bm_ptr = block_mask.data_ptr()
     delta = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     dq = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
     dk = torch.empty_like(q)
     dv = torch.empty_like(q)
     status = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                       delta.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, scale, causal,
-                      _stream_handle(stream), key_padding_mask=pad_ptr)
+                      _stream_handle(stream), key_padding_mask=pad_ptr, block_mask=bm_ptr)
     if status != ATTN_OK:
         raise AttnError(status, "attn_bwd")
     return dq, dk, dv

@@ -110,7 +110,9 @@ struct Bars {
 
 struct BwdParams {
     int BH, H, N, n_kb, n_qt, total_units, causal;
-    const uint8_t* key_pad;  // [B, N] (nonzero = padded key) or null
+    const uint8_t* key_pad;     // [B, N] (nonzero = padded key) or null
+    const uint8_t* block_mask;  // [n_bt, n_bt] (nonzero = block computed) or null
+    int n_bt;                   // ceil(N / 128)
     float scale, scale_log2;
     const float* lse;     // [BH, N]
     const float* delta;   // [BH, N]
@@ -141,6 +143,16 @@ __device__ __forceinline__ BwdUnit bwd_unit(int u, const BwdParams& p) {
     return w;
 }
 
+// Query tiles a unit visits: from w.i0 on, those whose block-mask entry
+// (query block, key block kb) is nonzero -- every one without a mask.  rows:
+// query rows per tile (128 at d = 64, 64 at d = 128); mask blocks are 128.
+__device__ __forceinline__ int next_tile(const BwdParams& p, const BwdUnit& w, int i, int rows) {
+    if (p.block_mask == nullptr) return i;
+    for (; i < p.n_qt; ++i)
+        if (p.block_mask[static_cast<size_t>(i * rows / 128) * p.n_bt + w.kb] != 0) break;
+    return i;
+}
+
 struct Ctx {
     uint32_t base, bar, tmem;
     volatile uint32_t* abort_flag;
@@ -161,6 +173,8 @@ __device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, c
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
+        int i = next_tile(p, w, w.i0, kBQ);
+        if (i >= p.n_qt) continue;  // no query tile meets this key block
         if (!wait_b(c, c.bar + Bars::kKVEmpty, (units & 1) ^ 1)) {
             ok = false;
             break;
@@ -169,7 +183,7 @@ __device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, c
         tma_load_4d(c.base + kOffK, tk, c.bar + Bars::kKVFull, 0, w.kb * kBK, w.bh, 0);
         tma_load_4d(c.base + kOffV, tv, c.bar + Bars::kKVFull, 0, w.kb * kBK, w.bh, 0);
         ++units;
-        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+        for (; i < p.n_qt; i = next_tile(p, w, i + 1, kBQ), ++g) {
             const uint32_t s = g & 1;
             if (!wait_b(c, c.bar + Bars::kQEmpty + 8 * s, ((g >> 1) & 1) ^ 1)) {
                 ok = false;
@@ -254,13 +268,15 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         BwdMma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kTile);
         tc_commit(c.bar + Bars::kSFull);
     };
-    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++units) {
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
-        const int n = p.n_qt - w.i0;
+        int i = next_tile(p, w, w.i0, kBQ);
+        if (i >= p.n_qt) continue;  // no query tile meets this key block
         if (!wait(c.bar + Bars::kKVFull, units & 1)) break;
         issue_s(g);
-        for (int it = 0; ok && it < n; ++it, ++g) {
-            if (it + 1 < n) issue_s(g + 1);  // overlaps the P/dS work of tile g
+        for (int it = 0; ok && i < p.n_qt; ++it, ++g) {
+            const int inext = next_tile(p, w, i + 1, kBQ);
+            if (inext < p.n_qt) issue_s(g + 1);  // overlaps the P/dS work of tile g
             if (!wait(c.bar + Bars::kPFull, g & 1)) break;
             if (it == 0 && !wait(c.bar + Bars::kDKVEmpty, (units & 1) ^ 1)) break;
             if (!wait(c.bar + Bars::kDQEmpty, (g & 1) ^ 1)) break;
@@ -274,11 +290,13 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
             tc_commit(c.bar + Bars::kDsFree + 8 * s);
             tc_commit(c.bar + Bars::kQEmpty + 8 * s);
             tc_commit(c.bar + Bars::kDQFull);
-            if (it + 1 == n) {
+            if (inext >= p.n_qt) {
                 tc_commit(c.bar + Bars::kDKVFull);
                 tc_commit(c.bar + Bars::kKVEmpty);
             }
+            i = inext;
         }
+        ++units;
     }
     if (!ok) {
         tc_commit(c.bar + Bars::kDrain);
@@ -330,7 +348,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
     const float sl2 = p.scale_log2;
     uint32_t g = 0, units = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++units) {
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
         const int key = w.kb * kBK + r;
         // padded keys (and rows past N) take no part: P = dS = 0 on their rows
@@ -351,8 +369,19 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
                 pre_d[e] = in ? dl_h[q] : 0.f;
             }
         };
-        fetch(w.i0);
-        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+        int i = next_tile(p, w, w.i0, kBQ);
+        if (i >= p.n_qt) {
+            // no query tile meets this key block: its dK and dV rows are zero
+            if (key < p.N) {
+                uint4* dst = reinterpret_cast<uint4*>((half == 0 ? p.dv : p.dk) +
+                                                      (static_cast<size_t>(w.bh) * p.N + key) * kD);
+#pragma unroll
+                for (int v4 = 0; v4 < kD / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            continue;
+        }
+        fetch(i);
+        for (; i < p.n_qt; ++g) {
             __syncwarp();
             asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(rows_smem + lane * 8), "f"(pre_l[0]), "f"(pre_l[1])
                          : "memory");
@@ -360,7 +389,8 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
                          "f"(pre_d[1])
                          : "memory");
             __syncwarp();
-            if (i + 1 < p.n_qt) fetch(i + 1);
+            const int inext = next_tile(p, w, i + 1, kBQ);
+            if (inext < p.n_qt) fetch(inext);
             bool got = wait_b(c, c.bar + Bars::kSFull, g & 1);
             got = __all_sync(0xffffffffu, got);
             if (!got) {
@@ -445,6 +475,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             tc_fence_before();
             fence_proxy_async();  // the tensor core reads what the generic proxy wrote
             mbar_arrive(c.bar + Bars::kPFull);
+            i = inext;
         }
         if (!ok) break;
         // unit epilogue: dV (warps 0-3) or dK times scale (warps 4-7) of this key row
@@ -454,6 +485,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             ok = false;
             break;
         }
+        ++units;
         tc_fence_after();
         uint32_t a[2][32];
         tmem_ld32(t_acc, a[0]);
@@ -498,7 +530,7 @@ __device__ __forceinline__ void role_dq(const Ctx& c, const CUtensorMap* tm_dq, 
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
-        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+        for (int i = next_tile(p, w, w.i0, kBQ); i < p.n_qt; i = next_tile(p, w, i + 1, kBQ), ++g) {
             bool got = wait_b(c, c.bar + Bars::kDQFull, g & 1);
             got = __all_sync(0xffffffffu, got);
             if (!got) {
@@ -706,6 +738,8 @@ __device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, c
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = unit(u, p);
+        int i = next_tile(p, w, w.i0, kBQ);
+        if (i >= p.n_qt) continue;  // no query tile meets this key block
         if (!wait_b(c, c.bar + Bars::kKVEmpty, (units & 1) ^ 1)) {
             ok = false;
             break;
@@ -717,7 +751,7 @@ __device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, c
             tma_load_4d(c.base + kOffV + x * kKHalf, tv, c.bar + Bars::kKVFull, x * 64, w.kb * 128, w.bh, 0);
         }
         ++units;
-        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+        for (; i < p.n_qt; i = next_tile(p, w, i + 1, kBQ), ++g) {
             const uint32_t s = g & 1;
             if (!wait_b(c, c.bar + Bars::kQEmpty + 8 * s, ((g >> 1) & 1) ^ 1)) {
                 ok = false;
@@ -796,13 +830,15 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         Mma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kQTile);
         tc_commit(c.bar + Bars::kSFull);
     };
-    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++units) {
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = unit(u, p);
-        const int n = p.n_qt - w.i0;
+        int i = next_tile(p, w, w.i0, kBQ);
+        if (i >= p.n_qt) continue;  // no query tile meets this key block
         if (!wait(c.bar + Bars::kKVFull, units & 1)) break;
         issue_s(g);
-        for (int it = 0; ok && it < n; ++it, ++g) {
-            if (it + 1 < n) issue_s(g + 1);
+        for (int it = 0; ok && i < p.n_qt; ++it, ++g) {
+            const int inext = next_tile(p, w, i + 1, kBQ);
+            if (inext < p.n_qt) issue_s(g + 1);
             if (!wait(c.bar + Bars::kPFull, g & 1)) break;
             if (it == 0 && !wait(c.bar + Bars::kDKVEmpty, (units & 1) ^ 1)) break;
             tc_fence_after();
@@ -816,11 +852,13 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
             tc_commit(c.bar + Bars::kDsFree + 8 * s);
             tc_commit(c.bar + Bars::kQEmpty + 8 * s);
             tc_commit(c.bar + Bars::kDQFull);
-            if (it + 1 == n) {
+            if (inext >= p.n_qt) {
                 tc_commit(c.bar + Bars::kDKVFull);
                 tc_commit(c.bar + Bars::kKVEmpty);
             }
+            i = inext;
         }
+        ++units;
     }
     if (!ok) {
         tc_commit(c.bar + Bars::kDrain);
@@ -842,7 +880,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
     const float sl2 = p.scale_log2;
     uint32_t g = 0, units = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++units) {
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = unit(u, p);
         const int key = w.kb * 128 + r;
         const bool key_ok = key < p.N && (p.key_pad == nullptr || p.key_pad[static_cast<size_t>(w.bh / p.H) * p.N + key] == 0);
@@ -856,13 +894,25 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             pre_l = in ? l * kLog2eB : INFINITY;
             pre_d = in ? dl_h[q] : 0.f;
         };
-        fetch(w.i0);
-        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+        int i = next_tile(p, w, w.i0, kBQ);
+        if (i >= p.n_qt) {
+            // no query tile meets this key block: its dK and dV rows are zero
+            if (key < p.N) {
+                uint4* dst = reinterpret_cast<uint4*>((half == 0 ? p.dv : p.dk) +
+                                                      (static_cast<size_t>(w.bh) * p.N + key) * kD);
+#pragma unroll
+                for (int v4 = 0; v4 < kD / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            continue;
+        }
+        fetch(i);
+        for (; i < p.n_qt; ++g) {
             __syncwarp();
             asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + lane * 4), "f"(pre_l) : "memory");
             asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + 128 + lane * 4), "f"(pre_d) : "memory");
             __syncwarp();
-            if (i + 1 < p.n_qt) fetch(i + 1);
+            const int inext = next_tile(p, w, i + 1, kBQ);
+            if (inext < p.n_qt) fetch(inext);
             bool got = wait_b(c, c.bar + Bars::kSFull, g & 1);
             got = __all_sync(0xffffffffu, got);
             if (!got) {
@@ -934,6 +984,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             tc_fence_before();
             fence_proxy_async();
             mbar_arrive(c.bar + Bars::kPFull);
+            i = inext;
         }
         if (!ok) break;
         // unit epilogue: dV (warps 0-3) or dK times scale (warps 4-7), 32 columns at a time
@@ -943,6 +994,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             ok = false;
             break;
         }
+        ++units;
         tc_fence_after();
         const float f = half == 0 ? 1.f : p.scale;
         uint4* dst = reinterpret_cast<uint4*>((half == 0 ? p.dv : p.dk) + (static_cast<size_t>(w.bh) * p.N + key) * kD);
@@ -983,7 +1035,7 @@ __device__ __forceinline__ void role_dq(const Ctx& c, int warp, int lane) {
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = unit(u, p);
-        for (int i = w.i0; i < p.n_qt; ++i, ++g) {
+        for (int i = next_tile(p, w, w.i0, kBQ); i < p.n_qt; i = next_tile(p, w, i + 1, kBQ), ++g) {
             bool got = wait_b(c, c.bar + Bars::kDQFull, g & 1);
             got = __all_sync(0xffffffffu, got);
             if (!got) {
@@ -1222,35 +1274,37 @@ float* noalloc_delta() {
 }
 
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-             const unsigned char* key_pad, float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d,
-             float scale, int causal, attn_stream_t stream);
+             const unsigned char* key_pad, const unsigned char* block_mask, float* delta, float* dq, void* dk,
+             void* dv, int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
 
 }  // namespace
 
 extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                        const float* lse, const unsigned char* key_padding_mask, float* delta, float* dq, void* dk,
-                        void* dv, int B, int H, int N, int d, float scale, int causal, attn_stream_t stream) {
-    return bwd_impl(q, k, v, o, dout, lse, key_padding_mask, delta, dq, dk, dv, B, H, N, d, scale, causal, stream);
+                        const float* lse, const unsigned char* key_padding_mask, const unsigned char* block_mask,
+                        float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                        int causal, attn_stream_t stream) {
+    return bwd_impl(q, k, v, o, dout, lse, key_padding_mask, block_mask, delta, dq, dk, dv, B, H, N, d, scale, causal,
+                    stream);
 }
 
 extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                                const float* lse, const unsigned char* key_padding_mask, float* dq, void* dk,
-                                void* dv, int B, int H, int N, int d, float scale, int causal,
-                                attn_stream_t stream) {
+                                const float* lse, const unsigned char* key_padding_mask,
+                                const unsigned char* block_mask, float* dq, void* dk, void* dv, int B, int H, int N,
+                                int d, float scale, int causal, attn_stream_t stream) {
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
     if (static_cast<long long>(B) * H * N > kNoAllocDeltaRows) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     float* delta = noalloc_delta();
     if (delta == nullptr) return ATTN_ERR_CUDA;
-    return bwd_impl(q, k, v, o, dout, lse, key_padding_mask, delta, dq, dk, dv, B, H, N, d, scale, causal,
-                    stream);
+    return bwd_impl(q, k, v, o, dout, lse, key_padding_mask, block_mask, delta, dq, dk, dv, B, H, N, d, scale,
+                    causal, stream);
 }
 
 namespace {
 
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-             const unsigned char* key_pad, float* delta, float* dq, void* dk, void* dv, int B, int H, int N, int d,
-             float scale, int causal, attn_stream_t stream) {
+             const unsigned char* key_pad, const unsigned char* block_mask, float* delta, float* dq, void* dk,
+             void* dv, int B, int H, int N, int d, float scale, int causal, attn_stream_t stream) {
     if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o || !dout || !lse || !delta || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
@@ -1269,12 +1323,15 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     const void* outs[4] = {delta, dq, dk, dv};
     const size_t out_b[4] = {lb, qb, tb, tb};
     const size_t pad_b = static_cast<size_t>(B) * N;
+    const int n_bt = (N + 127) / 128;
+    const size_t bm_b = static_cast<size_t>(n_bt) * n_bt;
     for (int a = 0; a < 4; ++a) {
         for (int b = 0; b < 6; ++b)
             if (!disjoint(outs[a], out_b[a], ins[b], in_b[b])) return ATTN_ERR_INVALID_ARG;
         for (int b = a + 1; b < 4; ++b)
             if (!disjoint(outs[a], out_b[a], outs[b], out_b[b])) return ATTN_ERR_INVALID_ARG;
         if (key_pad && !disjoint(outs[a], out_b[a], key_pad, pad_b)) return ATTN_ERR_INVALID_ARG;
+        if (block_mask && !disjoint(outs[a], out_b[a], block_mask, bm_b)) return ATTN_ERR_INVALID_ARG;
     }
     const BwdDriver& drv = bwd_driver();
     if (!drv.ok) return ATTN_ERR_CUDA;
@@ -1287,6 +1344,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     for (int a = 0; a < 4; ++a)
         if (!span_ok(range, outs[a], out_b[a], dev)) return ATTN_ERR_INVALID_ARG;
     if (key_pad && !span_ok(range, key_pad, pad_b, dev)) return ATTN_ERR_INVALID_ARG;
+    if (block_mask && !span_ok(range, block_mask, bm_b, dev)) return ATTN_ERR_INVALID_ARG;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
         return ATTN_ERR_CUDA;
@@ -1307,6 +1365,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     p.H = H;
     p.N = N;
     p.key_pad = key_pad;
+    p.block_mask = block_mask;
+    p.n_bt = n_bt;
     p.n_kb = (N + kBK - 1) / kBK;
     p.n_qt = (N + q_rows - 1) / q_rows;
     const long long units = BH * p.n_kb;

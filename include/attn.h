@@ -146,6 +146,10 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
  *                      (nonzero = padded key): padded keys get dK = dV = 0
  *                      and no query row attends to them; a row that saw no
  *                      key (LSE = -inf, O = 0) gets dQ = 0.
+ *   block_mask       : NULL, or the [T, T] byte block mask the forward used
+ *                      (T = ceil(N / 128), see attn_fwd_block_sparse): only
+ *                      nonzero (query block, key block) pairs are recomputed;
+ *                      a key block no query block meets gets dK = dV = 0.
  *   delta            : fp32 [B, H, N], written (delta_i above; a workspace
  *                      the caller owns, useful to nobody else).
  *   dq               : fp32 [B, H, N, d], written: dQ in fp32 (cleared, then
@@ -162,7 +166,7 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
  * by attn_check_device_status().
  */
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-             const float* lse, const unsigned char* key_padding_mask,
+             const float* lse, const unsigned char* key_padding_mask, const unsigned char* block_mask,
              float* delta, float* dq, void* dk, void* dv,
              int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
 
@@ -182,7 +186,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
  * order them on one stream or by events.  Everything else as attn_bwd.
  */
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                     const float* lse, const unsigned char* key_padding_mask,
+                     const float* lse, const unsigned char* key_padding_mask, const unsigned char* block_mask,
                      float* dq, void* dk, void* dv,
                      int B, int H, int N, int d, float scale, int causal, attn_stream_t stream);
 

@@ -167,3 +167,50 @@ def test_bwd_d128_long_causal_sampled():
     compare(np.take_along_axis(flat(dq), qs[..., None], 1), rq, "dQ")
     compare(np.take_along_axis(flat(dk), ks[..., None], 1), rk, "dK")
     compare(np.take_along_axis(flat(dv), ks[..., None], 1), rv, "dV")
+
+
+# ---- block-sparse mask (the forward's [T, T] mask over 128 x 128 blocks)
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [300, 700])
+def test_bwd_block_sparse_full(N, causal, d):
+    B, H = 2, 2
+    T = (N + 127) // 128
+    rng = np.random.default_rng(N + d + int(causal))
+    bm = rng.random((T, T)) < 0.6
+    np.fill_diagonal(bm[2:, 2:], True)
+    bm[1, :] = False                  # a query block that sees nothing: dQ = 0 there
+    bm[:, T - 2] = False              # a key block no query block meets: dK = dV = 0 there
+    pad = rng.random((B, N)) < 0.15
+    scale = 1.0 / math.sqrt(d)
+    dev = torch.device("cuda:0")
+    q, k, v = make_qkv(B, H, N, d, seed=N + 5)
+    do = make_dout(B, H, N, d, seed=N + 6)
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
+    bm_t, pad_t = torch.as_tensor(bm).to(dev), torch.as_tensor(pad).to(dev)
+    o, lse = pkg.forward(qd, kd, vd, scale=scale, causal=causal, key_padding_mask=pad_t, block_mask=bm_t)
+    dq, dk, dv = pkg.backward(qd, kd, vd, o, lse, dod, scale=scale, causal=causal, key_padding_mask=pad_t,
+                              block_mask=bm_t)
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    refs = oracle.attention_bwd_rows(q, k, v, do, scale, causal, key_pad=pad.astype(np.uint8),
+                                     block_mask=bm.astype(np.uint8))
+    for g, r, name in zip((dq, dk, dv), refs, ("dQ", "dK", "dV")):
+        compare(g.float().cpu().numpy(), r.reshape(B, H, N, d), name)
+    lo, hi = 128 * (T - 2), min(N, 128 * (T - 1))
+    assert (dk[:, :, lo:hi] == 0).all() and (dv[:, :, lo:hi] == 0).all()
+    assert (dq[:, :, 128:256] == 0).all()
+
+
+def test_bwd_all_ones_block_mask_matches_dense():
+    dev = torch.device("cuda:0")
+    B, H, N, d = 1, 3, 900, 64
+    T = (N + 127) // 128
+    q, k, v = (x.to(dev) for x in make_qkv(B, H, N, d, seed=71))
+    do = make_dout(B, H, N, d, seed=72).to(dev)
+    ones = torch.ones(T, T, dtype=torch.bool, device=dev)
+    for causal in (False, True):
+        o, lse = pkg.forward(q, k, v, causal=causal)
+        g1 = pkg.backward(q, k, v, o, lse, do, causal=causal, block_mask=ones)
+        g2 = pkg.backward(q, k, v, o, lse, do, causal=causal)
+        assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
+        assert torch.allclose(g1[0], g2[0], rtol=0, atol=1e-5 * float(g2[0].abs().max()))
