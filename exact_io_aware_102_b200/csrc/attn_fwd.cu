@@ -7,8 +7,10 @@
 // tile, so the N x N matrices never reach HBM, "Tiling"; scores, scaling,
 // masking, softmax and both matrix products run in ONE kernel, "Kernel
 // fusion"; only O and the per-row softmax statistics (here as one log-sum-exp)
-// are written, "Recomputation"; with a causal mask only the non-zero key
-// blocks are processed, "Block-sparse FlashAttention".
+// are written, "Recomputation"; with a causal mask or a block mask only the
+// non-zero (query block, key block) pairs are loaded and multiplied,
+// "Block-sparse FlashAttention"; padded keys (the key-padding mask of the
+// pages' patch self-attention module) are masked per element.
 //
 // How it maps to sm_100a (the page's A100 design is prior art, not followed):
 //   * persistent grid, one CTA per SM, each CTA walks work units
@@ -28,7 +30,9 @@
 //   * every mbarrier wait is bounded; on timeout a status word is set, the
 //     CTA drains its in-flight copies and MMAs, frees TMEM and returns.
 //
-// Memory layout: Q, K, V, O bf16 [B, H, N, d] contiguous, LSE fp32 [B, H, N].
+// Memory layout: Q, K, V, O bf16 [B, H, N, d] with element strides over
+// (b, h, n) and a contiguous head dimension ([B, N, H, d] and packed
+// projections included), LSE fp32 [B, H, N] contiguous.
 // Shared memory tiles use the 128-byte swizzle (TMA writes them, the tensor
 // cores read them through matrix descriptors); d = 128 tiles are stored as two
 // 64-column halves.  TMEM: S0 cols [0,128), S1 [128,256), O0 [256,256+d),
