@@ -188,3 +188,17 @@ def test_product_path_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "attn_oracle" not in text, f
+
+
+def test_forward_host_and_backward_check_arguments_first(lib):
+    import torch
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        pkg.forward_host(q, q, q[:, :1])                     # shapes differ
+    with pytest.raises(ValueError):
+        pkg.forward_host(q.float(), q.float(), q.float())    # not bf16
+    with pytest.raises(ValueError):
+        pkg.forward_host(q.transpose(2, 3), q.transpose(2, 3), q.transpose(2, 3))  # not contiguous
+    lse = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError):
+        pkg.backward(q, q, q, q, lse, q)                     # host tensors are rejected
