@@ -190,6 +190,16 @@ def test_product_path_does_not_import_the_oracle():
                 assert "attn_oracle" not in text, f
 
 
+def test_missing_library_fails_loudly():
+    # no fallback: without libattn.so every entry point raises
+    code = ("import exact_io_aware_102_b200 as p; p.LIB_PATH = '/nonexistent/libattn.so'\n"
+            "try:\n    p.attn_version()\nexcept ImportError:\n    print('raised')\n")
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT, timeout=120)
+    assert out.stdout.strip() == "raised", out.stdout + out.stderr
+
+
 def test_forward_host_and_backward_check_arguments_first(lib):
     import torch
     q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
