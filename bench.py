@@ -19,7 +19,8 @@ the same workload instead of the forward; it is a secondary line, not the
 headline metric.  ``--sweep`` prints one line per patch count of the pages'
 image sweep (N = 1944, 3952, 7776, 11616, 38400; B=1, H=16, d=64): TFLOP/s
 and the call's peak extra device bytes next to one materialised H x N x N
-bf16 score table.
+bf16 score table.  ``--pad-sweep`` times the 3 MP shape against the fraction
+of trailing keys that are padded (padded key tiles are skipped).
 """
 import argparse
 import hashlib
@@ -485,6 +486,49 @@ def run_sweep(args):
     return lines
 
 
+def run_pad_sweep(args):
+    """Key-padding sweep on the 3 MP shape (B=1, H=16, N=11616, d=64): the last
+    f*N keys padded, f in {0, 1/4, 1/2, 3/4}.  Tiles holding only padded keys
+    are skipped, so the time should fall with f; TFLOP/s counts the visible
+    (query, key) pairs only, 4*H*N*visible*d."""
+    import torch
+    import exact_io_aware_102_b200 as pkg
+    from exact_io_aware_102_b200.inputs import make_qkv
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    B, H, N, d = 1, 16, 11616, 64
+    q, k, v = (x.to(dev) for x in make_qkv(B, H, N, d, seed=0))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    lines = []
+    for frac in (0.0, 0.25, 0.5, 0.75):
+        visible = N - int(round(frac * N))
+        pad = torch.zeros((B, N), dtype=torch.bool, device=dev)
+        pad[:, visible:] = True
+        steps = max(5, min(args.steps, 50))
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            pkg.forward(q, k, v, out=o, lse=lse, key_padding_mask=pad)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record()
+            pkg.forward(q, k, v, out=o, lse=lse, key_padding_mask=pad)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        st = pkg.attn_check_device_status()
+        if st != pkg.ATTN_OK:
+            raise RuntimeError("device status: " + pkg.attn_status_string(st))
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        flop = 4.0 * B * H * N * visible * d
+        lines.append({"pad_sweep": "patch self-attention 3 MP, trailing keys padded", "B": B, "H": H, "N": N,
+                      "d": d, "padded_fraction": frac, "visible_keys": visible, "ms": round(ms, 4),
+                      "tflops_visible": round(flop / (ms * 1e-3) / 1e12, 2)})
+    return lines
+
+
 def run_reference(args, rank, world):
     """The fp64 CPU oracle timed on the host cores, each step a bounded sample."""
     from exact_io_aware_102_b200.inputs import make_qkv
@@ -529,6 +573,8 @@ def main(argv=None):
     ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
                     help="time the forward (the headline) or the backward")
     ap.add_argument("--sweep", action="store_true", help="TFLOP/s and peak extra bytes over the image sweep")
+    ap.add_argument("--pad-sweep", action="store_true",
+                    help="time against the fraction of padded keys (3 MP shape, trailing padding)")
     ap.add_argument("--config", choices=sorted(CONFIGS), default="headline",
                     help="workload (default: the headline patch self-attention 3 MP)")
     args = ap.parse_args(argv)
@@ -546,6 +592,13 @@ def main(argv=None):
         if world != 1:
             ap.error("--sweep runs on one GPU")
         for line in run_sweep(args):
+            print(json.dumps(line), flush=True)
+        return 0
+
+    if args.pad_sweep:
+        if world != 1:
+            ap.error("--pad-sweep runs on one GPU")
+        for line in run_pad_sweep(args):
             print(json.dumps(line), flush=True)
         return 0
 

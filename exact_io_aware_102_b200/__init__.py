@@ -7,7 +7,7 @@ library is missing, every entry point raises.
 
 The C entry points keep their names here (``attn_fwd``, ``attn_fwd_strided``,
 ``attn_fwd_block_sparse``, ``attn_bwd``, ``attn_bwd_noalloc``, ``attn_status_string``, ``attn_check_device_status``,
-``attn_selftest_wait_timeout``, ``attn_version``); ``forward`` is the tensor
+``attn_selftest_wait_timeout``, ``attn_selftest_ex2``, ``attn_version``); ``forward`` is the tensor
 convenience wrapper, ``forward_host`` the same on host tensors with the
 transfers overlapped with the kernel, and ``backward`` the gradient
 counterpart.
@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "AttnError", "LIB_PATH", "library", "attn_fwd", "attn_fwd_strided", "attn_fwd_block_sparse", "attn_bwd", "attn_bwd_noalloc", "attn_status_string", "attn_check_device_status",
-    "attn_selftest_wait_timeout", "attn_version", "forward", "forward_host", "backward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
+    "attn_selftest_wait_timeout", "attn_selftest_ex2", "attn_version", "forward", "forward_host", "backward", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
 ]
 
@@ -67,6 +67,8 @@ def library():
         lib.attn_check_device_status.argtypes = [vp]
         lib.attn_selftest_wait_timeout.restype = i32
         lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp]
+        lib.attn_selftest_ex2.restype = i32
+        lib.attn_selftest_ex2.argtypes = [vp, vp, i32, vp]
         lib.attn_version.restype = i32
         lib.attn_version.argtypes = []
         _lib = lib
@@ -125,6 +127,11 @@ def attn_check_device_status(stream=None):
 
 def attn_selftest_wait_timeout(limit_ns, stream=None):
     return library().attn_selftest_wait_timeout(int(limit_ns), _stream_handle(stream))
+
+
+def attn_selftest_ex2(x, y, n, stream=None):
+    """Raw C call: y[i] = the softmax's FMA-pipe 2^x[i] (device addresses as ints)."""
+    return library().attn_selftest_ex2(x, y, int(n), _stream_handle(stream))
 
 
 def attn_version():

@@ -110,6 +110,7 @@ struct Bars {
 
 struct BwdParams {
     int BH, H, N, n_kb, n_qt, total_units, causal;
+    int group_heads;            // causal unit order: heads per group (their Q, dO, dQ fit in L2)
     const uint8_t* key_pad;     // [B, N] (nonzero = padded key) or null
     const uint8_t* block_mask;  // [n_bt, n_bt] (nonzero = block computed) or null
     int n_bt;                   // ceil(N / 128)
@@ -128,12 +129,18 @@ struct BwdUnit {
 
 // Units: (head, key block).  Non-causal: heads-major, so the CTAs running at
 // one time stream the same Q / dO tiles (L2 reuse).  Causal: key block kb
-// meets query tiles kb .. n_qt-1; the blocks with most tiles go first.
+// meets query tiles kb .. n_qt-1; heads go in groups of p.group_heads, whose
+// Q, dO and dQ together fit in a third of L2, and within a group the blocks
+// with most tiles go first.
 __device__ __forceinline__ BwdUnit bwd_unit(int u, const BwdParams& p) {
     BwdUnit w;
     if (p.causal) {
-        w.kb = u / p.BH;
-        w.bh = u - w.kb * p.BH;
+        const int per_group = p.group_heads * p.n_kb;
+        const int g = u / per_group;
+        const int r = u - g * per_group;
+        const int gh = min(p.group_heads, p.BH - g * p.group_heads);  // heads in this group
+        w.kb = r / gh;
+        w.bh = g * p.group_heads + (r - w.kb * gh);
         w.i0 = w.kb;
     } else {
         w.bh = u / p.n_kb;
@@ -310,16 +317,6 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
 __device__ __forceinline__ uint32_t sw128_off(int r, int col) {
     const int h = col >> 6, c16 = (col & 63) >> 3;
     return static_cast<uint32_t>(h * kHalf + r * 128 + ((c16 ^ (r & 7)) << 4) + (col & 7) * 2);
-}
-
-// 32 lanes x 16 consecutive 32-bit TMEM columns from registers.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c4, uint32_t d) {
@@ -1254,20 +1251,30 @@ constexpr long long kNoAllocDeltaRows = 1LL << 20;  // B*H*N at most (4 MiB of f
 __device__ __align__(256) float g_noalloc_delta[kNoAllocDeltaRows];
 constexpr int kMaxDevices = 64;
 
-// Device address of g_noalloc_delta on the current device, resolved once
-// per device (cudaGetSymbolAddress); nullptr on failure.
+// Device address of g_noalloc_delta in the current context.  It is looked up
+// with cudaGetSymbolAddress on the first call in each context of a device
+// and cached under that context's id, so a device reset or a new context
+// (which loads the module afresh, maybe at another address) resolves it
+// again instead of reusing a stale address.  nullptr on failure.
 float* noalloc_delta() {
     static std::mutex m;
+    static unsigned long long ctx_of[kMaxDevices] = {};  // 0 = nothing cached
     static float* addr[kMaxDevices] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(m);
-    if (addr[dev] == nullptr) {
+    unsigned long long id = current_context_id();
+    if (id == 0 || id != ctx_of[dev]) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_delta) != cudaSuccess) {
             cudaGetLastError();
             return nullptr;
         }
+        // the runtime has a context current now (the lookup creates the
+        // primary context if needed): cache the address under its id
+        id = current_context_id();
+        if (id == 0) return nullptr;
+        ctx_of[dev] = id;
         addr[dev] = static_cast<float*>(ptr);
     }
     return addr[dev];
@@ -1373,6 +1380,11 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if (units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     p.total_units = static_cast<int>(units);
     p.causal = causal ? 1 : 0;
+    {
+        const long long head_bytes = 8LL * N * d;  // Q and dO (bf16) and dQ (fp32) of one head
+        const long long g = (40LL << 20) / head_bytes;
+        p.group_heads = static_cast<int>(g < 1 ? 1 : g > BH ? BH : g);
+    }
     p.scale = scale;
     p.scale_log2 = scale * kLog2eB;
     p.lse = lse;
@@ -1382,6 +1394,12 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     p.dv = static_cast<uint16_t*>(dv);
     p.wait_ns = kWaitNs;
 
+    // every fallible host step comes before the first launch: an error return
+    // means nothing was queued (dq, delta untouched)
+    auto kern = d == 64 ? attn_bwd_kernel : b128::kernel;
+    const int smem = d == 64 ? kSmemBytes : b128::kSmemBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const long long prep_blocks = (static_cast<long long>(rows) + 255) / 256;
     const int prep_grid = static_cast<int>(prep_blocks < 4 * sms ? prep_blocks : 4 * sms);
@@ -1392,10 +1410,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     else
         attn_bwd_prep_kernel<128><<<prep_grid, 256, 0, s>>>(o16, do16, delta, dq, static_cast<long long>(rows));
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    auto kern = d == 64 ? attn_bwd_kernel : b128::kernel;
-    const int smem = d == 64 ? kSmemBytes : b128::kSmemBytes;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return ATTN_ERR_CUDA;
     const int grid = static_cast<int>(units < sms ? units : sms);
     kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mdo, mdq, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

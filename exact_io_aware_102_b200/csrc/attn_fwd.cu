@@ -44,6 +44,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "attn.h"
@@ -138,6 +139,7 @@ enum : int { kModeFull = 0, kModeCausal = 1, kModeSparse = 2 };
 
 struct Params {
     int BH, H, N, n_pairs, n_kv_all, total_units;
+    int group_heads;             // causal unit order: heads per group (K/V of a group fit in L2)
     long long o_sb, o_sh, o_sn;  // element strides of O over (batch, head, row)
     const uint8_t* key_pad;      // [B, N] key-padding mask (nonzero = padded) or null
     int pad_vec;                 // key_pad rows may be read 16 bytes at a time
@@ -152,16 +154,24 @@ struct Unit {
 };
 
 // Work units: (head, pair of Q tiles).  Non-causal: heads-major so the CTAs
-// running at one time share K/V of few heads (L2 reuse).  Causal: the pairs
-// with the most key tiles first, so the short units fill the tail.
+// running at one time share K/V of few heads (L2 reuse).  Causal: heads in
+// groups of p.group_heads, whose K and V together fit in a third of L2; within
+// a group the pairs with the most key tiles come first, so that the short
+// units fill the tail while the CTAs running at one time read the K/V of
+// about one group only (ungrouped longest-first streams every head's K/V at
+// once and re-reads them from DRAM).
 template <int MODE>
 __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     Unit w;
     int pair;
     const bool longest_first = MODE == kModeCausal || (MODE == kModeSparse && p.causal);
     if (longest_first) {
-        pair = p.n_pairs - 1 - u / p.BH;
-        w.bh = u % p.BH;
+        const int per_group = p.group_heads * p.n_pairs;
+        const int g = u / per_group;
+        const int r = u - g * per_group;
+        const int gh = min(p.group_heads, p.BH - g * p.group_heads);  // heads in this group
+        pair = p.n_pairs - 1 - r / gh;
+        w.bh = g * p.group_heads + r % gh;
     } else {
         pair = u % p.n_pairs;
         w.bh = u / p.n_pairs;
@@ -174,32 +184,91 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
 
 constexpr int kNoTile = 0x7fffffff;
 
-// The key tiles one Q tile visits, in increasing order.
+// Bit i set iff byte i of x is nonzero (4 bits).
+__device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t x) {
+    const uint32_t y = __vcmpne4(x, 0u);  // 0xFF per nonzero byte
+    return ((y >> 7) & 1u) | ((y >> 14) & 2u) | ((y >> 21) & 4u) | ((y >> 28) & 8u);
+}
+
+// True when key tile j of a batch's key-padding row holds at least one key
+// that is not padded (a zero byte).  Bytes past N count as padded.  `vec`:
+// the row may be read 16 bytes at a time (16-byte aligned, N % 16 == 0).
+__device__ __forceinline__ bool pad_tile_has_key(const uint8_t* row, int j, int N, bool vec) {
+    const int k0 = j * kBlockN;
+    const int n = min(kBlockN, N - k0);
+    if (vec && n == kBlockN) {
+        uint32_t zero = 0u;
+#pragma unroll
+        for (int g = 0; g < kBlockN / 16; ++g) {
+            const uint4 x = ldg_nc16(row + k0 + 16 * g);
+            zero |= __vcmpeq4(x.x, 0u) | __vcmpeq4(x.y, 0u) | __vcmpeq4(x.z, 0u) | __vcmpeq4(x.w, 0u);
+        }
+        return zero != 0u;
+    }
+    for (int e = 0; e < n; ++e)
+        if (row[k0 + e] == 0) return true;
+    return false;
+}
+
+// The key tiles one Q tile visits, in increasing order.  In the sparse mode
+// (a block mask, a key-padding mask, or both) a tile is visited when its
+// block-mask bit is set (no block mask: every tile up to the causal bound)
+// and, with key padding, it holds a key that is not padded: tiles made only
+// of padded keys are neither loaded nor multiplied.  Every role evaluates the
+// same predicate for the same unit, so they all walk the same tiles.
 template <int MODE>
 struct KeyTiles {
     int lim;               // last key tile it may visit (-1: the tile has no rows)
     int off;               // sparse: bit index of its mask row, column 0
-    const uint32_t* bits;  // sparse: the block mask as bits, row-major, in shared memory
+    const uint32_t* bits;  // sparse: the block mask as bits, row-major, in shared memory (null: none)
+    const uint8_t* pad;    // sparse: the key-padding row of this unit's batch (null: none)
+    int n;                 // sparse with padding: keys N
+    bool pad_vec;          // sparse with padding: the row may be read 16 bytes at a time
 
+    __device__ __forceinline__ bool bit(int j) const {
+        return bits == nullptr || ((bits[(off + j) >> 5] >> ((off + j) & 31)) & 1u);
+    }
+    __device__ __forceinline__ bool keyed(int j) const { return pad == nullptr || pad_tile_has_key(pad, j, n, pad_vec); }
     __device__ __forceinline__ bool has(int j) const {
         if constexpr (MODE != kModeSparse) return j <= lim;
-        else return j <= lim && ((bits[(off + j) >> 5] >> ((off + j) & 31)) & 1u);
+        else return j >= 0 && j <= lim && bit(j) && keyed(j);
+    }
+    // first tile >= j whose block-mask bit is set (kNoTile if none)
+    __device__ __forceinline__ int next_bit(int j) const {
+        if (bits == nullptr) return j <= lim ? j : kNoTile;
+        while (j <= lim) {
+            const int f = off + j;
+            const uint32_t word = bits[f >> 5] >> (f & 31);
+            if (word != 0u) {
+                const int jj = j + __ffs(static_cast<int>(word)) - 1;
+                return jj <= lim ? jj : kNoTile;
+            }
+            j += 32 - (f & 31);
+        }
+        return kNoTile;
+    }
+    // last tile <= j whose block-mask bit is set (-1 if none)
+    __device__ __forceinline__ int prev_bit(int j) const {
+        if (bits == nullptr) return j;
+        while (j >= 0) {
+            const int f = off + j;
+            const uint32_t word = bits[f >> 5] << (31 - (f & 31));
+            if (word != 0u) {
+                const int jj = j - __clz(static_cast<int>(word));
+                return jj >= 0 ? jj : -1;
+            }
+            j -= (f & 31) + 1;
+        }
+        return -1;
     }
     // first key tile >= j (kNoTile if none)
     __device__ __forceinline__ int next(int j) const {
         if constexpr (MODE != kModeSparse) {
             return j <= lim ? j : kNoTile;
         } else {
-            while (j <= lim) {
-                const int f = off + j;
-                const uint32_t word = bits[f >> 5] >> (f & 31);
-                if (word != 0u) {
-                    const int jj = j + __ffs(static_cast<int>(word)) - 1;
-                    return jj <= lim ? jj : kNoTile;
-                }
-                j += 32 - (f & 31);
+            for (j = next_bit(j); j != kNoTile && !keyed(j); j = next_bit(j + 1)) {
             }
-            return kNoTile;
+            return j;
         }
     }
     // number of key tiles
@@ -208,15 +277,20 @@ struct KeyTiles {
             return lim + 1;
         } else {
             if (lim < 0) return 0;
+            if (pad != nullptr || bits == nullptr) {
+                int n_tiles = 0;
+                for (int j = next(0); j != kNoTile; j = next(j + 1)) ++n_tiles;
+                return n_tiles;
+            }
             const int f = off, e = off + lim;  // first and last bit, inclusive
-            int n = 0;
+            int n_tiles = 0;
             for (int wd = f >> 5; wd <= (e >> 5); ++wd) {
                 uint32_t x = bits[wd];
                 if (wd == (f >> 5)) x &= ~0u << (f & 31);
                 if (wd == (e >> 5)) x &= ~0u >> (31 - (e & 31));
-                n += __popc(x);
+                n_tiles += __popc(x);
             }
-            return n;
+            return n_tiles;
         }
     }
     // last key tile (-1 if none)
@@ -224,17 +298,9 @@ struct KeyTiles {
         if constexpr (MODE != kModeSparse) {
             return lim;
         } else {
-            int j = lim;
-            while (j >= 0) {
-                const int f = off + j;
-                const uint32_t word = bits[f >> 5] << (31 - (f & 31));
-                if (word != 0u) {
-                    const int jj = j - __clz(static_cast<int>(word));
-                    return jj >= 0 ? jj : -1;
-                }
-                j -= (f & 31) + 1;
-            }
-            return -1;
+            int j = prev_bit(lim);
+            while (j >= 0 && !keyed(j)) j = prev_bit(j - 1);
+            return j;
         }
     }
 };
@@ -249,7 +315,10 @@ __device__ __forceinline__ KeyTiles<MODE> key_tiles(const Unit& w, const Params&
     k.lim = (MODE == kModeSparse && w.q0 + t * kBlockM >= p.N) ? -1
             : causal ? min(p.n_kv_all - 1, qt) : p.n_kv_all - 1;
     k.off = qt * p.n_kv_all;
-    k.bits = bits;
+    k.bits = p.block_mask != nullptr ? bits : nullptr;
+    k.pad = p.key_pad != nullptr ? p.key_pad + static_cast<size_t>(w.b) * p.N : nullptr;
+    k.n = p.N;
+    k.pad_vec = p.pad_vec != 0;
     return k;
 }
 
@@ -725,6 +794,10 @@ __device__ __forceinline__ void role_mma_ordered(const Ctx& c) {
 }
 
 // ------------------------------------------------------- softmax + epilogue
+// Columns [32 G, 32 G + 32) of one row: p = 2^(sl2 * s - m) (negm = -m) as
+// 16 bf16 pairs in pk, summed into acc; the pairs marked in kPolyMask8 use
+// the FMA-pipe exponential and fold their raw scores into pmax, the rest
+// use MUFU (ex2.approx).
 // Warpgroup t owns Q tile t; thread = one query row = one TMEM lane.
 template <int D, int MODE, bool MASK>
 __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, uint16_t* __restrict__ out_o,
@@ -750,17 +823,18 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
     bool ok = true;
     int local = 0;
     uint32_t o_units = 0;  // sparse: units in which this Q tile has key tiles
-
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, ++local) {
         const Unit w = decode_unit<MODE>(u, p);
         const int row = w.q0 + t * kBlockM + r_in_tile;
         // step j visits key tile j (full, causal) or the j-th key tile kj of
         // this Q tile's mask row (sparse)
         const KeyTiles<MODE> kt = key_tiles<MODE>(w, p, c.mask_bits, t);
-        const int n_kv = kt.count();
+        // sparse: walk kt.next() until it runs out (no count: with key padding
+        // each step tests the mask bytes of the candidate tiles)
+        const int n_kv = MODE == kModeSparse ? 0 : kt.count();
         int kj = kt.next(0);
         if constexpr (MODE == kModeSparse) {
-            if (n_kv == 0) {
+            if (kj == kNoTile) {
                 // no key block at all: O = 0 and LSE = -inf, as for a row
                 // whose keys are all masked (no barrier of this unit is used)
                 if (row < p.N) {
@@ -778,7 +852,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
         float m = -INFINITY;  // reference max of scale*log2(e)*s (log2 units), shared by O and l
         float l = 0.f;        // sum of exp2(scale*log2(e)*s - m) over the keys seen so far
 
-        for (int j = 0; j < n_kv; ++j) {
+        for (int j = 0; MODE == kModeSparse ? kj != kNoTile : j < n_kv; ++j) {
             const int key_tile = MODE == kModeSparse ? kj : j;
             bool got = wait_bounded(b_s, s_phase, c.abort_flag, p.wait_ns);
             got = __all_sync(0xffffffffu, got);
@@ -807,30 +881,35 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
                 tc_fence_before();
                 mbar_arrive(b_sfree);
             }
-            // key padding: the 128 mask bytes of this key tile, 16 at a time;
-            // only 16-key groups that hold a padded key are touched
+            // key padding: the 128 mask bytes of this key tile, requested all
+            // at once (one round trip when they can be read 16 at a time); only
+            // 16-key groups that hold a padded key are touched
             if (MASK) {
                 const int key0 = key_tile * kBlockN;
                 const uint8_t* mrow = p.key_pad + static_cast<size_t>(w.b) * p.N + key0;
-                const bool vec = p.pad_vec && key0 + kBlockN <= p.N;
-#pragma unroll
-                for (int g = 0; g < kBlockN / 16; ++g) {
-                    uint4 x;
-                    if (vec) {
-                        x = ldg_nc16(mrow + 16 * g);
-                    } else {
-                        uint32_t wd[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            if (key0 + 16 * g + e < p.N)
-                                wd[e >> 2] |= static_cast<uint32_t>(mrow[16 * g + e] != 0) << (8 * (e & 3));
-                        x = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-                    }
+                auto mask16 = [&](int g, uint4 x) {
                     if (x.x | x.y | x.z | x.w) {
                         const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                         for (int e = 0; e < 16; ++e)
                             if ((wv[e >> 2] >> (8 * (e & 3))) & 0xFFu) s[16 * g + e] = -INFINITY;
+                    }
+                };
+                if (p.pad_vec && key0 + kBlockN <= p.N) {
+                    uint4 x[kBlockN / 16];
+#pragma unroll
+                    for (int g = 0; g < kBlockN / 16; ++g) x[g] = ldg_nc16(mrow + 16 * g);
+#pragma unroll
+                    for (int g = 0; g < kBlockN / 16; ++g) mask16(g, x[g]);
+                } else {
+#pragma unroll
+                    for (int g = 0; g < kBlockN / 16; ++g) {
+                        uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (key0 + 16 * g + e < p.N)
+                                wd[e >> 2] |= static_cast<uint32_t>(mrow[16 * g + e] != 0) << (8 * (e & 3));
+                        mask16(g, make_uint4(wd[0], wd[1], wd[2], wd[3]));
                     }
                 }
             }
@@ -854,7 +933,8 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
             }
             const float row_max = fmax3(fmax3(mx[0], mx[1], mx[2]), mx[3], -INFINITY) * sl2;
             // lazy rescaling: move the reference only when the row maximum
-            // exceeds it by more than 2^8 (always on the first tile)
+            // exceeds it by more than 2^8 (always on a row's first visible key);
+            // O and l always share the reference, so the result stays exact
             const bool move = row_max > m + kLazyRescaleLog2;
             float alpha = 1.f;
             if (move) {
@@ -867,7 +947,8 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
             const float2 negm = make_float2(-m_use, -m_use);
 
             // P = exp2(scale*log2(e)*s - m) as bf16 pairs; the pairs marked in
-            // kPolyMask8 use the FMA-pipe exponential, the rest MUFU.
+            // kPolyMask8 use the FMA-pipe exponential, the rest MUFU; masked
+            // scores (-inf) give exactly +0 on both.
             float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
             uint32_t pk[kBlockN / 2];
 #pragma unroll
@@ -965,10 +1046,6 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
 // Sparse mode: the [n_kv_all, n_kv_all] block-mask bytes become bits in shared
 // memory (bit f = byte f != 0, row-major), every thread taking whole 32-bit
 // words; full words read the bytes 16 at a time (the mask is 16-byte aligned).
-__device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t x) {
-    const uint32_t y = __vcmpne4(x, 0u);  // 0xFF per nonzero byte
-    return ((y >> 7) & 1u) | ((y >> 14) & 2u) | ((y >> 21) & 4u) | ((y >> 28) & 8u);
-}
 __device__ __forceinline__ void stage_block_mask(const Params& p, uint32_t* bits) {
     const long long total = static_cast<long long>(p.n_kv_all) * p.n_kv_all;
     const int words = static_cast<int>((total + 31) / 32);
@@ -1039,7 +1116,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_relinquish();
     }
     uint32_t* const mask_bits = reinterpret_cast<uint32_t*>(gbase + C::kMaskOff);
-    if (MODE == kModeSparse) stage_block_mask(p, mask_bits);
+    if (MODE == kModeSparse && p.block_mask != nullptr) stage_block_mask(p, mask_bits);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1083,6 +1160,20 @@ __global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
     __syncthreads();
     if (threadIdx.x == 0) wait_bounded(bar, 0, nullptr, limit_ns);
     __syncthreads();
+}
+
+// Evaluates the softmax's FMA-pipe exponential on a device buffer, two
+// elements per call as the kernel does, so that it can be checked against
+// 2^x on the host.  One thread per pair; an odd last element is paired with
+// itself.
+__global__ void ex2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+    const int pairs = (n + 1) / 2;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < pairs; i += gridDim.x * blockDim.x) {
+        const int a = 2 * i, b = min(2 * i + 1, n - 1);
+        const float2 r = ex2_poly2(make_float2(x[a], x[b]));
+        y[a] = r.x;
+        if (b != a) y[b] = r.y;
+    }
 }
 
 // ---------------------------------------------------------------- host side
@@ -1133,6 +1224,53 @@ bool encode_qkv_map(CUtensorMap* map, const void* ptr, int B, int H, int N, int 
                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor maps of recent calls.  A map is a pure function of (address, sizes,
+// strides), so a hit is always the map a fresh encode would give, whatever
+// happened to the memory in between; the cache only saves the encode.
+struct MapCache {
+    struct Entry {
+        const void* ptr;
+        int B, H, N, d;
+        long long sb, sh, sn;
+        bool used;
+        CUtensorMap map;
+    };
+    static constexpr int kEntries = 24;
+    std::mutex m;
+    Entry e[kEntries] = {};
+    int next = 0;
+};
+
+bool cached_qkv_map(CUtensorMap* map, const void* ptr, int B, int H, int N, int d, long long sb, long long sh,
+                    long long sn) {
+    static MapCache cache;
+    std::lock_guard<std::mutex> lock(cache.m);
+    for (const MapCache::Entry& x : cache.e)
+        if (x.used && x.ptr == ptr && x.B == B && x.H == H && x.N == N && x.d == d && x.sb == sb && x.sh == sh &&
+            x.sn == sn) {
+            *map = x.map;
+            return true;
+        }
+    if (!encode_qkv_map(map, ptr, B, H, N, d, sb, sh, sn)) return false;
+    MapCache::Entry& x = cache.e[cache.next];
+    cache.next = (cache.next + 1) % MapCache::kEntries;
+    x = MapCache::Entry{ptr, B, H, N, d, sb, sh, sn, true, *map};
+    return true;
+}
+
+constexpr int kMaxDevices = 64;
+
+// Multiprocessor count of a device, looked up once per device (0 on failure).
+int sm_count(int dev) {
+    static std::atomic<int> cached[kMaxDevices] = {};
+    if (dev < 0 || dev >= kMaxDevices) return 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 0;
+    cached[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 // Largest element offset + 1 of a [B, H, N, d] tensor with the given strides
 // (0 if it would not fit in 2^46 elements).
 size_t span_elems(int B, int H, int N, int d, long long sb, long long sh, long long sn) {
@@ -1163,17 +1301,61 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
+// True when the d-element rows (b, h, n) of a strided [B, H, N, d] output are
+// nested without overlap: taking the dimensions of extent > 1 by increasing
+// stride, each stride is at least the span of the rows below it.  Every
+// layout in which rows of different (b, h, n) could share an element fails
+// (CTAs would write the same bytes in no defined order); so do a few exotic
+// interleavings that happen to be disjoint.
+bool rows_nested(int B, int H, int N, int d, long long sb, long long sh, long long sn) {
+    struct Dim { long long stride, extent; } dims[3] = {{sb, B}, {sh, H}, {sn, N}};
+    for (int i = 1; i < 3; ++i)  // insertion sort by stride
+        for (int j = i; j > 0 && dims[j].stride < dims[j - 1].stride; --j) {
+            const Dim t = dims[j];
+            dims[j] = dims[j - 1];
+            dims[j - 1] = t;
+        }
+    long long span = d;  // elements covered by the rows of the smaller-stride dimensions
+    for (const Dim& x : dims) {
+        if (x.extent <= 1) continue;
+        if (x.stride < span) return false;
+        span += (x.extent - 1) * x.stride;  // stride <= 2^36 and extent < 2^31: no overflow
+    }
+    return true;
+}
+
+// Causal unit order: the K and V of the heads in flight should fit in about a
+// third of the 126 MB L2.
+constexpr long long kL2GroupBytes = 40LL << 20;
+
 // Largest block-mask side the shared-memory bit copy takes (N <= 65536).
 constexpr int kMaxMaskTiles = 512;
 
 template <int D, int MODE, bool MASK>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
-           const Params& p, int grid, cudaStream_t stream) {
+           const Params& p, int grid, int dev, cudaStream_t stream) {
     auto kernel = attn_fwd_kernel<D, MODE, MASK>;
-    const long long bits = static_cast<long long>(p.n_kv_all) * p.n_kv_all;
+    const long long bits = p.block_mask != nullptr ? static_cast<long long>(p.n_kv_all) * p.n_kv_all : 0;
     const int smem = Cfg<D>::kSmemBytes + (MODE == kModeSparse ? static_cast<int>((bits + 127) / 128) * 16 : 0);
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return ATTN_ERR_CUDA;
+    // the dynamic shared-memory limit of this instantiation, raised once per
+    // device to the largest size asked for so far
+    // device and context (a reset or a new context starts from the default)
+    static std::mutex m;
+    static int smem_set[kMaxDevices] = {};
+    static unsigned long long ctx_of[kMaxDevices] = {};
+    {
+        std::lock_guard<std::mutex> lock(m);
+        const unsigned long long ctx = current_context_id();
+        const bool known = dev >= 0 && dev < kMaxDevices && ctx != 0 && ctx_of[dev] == ctx;
+        if (!known || smem > smem_set[dev]) {
+            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+            if (dev >= 0 && dev < kMaxDevices && ctx != 0) {
+                smem_set[dev] = smem;
+                ctx_of[dev] = ctx;
+            }
+        }
+    }
     kernel<<<grid, kThreads, smem, stream>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -1217,6 +1399,7 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
     for (long long st : {qkv_sb, qkv_sh, qkv_sn, o_sb, o_sh, o_sn})
         if (st < 8 || st % 8 != 0 || st > lim) return ATTN_ERR_INVALID_ARG;
     if (qkv_sn < d || o_sn < d) return ATTN_ERR_INVALID_ARG;  // rows must not overlap
+    if (!rows_nested(B, H, N, d, o_sb, o_sh, o_sn)) return ATTN_ERR_INVALID_ARG;  // no two O rows may alias
     auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0; };
     if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) || misaligned(lse, 4))
         return ATTN_ERR_INVALID_ARG;
@@ -1246,14 +1429,13 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
         (key_padding_mask && !device_span_ok(key_padding_mask, pad_bytes, dev)) ||
         (block_mask && !device_span_ok(block_mask, bm_bytes, dev)))
         return ATTN_ERR_INVALID_ARG;
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
-        return ATTN_ERR_CUDA;
+    const int sms = sm_count(dev);
+    if (sms < 1) return ATTN_ERR_CUDA;
 
     alignas(64) CUtensorMap mq, mk, mv;
-    if (!encode_qkv_map(&mq, q, B, H, N, d, qkv_sb, qkv_sh, qkv_sn) ||
-        !encode_qkv_map(&mk, k, B, H, N, d, qkv_sb, qkv_sh, qkv_sn) ||
-        !encode_qkv_map(&mv, v, B, H, N, d, qkv_sb, qkv_sh, qkv_sn))
+    if (!cached_qkv_map(&mq, q, B, H, N, d, qkv_sb, qkv_sh, qkv_sn) ||
+        !cached_qkv_map(&mk, k, B, H, N, d, qkv_sb, qkv_sh, qkv_sn) ||
+        !cached_qkv_map(&mv, v, B, H, N, d, qkv_sb, qkv_sh, qkv_sn))
         return ATTN_ERR_CUDA;
 
     Params p;
@@ -1274,18 +1456,25 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
     p.total_units = static_cast<int>(units);
     p.scale_log2 = scale * kLog2e;
     p.wait_ns = kDefaultWaitNs;
+    {
+        const long long kv_bytes = 4LL * N * d;  // K and V of one head, bf16
+        const long long g = kL2GroupBytes / kv_bytes;
+        p.group_heads = static_cast<int>(g < 1 ? 1 : g > BH ? BH : g);
+    }
     const int grid = static_cast<int>(units < sms ? units : sms);
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool pad = key_padding_mask != nullptr;
-    const int mode = block_mask ? kModeSparse : causal ? kModeCausal : kModeFull;
-#define ATTN_LAUNCH(D_, M_, P_) launch<D_, M_, P_>(mq, mk, mv, o, lse, p, grid, s)
-#define ATTN_BY_MODE(D_, P_)                                      \
-    (mode == kModeSparse   ? ATTN_LAUNCH(D_, kModeSparse, P_)     \
-     : mode == kModeCausal ? ATTN_LAUNCH(D_, kModeCausal, P_)     \
-                           : ATTN_LAUNCH(D_, kModeFull, P_))
-    if (d == 64) return pad ? ATTN_BY_MODE(64, true) : ATTN_BY_MODE(64, false);
-    return pad ? ATTN_BY_MODE(128, true) : ATTN_BY_MODE(128, false);
+    // a block mask or key padding selects the tile-list loops (only visited
+    // tiles are loaded and multiplied); key padding also masks per key
+    const int mode = (block_mask || pad) ? kModeSparse : causal ? kModeCausal : kModeFull;
+#define ATTN_LAUNCH(D_, M_, P_) launch<D_, M_, P_>(mq, mk, mv, o, lse, p, grid, dev, s)
+#define ATTN_BY_MODE(D_)                                                                   \
+    (pad                   ? ATTN_LAUNCH(D_, kModeSparse, true)                            \
+     : mode == kModeSparse ? ATTN_LAUNCH(D_, kModeSparse, false)                           \
+     : mode == kModeCausal ? ATTN_LAUNCH(D_, kModeCausal, false)                           \
+                           : ATTN_LAUNCH(D_, kModeFull, false))
+    return d == 64 ? ATTN_BY_MODE(64) : ATTN_BY_MODE(128);
 #undef ATTN_BY_MODE
 #undef ATTN_LAUNCH
 }
@@ -1314,6 +1503,21 @@ int attn_check_device_status(attn_stream_t stream) {
     if (attn_bwd_take_device_status(&bwd_status) != ATTN_OK) return ATTN_ERR_CUDA;
     if (status == 0) status = bwd_status;
     return status == 0 ? ATTN_OK : status;
+}
+
+int attn_selftest_ex2(const float* x, float* y, int n, attn_stream_t stream) {
+    if (n < 1 || !x || !y) return ATTN_ERR_INVALID_ARG;
+    const size_t bytes = static_cast<size_t>(n) * 4;
+    if ((reinterpret_cast<uintptr_t>(x) & 3) || (reinterpret_cast<uintptr_t>(y) & 3) || overlaps(x, bytes, y, bytes))
+        return ATTN_ERR_INVALID_ARG;
+    if (!driver_fns().ok) return ATTN_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (!device_span_ok(x, bytes, dev) || !device_span_ok(y, bytes, dev)) return ATTN_ERR_INVALID_ARG;
+    const int pairs = (n + 1) / 2;
+    const int grid = pairs / 256 + 1 < 1024 ? pairs / 256 + 1 : 1024;
+    ex2_selftest_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int attn_selftest_wait_timeout(unsigned long long limit_ns, attn_stream_t stream) {

@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "attn.h"
 
 namespace {
@@ -195,13 +197,25 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// 32 lanes x 32 bits, 16 consecutive columns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 // 16 bytes through the read-only path (every thread of a warpgroup reads the
-// same mask bytes: one broadcast transaction, then L1 hits).
+// same mask bytes: one broadcast transaction, then L1 hits).  Only for
+// memory that no thread writes during the kernel; not volatile, so the
+// compiler may issue several of them before their first use.
 __device__ __forceinline__ uint4 ldg_nc16(const void* p) {
     uint4 r;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
+    asm("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
     return r;
 }
 
@@ -231,23 +245,27 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// 2^x for x <= 8 on the FMA/ALU pipes (no MUFU), two lanes at a time:
+// 2^x on the FMA/ALU pipes (no MUFU), two lanes at a time, for x <= 127:
 // x = j + f with j = round(x) and f in [-1/2, 1/2]; 2^f from a degree-3
-// polynomial fitted for minimal relative error on [-1/2, 1/2]
-// (fit_exp2_poly.py; max relative error 7.6e-5, far below the bf16 rounding
-// that P gets); 2^j by adding j to the exponent field.  x is clamped at -126
-// so the exponent never wraps (2^-126 stands in for 0).
+// polynomial with constant term exactly 1, its other coefficients fitted for
+// minimal relative error on [-1/2, 1/2] (fit_exp2_poly.py: max relative error
+// 1.013e-4, far below the bf16 rounding that P gets); 2^j by adding j to the
+// exponent field.  x is first clamped at -127: there j = -127, f = 0 and the
+// polynomial is exactly 1, so the exponent field becomes exactly 0 and the
+// result is +0 for every x <= -127, -inf (a masked score) included; for
+// -127 < x < -126 it is a subnormal below 2^-126.  Larger x than 127 is the
+// caller's to exclude (the exponent field would wrap).
 __device__ __forceinline__ float2 ex2_poly2(float2 x) {
     constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
-    constexpr float kC0 = 0.99992824f, kC1 = 0.6932636f, kC2 = 0.2426099f, kC3 = 0.05515746f;
-    x.x = fmaxf(x.x, -126.0f);
-    x.y = fmaxf(x.y, -126.0f);
+    constexpr float kC1 = 0.6932829f, kC2 = 0.24221095f, kC3 = 0.05500893f;
+    x.x = fmaxf(x.x, -127.0f);
+    x.y = fmaxf(x.y, -127.0f);
     const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
     const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
     const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
     float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
     q = __ffma2_rn(q, f, make_float2(kC1, kC1));
-    q = __ffma2_rn(q, f, make_float2(kC0, kC0));
+    q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
     // the low mantissa bits of t hold j (two's complement); t * 2^23 moves them
     // to the exponent field, added to q in one integer multiply-add
     uint32_t rx, ry;
@@ -273,6 +291,36 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool b_mn_ma
            | (1u << 10)                     // B format bf16
            | ((b_mn_major ? 1u : 0u) << 16)  // B major
            | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Process-unique id of the current CUDA context (cuCtxGetId), 0 if there is
+// none or it cannot be read.  Ids are never reused, unlike context handles,
+// so a cache keyed by it goes stale neither after a device reset nor across
+// contexts.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q1, q2;
+        void *f1 = nullptr, *f2 = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+            q2 == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+            get_id = reinterpret_cast<CtxGetIdFn>(f2);
+        }
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
 }
 
 }  // namespace

@@ -11,7 +11,8 @@
  * computed tile by tile in one kernel with a running row maximum m and a
  * running row sum l, so the N x N score and probability matrices never reach
  * device memory; the softmax statistics are kept as one fp32 log-sum-exp per
- * query row (the notes' "keep only O and the softmax statistics (m, l)").
+ * query row (per the notes' section "Recomputation", only O and the row
+ * statistics outlive the kernel).
  * With causal != 0, key j is visible to query i iff j <= i (square, top-left
  * aligned); tiles entirely above the diagonal are never computed.
  *
@@ -87,10 +88,13 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  *
  * Every stride must be a positive multiple of 8 (16 bytes, for the tensor
  * memory accelerator and the 16-byte O stores), qkv_sn and o_sn at least d,
- * and each pointer's allocation must cover its strided span; otherwise
- * ATTN_ERR_INVALID_ARG and nothing is launched.  Other arguments, ownership
- * and errors as attn_fwd (which is this call with contiguous strides and no
- * padding).
+ * and each pointer's allocation must cover its strided span.  The d-element
+ * rows of O must not alias: taking the dimensions of O with extent > 1 in
+ * order of increasing stride, each stride must be at least the span of the
+ * rows below it (every contiguous or transposed layout, [B, N, H, d]
+ * included, meets this).  Otherwise ATTN_ERR_INVALID_ARG and nothing is
+ * launched.  Other arguments, ownership and errors as attn_fwd (which is
+ * this call with contiguous strides and no padding).
  */
 int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
                      int B, int H, int N, int d,
@@ -179,8 +183,10 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
  * delta is kept in a static device array of the library (1 << 20 fp32 rows,
  * 4 MiB, part of the module image), so B*H*N must be at most 1048576
  * (otherwise ATTN_ERR_INVALID_ARG, checked before anything runs).  Its
- * address is looked up once per device (cudaGetSymbolAddress) on the first
- * call on that device: make that first call outside stream capture.  The
+ * address is looked up (cudaGetSymbolAddress) on the first call in each CUDA
+ * context of a device and cached under that context's id, so a device reset
+ * or a new context looks it up again: make the first call in a context
+ * outside stream capture.  The
  * array is shared by every call on a device, so calls whose executions may
  * overlap (different streams without ordering between them) race on it:
  * order them on one stream or by events.  Everything else as attn_bwd.
@@ -209,6 +215,28 @@ int attn_check_device_status(attn_stream_t stream);
  * returns normally; attn_check_device_status() then reports it.
  */
 int attn_selftest_wait_timeout(unsigned long long limit_ns, attn_stream_t stream);
+
+/*
+ * attn_selftest_ex2 -- evaluate, on the device, the exponential that the
+ * forward's softmax runs on the FMA pipe for part of its 2^x evaluations
+ * (a degree-3 polynomial for 2^f on [-1/2, 1/2] with 2^round(x) put into the
+ * exponent field), so that callers and tests can check it against 2^x.
+ *
+ *   x : fp32 [n] device buffer of arguments (read only).
+ *   y : fp32 [n] device buffer, written: y[i] ~ 2^x[i] for x[i] <= 127,
+ *       relative error at most 1.02e-4 for -126 <= x[i] <= 127; exactly +0
+ *       for x[i] <= -127 and for x[i] = -inf (a masked score); a subnormal
+ *       below 2^-126 for -127 < x[i] < -126.
+ *   n : >= 1.  x and y must be 4-byte aligned, must not overlap, and must lie
+ *       in device memory of the current device covering n floats
+ *       (ATTN_ERR_INVALID_ARG otherwise; nothing is launched).
+ *
+ * The polynomial is not the page's: the notes compute the softmax with exact
+ * exponentials; this is how part of them is evaluated on B200, and the test
+ * entry point exists so that its accuracy can be pinned.
+ * Asynchronous on `stream`.
+ */
+int attn_selftest_ex2(const float* x, float* y, int n, attn_stream_t stream);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int attn_version(void);

@@ -106,6 +106,31 @@ def test_bad_strides_rejected_on_host(lib, qkv, o):
                                 None) == pkg.ATTN_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("H,N,o", [
+    (2, 64, (8192, 8, 64)),        # heads 8 elements apart: rows of head 0 and 1 share bytes
+    (2, 64, (8192, 64, 64)),       # head stride = row stride: (h=1, n) is (h=0, n+1)
+    (2, 64, (8192, 4096, 128)),    # head stride inside the span of one head's rows
+    (3, 64, (65536, 64, 128)),     # interleaved heads, 3 heads in a 2-row stride
+])
+def test_aliasing_output_rows_rejected(lib, H, N, o):
+    # two different (b, h, n) rows of O would overlap: rejected before any launch
+    dense = (H * N * 64, N * 64, 64)
+    assert pkg.attn_fwd_strided(GIB, 2 * GIB, 3 * GIB, 4 * GIB, 5 * GIB, 1, H, N, 64, dense, o, 0.125, 0,
+                                None) == pkg.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("H,N,o", [
+    (2, 64, (8192, 4096, 64)),     # contiguous [B, H, N, d]
+    (2, 64, (8192, 64, 128)),      # [B, N, H, d]: heads interleaved, rows nested
+    (1, 64, (8192, 8, 64)),        # the stride of a size-1 dimension is never used
+])
+def test_nested_output_rows_accepted(lib, H, N, o):
+    dense = (H * N * 64, N * 64, 64)
+    # passes the host checks; with no GPU here it fails only at the driver
+    assert pkg.attn_fwd_strided(GIB, 2 * GIB, 3 * GIB, 4 * GIB, 5 * GIB, 1, H, N, 64, dense, o, 0.125, 0,
+                                None) not in (pkg.ATTN_ERR_INVALID_ARG, pkg.ATTN_OK)
+
+
 def test_strided_overlap_uses_the_strided_span(lib):
     # O's span under its strides reaches into q's allocation range: rejected
     base = 1 << 24

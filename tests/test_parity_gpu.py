@@ -54,6 +54,26 @@ def test_tiny_config_full():
     check(1, 2, 128, 64, False)
 
 
+# ---- the 12-argument entry point itself, attn_fwd(q, k, v, o, lse, B, H, N, d,
+# scale, causal, stream), on contiguous device buffers, against the oracle
+@pytest.mark.parametrize("B,H,N,d", [(1, 2, 128, 64), (1, 16, 1944, 64), (2, 3, 700, 128)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_attn_fwd_entry_point_full(B, H, N, d, causal):
+    dev = torch.device("cuda:0")
+    q, k, v = make_qkv(B, H, N, d, seed=N + d)
+    qd, kd, vd = (x.to(dev).contiguous() for x in (q, k, v))
+    o = torch.full((B, H, N, d), 7.0, dtype=torch.bfloat16, device=dev)
+    lse = torch.full((B, H, N), 7.0, dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(d)
+    st = pkg.attn_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d, scale,
+                      causal, torch.cuda.current_stream().cuda_stream)
+    assert st == pkg.ATTN_OK
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    o_ref, lse_ref = oracle.attention_rows(q, k, v, scale, causal)
+    assert np.abs(o.float().cpu().numpy().reshape(o_ref.shape) - o_ref).max() <= TOL_O
+    assert np.abs(lse.cpu().numpy().reshape(lse_ref.shape) - lse_ref).max() <= TOL_LSE
+
+
 # ---- several tiles plus ragged tails, both head sizes, both masks: full comparison
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
@@ -230,6 +250,32 @@ def test_key_padding_fully_padded_batch_and_no_padding():
     o1, l1 = pkg.forward(q, k, v, key_padding_mask=none)
     o2, l2 = pkg.forward(q, k, v)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_padding_skips_padded_tiles_full(causal):
+    # the 0.5 MP shape with two batches, the second one's last 1024 patches
+    # padded: 8 of its 16 key tiles hold only padded keys and are skipped
+    # (never loaded or multiplied); the partly padded tile is masked per key.
+    # Full element-wise comparison with the oracle.
+    B, H, N, d = 2, 16, 1944, 64
+    pad = np.zeros((B, N), dtype=bool)
+    pad[1, N - 1024:] = True
+    masked_check(B, H, N, d, causal, pad, seed=5)
+
+
+def test_key_padding_skipped_tiles_in_the_middle_full():
+    # whole padded key tiles between visible ones, at both head sizes, and a
+    # batch whose only visible keys sit in its last (ragged) tile
+    for d in (64, 128):
+        B, H, N = 3, 2, 1000
+        pad = np.zeros((B, N), dtype=bool)
+        pad[0, 128:512] = True            # key tiles 1-3 skipped
+        pad[1, :896] = True               # only the ragged last tile is visible
+        pad[2, 256:384] = True
+        pad[2, 640:] = True               # tiles 2, 5, 6, 7 skipped
+        for causal in (False, True):
+            masked_check(B, H, N, d, causal, pad, seed=d + int(causal))
 
 
 def test_key_padding_image_workload_sampled():
