@@ -110,7 +110,6 @@ struct Bars {
 
 struct BwdParams {
     int BH, H, N, n_kb, n_qt, total_units, causal;
-    int group_heads;            // causal unit order: heads per group (their Q, dO, dQ fit in L2)
     const uint8_t* key_pad;     // [B, N] (nonzero = padded key) or null
     const uint8_t* block_mask;  // [n_bt, n_bt] (nonzero = block computed) or null
     int n_bt;                   // ceil(N / 128)
@@ -129,18 +128,18 @@ struct BwdUnit {
 
 // Units: (head, key block).  Non-causal: heads-major, so the CTAs running at
 // one time stream the same Q / dO tiles (L2 reuse).  Causal: key block kb
-// meets query tiles kb .. n_qt-1; heads go in groups of p.group_heads, whose
-// Q, dO and dQ together fit in a third of L2, and within a group the blocks
-// with most tiles go first.
+// meets query tiles kb .. n_qt-1; the blocks with most tiles go first, and
+// since CTA c takes units c, c + grid, ..., odd rounds run that list
+// backwards ("snake" order) so that every CTA's total is close to the mean.
 __device__ __forceinline__ BwdUnit bwd_unit(int u, const BwdParams& p) {
     BwdUnit w;
     if (p.causal) {
-        const int per_group = p.group_heads * p.n_kb;
-        const int g = u / per_group;
-        const int r = u - g * per_group;
-        const int gh = min(p.group_heads, p.BH - g * p.group_heads);  // heads in this group
-        w.kb = r / gh;
-        w.bh = g * p.group_heads + (r - w.kb * gh);
+        const int g = static_cast<int>(gridDim.x);
+        const int k = u / g, c = u - k * g;
+        const int rem = min(g, p.total_units - k * g);  // the last round may be partial
+        const int pos = (k & 1) ? k * g + (rem - 1 - c) : u;
+        w.kb = pos / p.BH;
+        w.bh = pos - w.kb * p.BH;
         w.i0 = w.kb;
     } else {
         w.bh = u / p.n_kb;
@@ -1380,11 +1379,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if (units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     p.total_units = static_cast<int>(units);
     p.causal = causal ? 1 : 0;
-    {
-        const long long head_bytes = 8LL * N * d;  // Q and dO (bf16) and dQ (fp32) of one head
-        const long long g = (40LL << 20) / head_bytes;
-        p.group_heads = static_cast<int>(g < 1 ? 1 : g > BH ? BH : g);
-    }
     p.scale = scale;
     p.scale_log2 = scale * kLog2eB;
     p.lse = lse;

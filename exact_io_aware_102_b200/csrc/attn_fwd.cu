@@ -128,6 +128,7 @@ struct Bars {
     static constexpr int kKEmpty = 208;    // [8] MMA -> TMA: K (or K/V) ring slot free
     static constexpr int kVFull = 272;     // [8] V ring (split layout)
     static constexpr int kVEmpty = 336;    // [8]
+    static constexpr int kPadRows = 400;   // int: staged key-padding rows
 };
 
 // ------------------------------------------------------------- the scheduler
@@ -139,10 +140,15 @@ enum : int { kModeFull = 0, kModeCausal = 1, kModeSparse = 2 };
 
 struct Params {
     int BH, H, N, n_pairs, n_kv_all, total_units;
-    int group_heads;             // causal unit order: heads per group (K/V of a group fit in L2)
     long long o_sb, o_sh, o_sn;  // element strides of O over (batch, head, row)
     const uint8_t* key_pad;      // [B, N] key-padding mask (nonzero = padded) or null
     int pad_vec;                 // key_pad rows may be read 16 bytes at a time
+    // key padding staged in shared memory as one bit per key (set = padded,
+    // keys >= N included), one row per batch that the CTA's units touch:
+    int pad_staged;              // 0: not staged (no tile is skipped; masks read from global memory)
+    int pad_row_words;           // 32-bit words per row (4 per key tile)
+    int pad_units;               // units per CTA at most (entries of the unit -> row map)
+    int pad_map_off, pad_rowb_off, pad_rows_off;  // byte offsets of the map, row batches and rows
     const uint8_t* block_mask;   // [n_kv_all, n_kv_all] block mask (nonzero = computed), sparse mode
     int causal;                  // causal bound on top of the block mask (sparse mode)
     float scale_log2;  // scale * log2(e)
@@ -151,27 +157,29 @@ struct Params {
 
 struct Unit {
     int bh, b, h, q0;  // head (flat, batch, within batch), first query row
+    int local;         // index of the unit among this CTA's units
 };
 
 // Work units: (head, pair of Q tiles).  Non-causal: heads-major so the CTAs
-// running at one time share K/V of few heads (L2 reuse).  Causal: heads in
-// groups of p.group_heads, whose K and V together fit in a third of L2; within
-// a group the pairs with the most key tiles come first, so that the short
-// units fill the tail while the CTAs running at one time read the K/V of
-// about one group only (ungrouped longest-first streams every head's K/V at
-// once and re-reads them from DRAM).
+// running at one time share K/V of few heads (L2 reuse).  Causal: the pairs
+// with the most key tiles first.  CTA c takes units c, c + grid, c + 2 grid,
+// ...; with units of unequal cost a plain round-robin over a longest-first
+// list gives CTA 0 the longest unit of every round, so odd rounds run the
+// list backwards ("snake" order): each CTA's total comes out close to the
+// mean.
 template <int MODE>
 __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     Unit w;
     int pair;
     const bool longest_first = MODE == kModeCausal || (MODE == kModeSparse && p.causal);
     if (longest_first) {
-        const int per_group = p.group_heads * p.n_pairs;
-        const int g = u / per_group;
-        const int r = u - g * per_group;
-        const int gh = min(p.group_heads, p.BH - g * p.group_heads);  // heads in this group
-        pair = p.n_pairs - 1 - r / gh;
-        w.bh = g * p.group_heads + r % gh;
+        // the last round may be partial: reverse it within its own length
+        const int g = static_cast<int>(gridDim.x);
+        const int k = u / g, c = u - k * g;
+        const int rem = min(g, p.total_units - k * g);
+        const int pos = (k & 1) ? k * g + (rem - 1 - c) : u;
+        pair = p.n_pairs - 1 - pos / p.BH;
+        w.bh = pos % p.BH;
     } else {
         pair = u % p.n_pairs;
         w.bh = u / p.n_pairs;
@@ -179,6 +187,7 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     w.b = w.bh / p.H;
     w.h = w.bh - w.b * p.H;
     w.q0 = pair * kUnitRows;
+    w.local = (u - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
     return w;
 }
 
@@ -190,24 +199,9 @@ __device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t x) {
     return ((y >> 7) & 1u) | ((y >> 14) & 2u) | ((y >> 21) & 4u) | ((y >> 28) & 8u);
 }
 
-// True when key tile j of a batch's key-padding row holds at least one key
-// that is not padded (a zero byte).  Bytes past N count as padded.  `vec`:
-// the row may be read 16 bytes at a time (16-byte aligned, N % 16 == 0).
-__device__ __forceinline__ bool pad_tile_has_key(const uint8_t* row, int j, int N, bool vec) {
-    const int k0 = j * kBlockN;
-    const int n = min(kBlockN, N - k0);
-    if (vec && n == kBlockN) {
-        uint32_t zero = 0u;
-#pragma unroll
-        for (int g = 0; g < kBlockN / 16; ++g) {
-            const uint4 x = ldg_nc16(row + k0 + 16 * g);
-            zero |= __vcmpeq4(x.x, 0u) | __vcmpeq4(x.y, 0u) | __vcmpeq4(x.z, 0u) | __vcmpeq4(x.w, 0u);
-        }
-        return zero != 0u;
-    }
-    for (int e = 0; e < n; ++e)
-        if (row[k0 + e] == 0) return true;
-    return false;
+// The 128 padding bits of key tile j in a staged row (bit set = padded).
+__device__ __forceinline__ uint4 pad_tile_bits(const uint32_t* row, int j) {
+    return *reinterpret_cast<const uint4*>(row + 4 * j);
 }
 
 // The key tiles one Q tile visits, in increasing order.  In the sparse mode
@@ -221,14 +215,16 @@ struct KeyTiles {
     int lim;               // last key tile it may visit (-1: the tile has no rows)
     int off;               // sparse: bit index of its mask row, column 0
     const uint32_t* bits;  // sparse: the block mask as bits, row-major, in shared memory (null: none)
-    const uint8_t* pad;    // sparse: the key-padding row of this unit's batch (null: none)
-    int n;                 // sparse with padding: keys N
-    bool pad_vec;          // sparse with padding: the row may be read 16 bytes at a time
+    const uint32_t* pad;   // sparse: the staged padding bits of this unit's batch (null: none)
 
     __device__ __forceinline__ bool bit(int j) const {
         return bits == nullptr || ((bits[(off + j) >> 5] >> ((off + j) & 31)) & 1u);
     }
-    __device__ __forceinline__ bool keyed(int j) const { return pad == nullptr || pad_tile_has_key(pad, j, n, pad_vec); }
+    __device__ __forceinline__ bool keyed(int j) const {
+        if (pad == nullptr) return true;
+        const uint4 b = pad_tile_bits(pad, j);
+        return (b.x & b.y & b.z & b.w) != ~0u;  // some key of the tile is not padded
+    }
     __device__ __forceinline__ bool has(int j) const {
         if constexpr (MODE != kModeSparse) return j <= lim;
         else return j >= 0 && j <= lim && bit(j) && keyed(j);
@@ -305,8 +301,15 @@ struct KeyTiles {
     }
 };
 
+// Per-CTA shared-memory copies of the masks (sparse mode).
+struct Masks {
+    const uint32_t* bits;      // block mask bits, or null
+    const uint16_t* pad_map;   // local unit index -> staged padding row, or null
+    const uint32_t* pad_rows;  // staged padding rows, or null
+};
+
 template <int MODE>
-__device__ __forceinline__ KeyTiles<MODE> key_tiles(const Unit& w, const Params& p, const uint32_t* bits, int t) {
+__device__ __forceinline__ KeyTiles<MODE> key_tiles(const Unit& w, const Params& p, const Masks& mk, int t) {
     const bool causal = MODE == kModeCausal || (MODE == kModeSparse && p.causal);
     const int qt = w.q0 / kBlockM + t;
     KeyTiles<MODE> k;
@@ -315,10 +318,8 @@ __device__ __forceinline__ KeyTiles<MODE> key_tiles(const Unit& w, const Params&
     k.lim = (MODE == kModeSparse && w.q0 + t * kBlockM >= p.N) ? -1
             : causal ? min(p.n_kv_all - 1, qt) : p.n_kv_all - 1;
     k.off = qt * p.n_kv_all;
-    k.bits = p.block_mask != nullptr ? bits : nullptr;
-    k.pad = p.key_pad != nullptr ? p.key_pad + static_cast<size_t>(w.b) * p.N : nullptr;
-    k.n = p.N;
-    k.pad_vec = p.pad_vec != 0;
+    k.bits = mk.bits;
+    k.pad = mk.pad_rows != nullptr ? mk.pad_rows + mk.pad_map[w.local] * p.pad_row_words : nullptr;
     return k;
 }
 
@@ -337,10 +338,10 @@ struct Plan {
 };
 
 template <int MODE>
-__device__ __forceinline__ Plan<MODE> make_plan(const Unit& w, const Params& p, const uint32_t* bits) {
+__device__ __forceinline__ Plan<MODE> make_plan(const Unit& w, const Params& p, const Masks& mk) {
     Plan<MODE> pl;
-    pl.q[0] = key_tiles<MODE>(w, p, bits, 0);
-    pl.q[1] = key_tiles<MODE>(w, p, bits, 1);
+    pl.q[0] = key_tiles<MODE>(w, p, mk, 0);
+    pl.q[1] = key_tiles<MODE>(w, p, mk, 1);
     return pl;
 }
 
@@ -350,7 +351,7 @@ struct Ctx {
     uint32_t bar;    // barrier block
     uint32_t tmem;   // TMEM base address
     volatile uint32_t* abort_flag;
-    const uint32_t* mask_bits;  // sparse mode: staged block mask bits
+    Masks masks;                // sparse mode: shared-memory copies of the masks
     Params p;
 };
 
@@ -389,7 +390,7 @@ __device__ __forceinline__ void role_producer(const Ctx& c, const CUtensorMap* t
         int local = 0;
         for (int u = blockIdx.x; ok && u < c.p.total_units; u += gridDim.x, ++local) {
             const Unit w = decode_unit<MODE>(u, c.p);
-            const int n1 = make_plan<MODE>(w, c.p, c.mask_bits).q[1].lim + 1;
+            const int n1 = make_plan<MODE>(w, c.p, c.masks).q[1].lim + 1;
             if (!wait_bounded(c.bar + Bars::kQEmpty, (local & 1) ^ 1, c.abort_flag, c.p.wait_ns)) {
                 ok = false;
                 break;
@@ -437,7 +438,7 @@ __device__ __forceinline__ void role_producer(const Ctx& c, const CUtensorMap* t
         };
         for (int u = blockIdx.x; ok && u < c.p.total_units; u += gridDim.x) {
             const Unit w = decode_unit<MODE>(u, c.p);
-            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.masks);
             int j = pl.next(0);
             if (j == kNoTile) continue;
             if (!wait_bounded(c.bar + Bars::kQEmpty, (q_issued & 1) ^ 1, c.abort_flag, c.p.wait_ns)) {
@@ -533,7 +534,7 @@ __device__ __forceinline__ void role_mma_s(const Ctx& c) {
         int local = 0;
         for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
             const Unit w = decode_unit<MODE>(u, c.p);
-            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.masks);
             const int n0 = pl.q[0].lim + 1, n1 = pl.q[1].lim + 1;
             if (!wait(c.bar + Bars::kQFull + 0, local & 1) || !wait(c.bar + Bars::kQFull + 8, local & 1)) break;
             for (int j = 0; j < n1; ++j) {
@@ -562,7 +563,7 @@ __device__ __forceinline__ void role_mma_s(const Ctx& c) {
         uint32_t q_units = 0;
         for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x) {
             const Unit w = decode_unit<MODE>(u, c.p);
-            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.masks);
             int j = pl.next(0);
             if (j == kNoTile) continue;
             if (!wait(c.bar + Bars::kQFull + 0, q_units & 1) || !wait(c.bar + Bars::kQFull + 8, q_units & 1)) break;
@@ -601,7 +602,7 @@ __device__ __forceinline__ void role_mma_pv(const Ctx& c) {
         int local = 0;
         for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
             const Unit w = decode_unit<MODE>(u, c.p);
-            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.masks);
             const int n0 = pl.q[0].lim + 1, n1 = pl.q[1].lim + 1;
             for (int j = 0; j < n1; ++j) {
                 uint32_t vs;
@@ -631,7 +632,7 @@ __device__ __forceinline__ void role_mma_pv(const Ctx& c) {
         uint32_t o_units[2] = {0u, 0u};  // units in which Q tile t accumulated an O
         for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x) {
             const Unit w = decode_unit<MODE>(u, c.p);
-            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.masks);
             const int first[2] = {pl.q[0].next(0), pl.q[1].next(0)};
             const int last[2] = {pl.q[0].last(), pl.q[1].last()};
             for (int j = pl.next(0); j != kNoTile; j = pl.next(j + 1)) {
@@ -676,7 +677,7 @@ __device__ __forceinline__ void role_mma_ordered(const Ctx& c) {
         auto smem = [&](uint32_t slot) { return r.smem + slot * C::kTileBytes; };
         for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x, ++local) {
             const Unit w = decode_unit<MODE>(u, c.p);
-            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.masks);
             const int n0 = pl.q[0].lim + 1, n1 = pl.q[1].lim + 1;
             if (!wait(c.bar + Bars::kQFull + 0, local & 1) || !wait(c.bar + Bars::kQFull + 8, local & 1)) break;
             uint32_t ks;
@@ -734,7 +735,7 @@ __device__ __forceinline__ void role_mma_ordered(const Ctx& c) {
         auto smem = [&](uint32_t slot) { return r.smem + slot * C::kTileBytes; };
         for (int u = blockIdx.x; wait.ok && u < c.p.total_units; u += gridDim.x) {
             const Unit w = decode_unit<MODE>(u, c.p);
-            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.mask_bits);
+            const Plan<MODE> pl = make_plan<MODE>(w, c.p, c.masks);
             int j = pl.next(0);
             if (j == kNoTile) continue;
             const int first[2] = {pl.q[0].next(0), pl.q[1].next(0)};
@@ -828,7 +829,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
         const int row = w.q0 + t * kBlockM + r_in_tile;
         // step j visits key tile j (full, causal) or the j-th key tile kj of
         // this Q tile's mask row (sparse)
-        const KeyTiles<MODE> kt = key_tiles<MODE>(w, p, c.mask_bits, t);
+        const KeyTiles<MODE> kt = key_tiles<MODE>(w, p, c.masks, t);
         // sparse: walk kt.next() until it runs out (no count: with key padding
         // each step tests the mask bytes of the candidate tiles)
         const int n_kv = MODE == kModeSparse ? 0 : kt.count();
@@ -881,36 +882,44 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
                 tc_fence_before();
                 mbar_arrive(b_sfree);
             }
-            // key padding: the 128 mask bytes of this key tile, requested all
-            // at once (one round trip when they can be read 16 at a time); only
-            // 16-key groups that hold a padded key are touched
+            // key padding: the tile's 128 padding bits (staged: from shared
+            // memory; otherwise built from its 128 mask bytes), then padded
+            // keys get -inf -- behind one warp-wide branch, so that tiles
+            // without a padded key (all but the boundary tiles, usually) pay
+            // only for the test
             if (MASK) {
-                const int key0 = key_tile * kBlockN;
-                const uint8_t* mrow = p.key_pad + static_cast<size_t>(w.b) * p.N + key0;
-                auto mask16 = [&](int g, uint4 x) {
-                    if (x.x | x.y | x.z | x.w) {
-                        const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            if ((wv[e >> 2] >> (8 * (e & 3))) & 0xFFu) s[16 * g + e] = -INFINITY;
-                    }
-                };
-                if (p.pad_vec && key0 + kBlockN <= p.N) {
-                    uint4 x[kBlockN / 16];
-#pragma unroll
-                    for (int g = 0; g < kBlockN / 16; ++g) x[g] = ldg_nc16(mrow + 16 * g);
-#pragma unroll
-                    for (int g = 0; g < kBlockN / 16; ++g) mask16(g, x[g]);
+                uint32_t pw[4];
+                if (kt.pad != nullptr) {
+                    const uint4 pb = pad_tile_bits(kt.pad, key_tile);
+                    pw[0] = pb.x, pw[1] = pb.y, pw[2] = pb.z, pw[3] = pb.w;
                 } else {
+                    // not staged (too large for shared memory): 16 bytes at a time
+                    const int key0 = key_tile * kBlockN;
+                    const uint8_t* mrow = p.key_pad + static_cast<size_t>(w.b) * p.N + key0;
+                    const bool vec = p.pad_vec && key0 + kBlockN <= p.N;
 #pragma unroll
                     for (int g = 0; g < kBlockN / 16; ++g) {
-                        uint32_t wd[4] = {0u, 0u, 0u, 0u};
+                        uint4 x;
+                        if (vec) {
+                            x = ldg_nc16(mrow + 16 * g);
+                        } else {
+                            uint32_t wd[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            if (key0 + 16 * g + e < p.N)
-                                wd[e >> 2] |= static_cast<uint32_t>(mrow[16 * g + e] != 0) << (8 * (e & 3));
-                        mask16(g, make_uint4(wd[0], wd[1], wd[2], wd[3]));
+                            for (int e = 0; e < 16; ++e)
+                                if (key0 + 16 * g + e < p.N)
+                                    wd[e >> 2] |= static_cast<uint32_t>(mrow[16 * g + e] != 0) << (8 * (e & 3));
+                            x = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                        }
+                        const uint32_t bits16 = nonzero_bytes4(x.x) | (nonzero_bytes4(x.y) << 4) |
+                                                (nonzero_bytes4(x.z) << 8) | (nonzero_bytes4(x.w) << 12);
+                        if (g & 1) pw[g >> 1] |= bits16 << 16;
+                        else pw[g >> 1] = bits16;
                     }
+                }
+                if (__any_sync(0xffffffffu, (pw[0] | pw[1] | pw[2] | pw[3]) != 0u)) {
+#pragma unroll
+                    for (int cc = 0; cc < kBlockN; ++cc)
+                        if ((pw[cc >> 5] >> (cc & 31)) & 1u) s[cc] = -INFINITY;
                 }
             }
             // key-tail and causal mask: keys past last_key get -inf
@@ -1066,6 +1075,46 @@ __device__ __forceinline__ void stage_block_mask(const Params& p, uint32_t* bits
     }
 }
 
+// Key padding, staged: thread 0 maps each of this CTA's units to a row (one
+// per distinct batch), then every thread fills whole 32-bit words of the rows
+// (bit = key padded; keys past N count as padded).  Rows are read 16 bytes
+// at a time when the mask allows it.
+template <int MODE>
+__device__ __forceinline__ void stage_key_padding(const Params& p, uint16_t* map, int* rowb, uint32_t* rows,
+                                                  int& n_rows) {
+    if (threadIdx.x == 0) {
+        int nr = 0;
+        int k = 0;
+        for (int u = blockIdx.x; u < p.total_units && k < p.pad_units; u += gridDim.x, ++k) {
+            const int b = decode_unit<MODE>(u, p).b;
+            int r = 0;
+            while (r < nr && rowb[r] != b) ++r;
+            if (r == nr) rowb[nr++] = b;
+            map[k] = static_cast<uint16_t>(r);
+        }
+        n_rows = nr;
+    }
+    __syncthreads();
+    const int words = n_rows * p.pad_row_words;
+    for (int i = threadIdx.x; i < words; i += kThreads) {
+        const int r = i / p.pad_row_words;
+        const int key0 = (i - r * p.pad_row_words) * 32;
+        const uint8_t* src = p.key_pad + static_cast<size_t>(rowb[r]) * p.N;
+        uint32_t word;
+        if (p.pad_vec && key0 + 32 <= p.N) {
+            const uint4 a = ldg_nc16(src + key0), b = ldg_nc16(src + key0 + 16);
+            word = nonzero_bytes4(a.x) | (nonzero_bytes4(a.y) << 4) | (nonzero_bytes4(a.z) << 8) |
+                   (nonzero_bytes4(a.w) << 12) | (nonzero_bytes4(b.x) << 16) | (nonzero_bytes4(b.y) << 20) |
+                   (nonzero_bytes4(b.z) << 24) | (nonzero_bytes4(b.w) << 28);
+        } else {
+            word = 0u;
+            for (int e = 0; e < 32; ++e)
+                if (key0 + e >= p.N || src[key0 + e] != 0) word |= 1u << e;
+        }
+        rows[i] = word;
+    }
+}
+
 // ----------------------------------------------------------------- the kernel
 template <int D, int MODE, bool MASK>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1117,10 +1166,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     uint32_t* const mask_bits = reinterpret_cast<uint32_t*>(gbase + C::kMaskOff);
     if (MODE == kModeSparse && p.block_mask != nullptr) stage_block_mask(p, mask_bits);
+    Masks masks{MODE == kModeSparse && p.block_mask != nullptr ? mask_bits : nullptr, nullptr, nullptr};
+    if (MODE == kModeSparse && MASK && p.pad_staged) {
+        uint16_t* map = reinterpret_cast<uint16_t*>(gbase + p.pad_map_off);
+        int* rowb = reinterpret_cast<int*>(gbase + p.pad_rowb_off);
+        uint32_t* rows = reinterpret_cast<uint32_t*>(gbase + p.pad_rows_off);
+        stage_key_padding<MODE>(p, map, rowb, rows, *reinterpret_cast<int*>(gbase + C::kBarOff + Bars::kPadRows));
+        masks.pad_map = map;
+        masks.pad_rows = rows;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const Ctx ctx{base, bar, *tmem_slot, abort_flag, mask_bits, p};
+    const Ctx ctx{base, bar, *tmem_slot, abort_flag, masks, p};
 
     if (warp >= kLoadWarp) {
         regs_decrease<kOtherRegs>();
@@ -1324,19 +1382,43 @@ bool rows_nested(int B, int H, int N, int d, long long sb, long long sh, long lo
     return true;
 }
 
-// Causal unit order: the K and V of the heads in flight should fit in about a
-// third of the 126 MB L2.
-constexpr long long kL2GroupBytes = 40LL << 20;
-
 // Largest block-mask side the shared-memory bit copy takes (N <= 65536).
 constexpr int kMaxMaskTiles = 512;
 
+// Dynamic shared memory of one CTA: the fixed part, the block-mask bits, and
+// (when it fits) the staged key padding, whose offsets are written to p.
+constexpr int kMaxSmemPerBlock = 232448;       // 227 KB opt-in limit per block on sm_100
+constexpr int kMaxPadStageBytes = 48 * 1024;   // cap on the staged key padding
+
+template <int D>
+int smem_layout(Params& p, bool sparse) {
+    const long long bits = p.block_mask != nullptr ? static_cast<long long>(p.n_kv_all) * p.n_kv_all : 0;
+    int smem = Cfg<D>::kSmemBytes + (sparse ? static_cast<int>((bits + 127) / 128) * 16 : 0);
+    p.pad_staged = 0;
+    if (sparse && p.key_pad != nullptr) {
+        auto up16 = [](long long x) { return (x + 15) / 16 * 16; };
+        const long long units = p.pad_units;
+        const long long rows = units < p.BH / p.H ? units : p.BH / p.H;  // distinct batches at most
+        const long long row_bytes = 4LL * p.pad_row_words;
+        const long long need = up16(2 * units) + up16(4 * units) + rows * row_bytes;
+        if (need <= kMaxPadStageBytes && smem + need <= kMaxSmemPerBlock) {
+            // offsets from the 1 KB aligned base: after the block-mask bits
+            const long long base_off = Cfg<D>::kMaskOff + (sparse ? (bits + 127) / 128 * 16 : 0);
+            p.pad_map_off = static_cast<int>(base_off);
+            p.pad_rowb_off = static_cast<int>(base_off + up16(2 * units));
+            p.pad_rows_off = static_cast<int>(base_off + up16(2 * units) + up16(4 * units));
+            p.pad_staged = 1;
+            smem += static_cast<int>(need);
+        }
+    }
+    return smem;
+}
+
 template <int D, int MODE, bool MASK>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
-           const Params& p, int grid, int dev, cudaStream_t stream) {
+           Params p, int grid, int dev, cudaStream_t stream) {
     auto kernel = attn_fwd_kernel<D, MODE, MASK>;
-    const long long bits = p.block_mask != nullptr ? static_cast<long long>(p.n_kv_all) * p.n_kv_all : 0;
-    const int smem = Cfg<D>::kSmemBytes + (MODE == kModeSparse ? static_cast<int>((bits + 127) / 128) * 16 : 0);
+    const int smem = smem_layout<D>(p, MODE == kModeSparse);
     // the dynamic shared-memory limit of this instantiation, raised once per
     // device to the largest size asked for so far
     // device and context (a reset or a new context starts from the default)
@@ -1456,12 +1538,11 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
     p.total_units = static_cast<int>(units);
     p.scale_log2 = scale * kLog2e;
     p.wait_ns = kDefaultWaitNs;
-    {
-        const long long kv_bytes = 4LL * N * d;  // K and V of one head, bf16
-        const long long g = kL2GroupBytes / kv_bytes;
-        p.group_heads = static_cast<int>(g < 1 ? 1 : g > BH ? BH : g);
-    }
+    p.pad_row_words = 4 * p.n_kv_all;
+    p.pad_staged = 0;
+    p.pad_map_off = p.pad_rowb_off = p.pad_rows_off = 0;
     const int grid = static_cast<int>(units < sms ? units : sms);
+    p.pad_units = static_cast<int>((units + grid - 1) / grid);
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool pad = key_padding_mask != nullptr;
