@@ -199,10 +199,9 @@ __device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t x) {
     return ((y >> 7) & 1u) | ((y >> 14) & 2u) | ((y >> 21) & 4u) | ((y >> 28) & 8u);
 }
 
-// The 128 padding bits of key tile j in a staged row (bit set = padded).
-__device__ __forceinline__ uint4 pad_tile_bits(const uint32_t* row, int j) {
-    return *reinterpret_cast<const uint4*>(row + 4 * j);
-}
+// The 128 padding bits of key tile j in a staged row (bit set = padded);
+// row: shared-window address of the row.
+__device__ __forceinline__ uint4 pad_tile_bits(uint32_t row, int j) { return lds_u32x4(row + 16 * j); }
 
 // The key tiles one Q tile visits, in increasing order.  In the sparse mode
 // (a block mask, a key-padding mask, or both) a tile is visited when its
@@ -214,14 +213,14 @@ template <int MODE>
 struct KeyTiles {
     int lim;               // last key tile it may visit (-1: the tile has no rows)
     int off;               // sparse: bit index of its mask row, column 0
-    const uint32_t* bits;  // sparse: the block mask as bits, row-major, in shared memory (null: none)
-    const uint32_t* pad;   // sparse: the staged padding bits of this unit's batch (null: none)
+    uint32_t bits;         // sparse: shared-window address of the block mask bits, row-major (0: none)
+    uint32_t pad;          // sparse: shared-window address of this unit's staged padding row (0: none)
 
     __device__ __forceinline__ bool bit(int j) const {
-        return bits == nullptr || ((bits[(off + j) >> 5] >> ((off + j) & 31)) & 1u);
+        return bits == 0u || ((lds_u32(bits + 4 * ((off + j) >> 5)) >> ((off + j) & 31)) & 1u);
     }
     __device__ __forceinline__ bool keyed(int j) const {
-        if (pad == nullptr) return true;
+        if (pad == 0u) return true;
         const uint4 b = pad_tile_bits(pad, j);
         return (b.x & b.y & b.z & b.w) != ~0u;  // some key of the tile is not padded
     }
@@ -231,10 +230,10 @@ struct KeyTiles {
     }
     // first tile >= j whose block-mask bit is set (kNoTile if none)
     __device__ __forceinline__ int next_bit(int j) const {
-        if (bits == nullptr) return j <= lim ? j : kNoTile;
+        if (bits == 0u) return j <= lim ? j : kNoTile;
         while (j <= lim) {
             const int f = off + j;
-            const uint32_t word = bits[f >> 5] >> (f & 31);
+            const uint32_t word = lds_u32(bits + 4 * (f >> 5)) >> (f & 31);
             if (word != 0u) {
                 const int jj = j + __ffs(static_cast<int>(word)) - 1;
                 return jj <= lim ? jj : kNoTile;
@@ -245,10 +244,10 @@ struct KeyTiles {
     }
     // last tile <= j whose block-mask bit is set (-1 if none)
     __device__ __forceinline__ int prev_bit(int j) const {
-        if (bits == nullptr) return j;
+        if (bits == 0u) return j;
         while (j >= 0) {
             const int f = off + j;
-            const uint32_t word = bits[f >> 5] << (31 - (f & 31));
+            const uint32_t word = lds_u32(bits + 4 * (f >> 5)) << (31 - (f & 31));
             if (word != 0u) {
                 const int jj = j - __clz(static_cast<int>(word));
                 return jj >= 0 ? jj : -1;
@@ -273,7 +272,7 @@ struct KeyTiles {
             return lim + 1;
         } else {
             if (lim < 0) return 0;
-            if (pad != nullptr || bits == nullptr) {
+            if (pad != 0u || bits == 0u) {
                 int n_tiles = 0;
                 for (int j = next(0); j != kNoTile; j = next(j + 1)) ++n_tiles;
                 return n_tiles;
@@ -281,7 +280,7 @@ struct KeyTiles {
             const int f = off, e = off + lim;  // first and last bit, inclusive
             int n_tiles = 0;
             for (int wd = f >> 5; wd <= (e >> 5); ++wd) {
-                uint32_t x = bits[wd];
+                uint32_t x = lds_u32(bits + 4 * wd);
                 if (wd == (f >> 5)) x &= ~0u << (f & 31);
                 if (wd == (e >> 5)) x &= ~0u >> (31 - (e & 31));
                 n_tiles += __popc(x);
@@ -303,9 +302,9 @@ struct KeyTiles {
 
 // Per-CTA shared-memory copies of the masks (sparse mode).
 struct Masks {
-    const uint32_t* bits;      // block mask bits, or null
-    const uint16_t* pad_map;   // local unit index -> staged padding row, or null
-    const uint32_t* pad_rows;  // staged padding rows, or null
+    uint32_t bits;             // shared-window address of the block mask bits (0: none)
+    uint32_t pad_map;          // shared-window address of the map local unit -> staged row (u32 each)
+    uint32_t pad_rows;         // shared-window address of the staged padding rows (0: none)
 };
 
 template <int MODE>
@@ -319,7 +318,9 @@ __device__ __forceinline__ KeyTiles<MODE> key_tiles(const Unit& w, const Params&
             : causal ? min(p.n_kv_all - 1, qt) : p.n_kv_all - 1;
     k.off = qt * p.n_kv_all;
     k.bits = mk.bits;
-    k.pad = mk.pad_rows != nullptr ? mk.pad_rows + mk.pad_map[w.local] * p.pad_row_words : nullptr;
+    k.pad = mk.pad_rows != 0u
+                ? mk.pad_rows + 4u * lds_u32(mk.pad_map + 4u * w.local) * static_cast<uint32_t>(p.pad_row_words)
+                : 0u;
     return k;
 }
 
@@ -889,7 +890,7 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
             // only for the test
             if (MASK) {
                 uint32_t pw[4];
-                if (kt.pad != nullptr) {
+                if (kt.pad != 0u) {
                     const uint4 pb = pad_tile_bits(kt.pad, key_tile);
                     pw[0] = pb.x, pw[1] = pb.y, pw[2] = pb.z, pw[3] = pb.w;
                 } else {
@@ -1080,7 +1081,7 @@ __device__ __forceinline__ void stage_block_mask(const Params& p, uint32_t* bits
 // (bit = key padded; keys past N count as padded).  Rows are read 16 bytes
 // at a time when the mask allows it.
 template <int MODE>
-__device__ __forceinline__ void stage_key_padding(const Params& p, uint16_t* map, int* rowb, uint32_t* rows,
+__device__ __forceinline__ void stage_key_padding(const Params& p, uint32_t* map, int* rowb, uint32_t* rows,
                                                   int& n_rows) {
     if (threadIdx.x == 0) {
         int nr = 0;
@@ -1090,7 +1091,7 @@ __device__ __forceinline__ void stage_key_padding(const Params& p, uint16_t* map
             int r = 0;
             while (r < nr && rowb[r] != b) ++r;
             if (r == nr) rowb[nr++] = b;
-            map[k] = static_cast<uint16_t>(r);
+            map[k] = static_cast<uint32_t>(r);
         }
         n_rows = nr;
     }
@@ -1166,14 +1167,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     uint32_t* const mask_bits = reinterpret_cast<uint32_t*>(gbase + C::kMaskOff);
     if (MODE == kModeSparse && p.block_mask != nullptr) stage_block_mask(p, mask_bits);
-    Masks masks{MODE == kModeSparse && p.block_mask != nullptr ? mask_bits : nullptr, nullptr, nullptr};
+    Masks masks{MODE == kModeSparse && p.block_mask != nullptr ? smem_addr(mask_bits) : 0u, 0u, 0u};
     if (MODE == kModeSparse && MASK && p.pad_staged) {
-        uint16_t* map = reinterpret_cast<uint16_t*>(gbase + p.pad_map_off);
+        uint32_t* map = reinterpret_cast<uint32_t*>(gbase + p.pad_map_off);
         int* rowb = reinterpret_cast<int*>(gbase + p.pad_rowb_off);
         uint32_t* rows = reinterpret_cast<uint32_t*>(gbase + p.pad_rows_off);
         stage_key_padding<MODE>(p, map, rowb, rows, *reinterpret_cast<int*>(gbase + C::kBarOff + Bars::kPadRows));
-        masks.pad_map = map;
-        masks.pad_rows = rows;
+        masks.pad_map = smem_addr(map);
+        masks.pad_rows = smem_addr(rows);
     }
     tc_fence_before();
     __syncthreads();
@@ -1400,13 +1401,13 @@ int smem_layout(Params& p, bool sparse) {
         const long long units = p.pad_units;
         const long long rows = units < p.BH / p.H ? units : p.BH / p.H;  // distinct batches at most
         const long long row_bytes = 4LL * p.pad_row_words;
-        const long long need = up16(2 * units) + up16(4 * units) + rows * row_bytes;
+        const long long need = up16(4 * units) + up16(4 * units) + rows * row_bytes;
         if (need <= kMaxPadStageBytes && smem + need <= kMaxSmemPerBlock) {
             // offsets from the 1 KB aligned base: after the block-mask bits
             const long long base_off = Cfg<D>::kMaskOff + (sparse ? (bits + 127) / 128 * 16 : 0);
             p.pad_map_off = static_cast<int>(base_off);
-            p.pad_rowb_off = static_cast<int>(base_off + up16(2 * units));
-            p.pad_rows_off = static_cast<int>(base_off + up16(2 * units) + up16(4 * units));
+            p.pad_rowb_off = static_cast<int>(base_off + up16(4 * units));
+            p.pad_rows_off = static_cast<int>(base_off + up16(4 * units) + up16(4 * units));
             p.pad_staged = 1;
             smem += static_cast<int>(need);
         }
