@@ -307,6 +307,24 @@ def run_cuda(args, rank, world, dist):
                 "algorithmic_bytes": algorithmic_bytes(B, H, N, d),
                 "frac_of_datasheet_2250": round(achieved / DATASHEET_BF16_TFLOPS, 4)}
 
+    # host time of one call of the 12-argument C entry point (argument checks,
+    # tensor-map lookup, launch; the kernel runs asynchronously): median over
+    # calls issued back to back, next to the kernel's own time
+    host_us = None
+    if not args.no_host_time:
+        sh = torch.cuda.current_stream().cuda_stream
+        ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr())
+        n_calls = 200 if ms_local < 0.5 else 50
+        times = []
+        for _ in range(n_calls):
+            t0 = time.perf_counter()
+            st = pkg.attn_fwd(*ptrs, B, H, N, d, scale, causal, sh)
+            times.append(time.perf_counter() - t0)
+            if st != pkg.ATTN_OK:
+                raise RuntimeError("attn_fwd: " + pkg.attn_status_string(st))
+        torch.cuda.synchronize()
+        host_us = round(statistics.median(times) * 1e6, 2)
+
     # end to end through the public call: pinned host inputs -> device -> attention -> host outputs
     e2e = None
     if not args.no_e2e:
@@ -369,6 +387,7 @@ def run_cuda(args, rank, world, dist):
                              "device_free_delta": int(free0 - free1),
                              "method": "memory_allocated base, reset_peak_memory_stats, call, max_memory_allocated - base"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+        "host_us_per_call": host_us,
         "clocks": clocks.summary(), "step_ms_min": round(min(step_ms), 4), "step_ms_max": round(max(step_ms), 4),
     }
     return line
@@ -570,6 +589,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-host-time", action="store_true",
+                    help="skip timing the host side of one attn_fwd call")
     ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
                     help="time the forward (the headline) or the backward")
     ap.add_argument("--sweep", action="store_true", help="TFLOP/s and peak extra bytes over the image sweep")

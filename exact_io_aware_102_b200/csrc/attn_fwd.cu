@@ -199,8 +199,26 @@ __device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t x) {
     return ((y >> 7) & 1u) | ((y >> 14) & 2u) | ((y >> 21) & 4u) | ((y >> 28) & 8u);
 }
 
-// The 128 padding bits of key tile j in a staged row (bit set = padded);
-// row: shared-window address of the row.
+// A staged key-padding row (shared memory, one per batch that the CTA's units
+// touch): 4 words per key tile with one bit per key (set = padded, keys >= N
+// included), then two bitmaps with one bit per key tile: "holds an unpadded
+// key" (the tile is visited) and "holds a padded key" (the tile needs the
+// per-key mask).
+struct PadRow {
+    static __device__ __forceinline__ uint32_t occ(uint32_t row, int n_tiles) { return row + 16u * n_tiles; }
+    static __device__ __forceinline__ uint32_t mix(uint32_t row, int n_tiles) {
+        return row + 16u * n_tiles + 4u * ((n_tiles + 31) / 32);
+    }
+    // last key tile that holds an unpadded key (-1: none), one int
+    static __device__ __forceinline__ uint32_t last(uint32_t row, int n_tiles) {
+        return row + 16u * n_tiles + 8u * ((n_tiles + 31) / 32);
+    }
+    static __host__ __device__ constexpr int words(int n_tiles) {
+        return (4 * n_tiles + 2 * ((n_tiles + 31) / 32) + 1 + 3) / 4 * 4;  // 16-byte multiple
+    }
+};
+
+// The 128 padding bits of key tile j in a staged row; row: shared-window address.
 __device__ __forceinline__ uint4 pad_tile_bits(uint32_t row, int j) { return lds_u32x4(row + 16 * j); }
 
 // The key tiles one Q tile visits, in increasing order.  In the sparse mode
@@ -209,61 +227,60 @@ __device__ __forceinline__ uint4 pad_tile_bits(uint32_t row, int j) { return lds
 // and, with key padding, it holds a key that is not padded: tiles made only
 // of padded keys are neither loaded nor multiplied.  Every role evaluates the
 // same predicate for the same unit, so they all walk the same tiles.
+//
+// The predicate of 32 consecutive tiles is read from shared memory into one
+// word (block-mask bits, "holds an unpadded key" bits and the causal bound
+// combined) and kept: tiles are walked in order, so the common step costs no
+// shared-memory load (those queue behind the tensor core's operand reads and
+// take hundreds of cycles).
 template <int MODE>
 struct KeyTiles {
     int lim;               // last key tile it may visit (-1: the tile has no rows)
-    int off;               // sparse: bit index of its mask row, column 0
+    int off;               // sparse: bit index of its block-mask row, column 0
     uint32_t bits;         // sparse: shared-window address of the block mask bits, row-major (0: none)
     uint32_t pad;          // sparse: shared-window address of this unit's staged padding row (0: none)
+    int n_tiles;           // sparse: key tiles per row (block-mask rows and padding bitmaps)
+    mutable int wi;        // sparse: window index held in ww (tiles 32 wi .. 32 wi + 31), -1: none
+    mutable uint32_t ww;   // sparse: visited tiles of that window
 
-    __device__ __forceinline__ bool bit(int j) const {
-        return bits == 0u || ((lds_u32(bits + 4 * ((off + j) >> 5)) >> ((off + j) & 31)) & 1u);
+    __device__ __forceinline__ uint32_t load_window(int i) const {
+        const int j0 = 32 * i;
+        if (j0 > lim) return 0u;
+        uint32_t v = ~0u;
+        if (bits != 0u) {
+            const int f = off + j0;  // first bit; the row ends at off + n_tiles - 1
+            const int total_words = (n_tiles * n_tiles + 31) / 32;
+            const uint32_t lo = lds_u32(bits + 4u * (f >> 5));
+            const uint32_t hi = ((f & 31) != 0 && (f >> 5) + 1 < total_words) ? lds_u32(bits + 4u * ((f >> 5) + 1)) : 0u;
+            v = __funnelshift_r(lo, hi, f & 31);
+        }
+        if (pad != 0u) v &= lds_u32(PadRow::occ(pad, n_tiles) + 4u * i);
+        const int last = lim - j0;  // >= 0 here
+        if (last < 31) v &= ~0u >> (31 - last);
+        return v;
     }
-    __device__ __forceinline__ bool keyed(int j) const {
-        if (pad == 0u) return true;
-        const uint4 b = pad_tile_bits(pad, j);
-        return (b.x & b.y & b.z & b.w) != ~0u;  // some key of the tile is not padded
+    __device__ __forceinline__ uint32_t window(int i) const {
+        if (i != wi) {
+            ww = load_window(i);
+            wi = i;
+        }
+        return ww;
     }
     __device__ __forceinline__ bool has(int j) const {
         if constexpr (MODE != kModeSparse) return j <= lim;
-        else return j >= 0 && j <= lim && bit(j) && keyed(j);
-    }
-    // first tile >= j whose block-mask bit is set (kNoTile if none)
-    __device__ __forceinline__ int next_bit(int j) const {
-        if (bits == 0u) return j <= lim ? j : kNoTile;
-        while (j <= lim) {
-            const int f = off + j;
-            const uint32_t word = lds_u32(bits + 4 * (f >> 5)) >> (f & 31);
-            if (word != 0u) {
-                const int jj = j + __ffs(static_cast<int>(word)) - 1;
-                return jj <= lim ? jj : kNoTile;
-            }
-            j += 32 - (f & 31);
-        }
-        return kNoTile;
-    }
-    // last tile <= j whose block-mask bit is set (-1 if none)
-    __device__ __forceinline__ int prev_bit(int j) const {
-        if (bits == 0u) return j;
-        while (j >= 0) {
-            const int f = off + j;
-            const uint32_t word = lds_u32(bits + 4 * (f >> 5)) << (31 - (f & 31));
-            if (word != 0u) {
-                const int jj = j - __clz(static_cast<int>(word));
-                return jj >= 0 ? jj : -1;
-            }
-            j -= (f & 31) + 1;
-        }
-        return -1;
+        else return j >= 0 && j <= lim && ((window(j >> 5) >> (j & 31)) & 1u);
     }
     // first key tile >= j (kNoTile if none)
     __device__ __forceinline__ int next(int j) const {
         if constexpr (MODE != kModeSparse) {
             return j <= lim ? j : kNoTile;
         } else {
-            for (j = next_bit(j); j != kNoTile && !keyed(j); j = next_bit(j + 1)) {
+            while (j <= lim) {
+                const uint32_t w = window(j >> 5) >> (j & 31);
+                if (w != 0u) return j + __ffs(static_cast<int>(w)) - 1;
+                j = (j | 31) + 1;
             }
-            return j;
+            return kNoTile;
         }
     }
     // number of key tiles
@@ -271,21 +288,9 @@ struct KeyTiles {
         if constexpr (MODE != kModeSparse) {
             return lim + 1;
         } else {
-            if (lim < 0) return 0;
-            if (pad != 0u || bits == 0u) {
-                int n_tiles = 0;
-                for (int j = next(0); j != kNoTile; j = next(j + 1)) ++n_tiles;
-                return n_tiles;
-            }
-            const int f = off, e = off + lim;  // first and last bit, inclusive
-            int n_tiles = 0;
-            for (int wd = f >> 5; wd <= (e >> 5); ++wd) {
-                uint32_t x = lds_u32(bits + 4 * wd);
-                if (wd == (f >> 5)) x &= ~0u << (f & 31);
-                if (wd == (e >> 5)) x &= ~0u >> (31 - (e & 31));
-                n_tiles += __popc(x);
-            }
-            return n_tiles;
+            int n = 0;
+            for (int i = 0; 32 * i <= lim; ++i) n += __popc(window(i));
+            return n;
         }
     }
     // last key tile (-1 if none)
@@ -293,9 +298,11 @@ struct KeyTiles {
         if constexpr (MODE != kModeSparse) {
             return lim;
         } else {
-            int j = prev_bit(lim);
-            while (j >= 0 && !keyed(j)) j = prev_bit(j - 1);
-            return j;
+            for (int i = lim >> 5; i >= 0 && lim >= 0; --i) {
+                const uint32_t w = window(i);
+                if (w != 0u) return 32 * i + 31 - __clz(static_cast<int>(w));
+            }
+            return -1;
         }
     }
 };
@@ -307,8 +314,16 @@ struct Masks {
     uint32_t pad_rows;         // shared-window address of the staged padding rows (0: none)
 };
 
+// Shared-window address of the staged padding row of a unit (0: none).
+__device__ __forceinline__ uint32_t pad_row_of(const Unit& w, const Params& p, const Masks& mk) {
+    return mk.pad_rows != 0u
+               ? mk.pad_rows + 4u * lds_u32(mk.pad_map + 4u * w.local) * static_cast<uint32_t>(p.pad_row_words)
+               : 0u;
+}
+
 template <int MODE>
-__device__ __forceinline__ KeyTiles<MODE> key_tiles(const Unit& w, const Params& p, const Masks& mk, int t) {
+__device__ __forceinline__ KeyTiles<MODE> key_tiles_row(const Unit& w, const Params& p, const Masks& mk, int t,
+                                                        uint32_t pad_row, int wi = -1, uint32_t ww = 0u) {
     const bool causal = MODE == kModeCausal || (MODE == kModeSparse && p.causal);
     const int qt = w.q0 / kBlockM + t;
     KeyTiles<MODE> k;
@@ -316,12 +331,25 @@ __device__ __forceinline__ KeyTiles<MODE> key_tiles(const Unit& w, const Params&
     // rows (nothing of it is stored); the sparse mode skips it
     k.lim = (MODE == kModeSparse && w.q0 + t * kBlockM >= p.N) ? -1
             : causal ? min(p.n_kv_all - 1, qt) : p.n_kv_all - 1;
+    if (MODE != kModeSparse && pad_row != 0u) {
+        // key padding in the dense loops: the tiles after the batch's last
+        // tile holding an unpadded key are never visited (a batch without any
+        // visits tile 0, fully masked, so that every Q tile has a tile)
+        const int last = static_cast<int>(lds_u32(PadRow::last(pad_row, p.n_kv_all)));
+        k.lim = min(k.lim, max(last, 0));
+    }
     k.off = qt * p.n_kv_all;
     k.bits = mk.bits;
-    k.pad = mk.pad_rows != 0u
-                ? mk.pad_rows + 4u * lds_u32(mk.pad_map + 4u * w.local) * static_cast<uint32_t>(p.pad_row_words)
-                : 0u;
+    k.pad = pad_row;
+    k.n_tiles = p.n_kv_all;
+    k.wi = wi;
+    k.ww = ww;
     return k;
+}
+
+template <int MODE>
+__device__ __forceinline__ KeyTiles<MODE> key_tiles(const Unit& w, const Params& p, const Masks& mk, int t) {
+    return key_tiles_row<MODE>(w, p, mk, t, pad_row_of(w, p, mk));
 }
 
 // The key tiles of one unit, as the load and MMA roles walk them: the union
@@ -830,11 +858,24 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
         const int row = w.q0 + t * kBlockM + r_in_tile;
         // step j visits key tile j (full, causal) or the j-th key tile kj of
         // this Q tile's mask row (sparse)
-        const KeyTiles<MODE> kt = key_tiles<MODE>(w, p, c.masks, t);
-        // sparse: walk kt.next() until it runs out (no count: with key padding
-        // each step tests the mask bytes of the candidate tiles)
-        const int n_kv = MODE == kModeSparse ? 0 : kt.count();
-        int kj = kt.next(0);
+        // sparse: walk next() until it runs out.  Across a step only the
+        // padding row and the current 32-tile window (which tiles are
+        // visited, which hold a padded key) stay live; the rest of the tile
+        // walker is rebuilt when needed (the softmax thread is at its
+        // register limit during the exponentials).
+        const uint32_t pad_row = (MODE == kModeSparse || MASK) ? pad_row_of(w, p, c.masks) : 0u;
+        int wi = -1;          // window index (tiles 32 wi .. 32 wi + 31)
+        uint32_t ww = 0u;     // its visited tiles
+        int mix_i = -1;       // staged padding: index of the "holds a padded key" word in mix_w
+        uint32_t mix_w = 0u;
+        const int n_kv = MODE == kModeSparse ? 0 : key_tiles<MODE>(w, p, c.masks, t).count();
+        int kj;
+        {
+            const KeyTiles<MODE> kt = key_tiles_row<MODE>(w, p, c.masks, t, pad_row);
+            kj = kt.next(0);
+            wi = kt.wi;
+            ww = kt.ww;
+        }
         if constexpr (MODE == kModeSparse) {
             if (kj == kNoTile) {
                 // no key block at all: O = 0 and LSE = -inf, as for a row
@@ -856,6 +897,18 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
 
         for (int j = 0; MODE == kModeSparse ? kj != kNoTile : j < n_kv; ++j) {
             const int key_tile = MODE == kModeSparse ? kj : j;
+            if constexpr (MODE == kModeSparse) {
+                // the next step's tile; the window moves (one shared load) every 32 tiles
+                const KeyTiles<MODE> kt = key_tiles_row<MODE>(w, p, c.masks, t, pad_row, wi, ww);
+                kj = kt.next(kj + 1);
+                wi = kt.wi;
+                ww = kt.ww;
+            }
+            if (MASK && pad_row != 0u && (key_tile >> 5) != mix_i) {
+                // which tiles of this 32-tile window hold a padded key (one shared load)
+                mix_i = key_tile >> 5;
+                mix_w = lds_u32(PadRow::mix(pad_row, p.n_kv_all) + 4u * mix_i);
+            }
             bool got = wait_bounded(b_s, s_phase, c.abort_flag, p.wait_ns);
             got = __all_sync(0xffffffffu, got);
             if (!got) {
@@ -883,16 +936,17 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
                 tc_fence_before();
                 mbar_arrive(b_sfree);
             }
-            // key padding: the tile's 128 padding bits (staged: from shared
-            // memory; otherwise built from its 128 mask bytes), then padded
-            // keys get -inf -- behind one warp-wide branch, so that tiles
-            // without a padded key (all but the boundary tiles, usually) pay
-            // only for the test
+            // key padding: padded keys get -inf.  Staged: the tile's "holds a
+            // padded key" bit (one shared load per 32 tiles) says whether its
+            // 128 per-key bits are needed at all; otherwise the 128 mask bytes
+            // are read.  The masking sits behind one warp-wide branch.
             if (MASK) {
-                uint32_t pw[4];
-                if (kt.pad != 0u) {
-                    const uint4 pb = pad_tile_bits(kt.pad, key_tile);
-                    pw[0] = pb.x, pw[1] = pb.y, pw[2] = pb.z, pw[3] = pb.w;
+                uint32_t pw[4] = {0u, 0u, 0u, 0u};
+                if (pad_row != 0u) {
+                    if ((mix_w >> (key_tile & 31)) & 1u) {
+                        const uint4 pb = pad_tile_bits(pad_row, key_tile);
+                        pw[0] = pb.x, pw[1] = pb.y, pw[2] = pb.z, pw[3] = pb.w;
+                    }
                 } else {
                     // not staged (too large for shared memory): 16 bytes at a time
                     const int key0 = key_tile * kBlockN;
@@ -1010,7 +1064,6 @@ __device__ __forceinline__ void role_softmax(const Ctx& c, int warp, int lane, u
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(b_p);
-            if constexpr (MODE == kModeSparse) kj = kt.next(kj + 1);
         }
         if (!ok) break;
 
@@ -1096,10 +1149,10 @@ __device__ __forceinline__ void stage_key_padding(const Params& p, uint32_t* map
         n_rows = nr;
     }
     __syncthreads();
-    const int words = n_rows * p.pad_row_words;
-    for (int i = threadIdx.x; i < words; i += kThreads) {
-        const int r = i / p.pad_row_words;
-        const int key0 = (i - r * p.pad_row_words) * 32;
+    const int key_words = 4 * p.n_kv_all;  // per row
+    for (int i = threadIdx.x; i < n_rows * key_words; i += kThreads) {
+        const int r = i / key_words;
+        const int key0 = (i - r * key_words) * 32;
         const uint8_t* src = p.key_pad + static_cast<size_t>(rowb[r]) * p.N;
         uint32_t word;
         if (p.pad_vec && key0 + 32 <= p.N) {
@@ -1112,7 +1165,33 @@ __device__ __forceinline__ void stage_key_padding(const Params& p, uint32_t* map
             for (int e = 0; e < 32; ++e)
                 if (key0 + e >= p.N || src[key0 + e] != 0) word |= 1u << e;
         }
-        rows[i] = word;
+        rows[static_cast<size_t>(r) * p.pad_row_words + (i - r * key_words)] = word;
+    }
+    __syncthreads();
+    // the two tile bitmaps of every row: bit t of word i is tile 32 i + t
+    const int n_tiles = p.n_kv_all;
+    const int bm_words = (n_tiles + 31) / 32;
+    for (int i = threadIdx.x; i < 2 * n_rows * bm_words; i += kThreads) {
+        const int kind = i / (n_rows * bm_words);  // 0: holds an unpadded key, 1: holds a padded key
+        const int rem = i - kind * n_rows * bm_words;
+        const int r = rem / bm_words, wd = rem - r * bm_words;
+        const uint32_t* row = rows + static_cast<size_t>(r) * p.pad_row_words;
+        uint32_t word = 0u;
+        for (int t = 0; t < 32 && 32 * wd + t < n_tiles; ++t) {
+            const uint4 b = *reinterpret_cast<const uint4*>(row + 4 * (32 * wd + t));
+            const bool flag = kind == 0 ? (b.x & b.y & b.z & b.w) != ~0u : (b.x | b.y | b.z | b.w) != 0u;
+            word |= static_cast<uint32_t>(flag) << t;
+        }
+        rows[static_cast<size_t>(r) * p.pad_row_words + 4 * n_tiles + kind * bm_words + wd] = word;
+    }
+    __syncthreads();
+    // the last tile holding an unpadded key, from the first bitmap
+    for (int r = threadIdx.x; r < n_rows; r += kThreads) {
+        const uint32_t* occ = rows + static_cast<size_t>(r) * p.pad_row_words + 4 * n_tiles;
+        int last = -1;
+        for (int wd = bm_words - 1; wd >= 0 && last < 0; --wd)
+            if (occ[wd] != 0u) last = 32 * wd + 31 - __clz(static_cast<int>(occ[wd]));
+        rows[static_cast<size_t>(r) * p.pad_row_words + 4 * n_tiles + 2 * bm_words] = static_cast<uint32_t>(last);
     }
 }
 
@@ -1168,7 +1247,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint32_t* const mask_bits = reinterpret_cast<uint32_t*>(gbase + C::kMaskOff);
     if (MODE == kModeSparse && p.block_mask != nullptr) stage_block_mask(p, mask_bits);
     Masks masks{MODE == kModeSparse && p.block_mask != nullptr ? smem_addr(mask_bits) : 0u, 0u, 0u};
-    if (MODE == kModeSparse && MASK && p.pad_staged) {
+    if (MASK && p.pad_staged) {
         uint32_t* map = reinterpret_cast<uint32_t*>(gbase + p.pad_map_off);
         int* rowb = reinterpret_cast<int*>(gbase + p.pad_rowb_off);
         uint32_t* rows = reinterpret_cast<uint32_t*>(gbase + p.pad_rows_off);
@@ -1396,7 +1475,7 @@ int smem_layout(Params& p, bool sparse) {
     const long long bits = p.block_mask != nullptr ? static_cast<long long>(p.n_kv_all) * p.n_kv_all : 0;
     int smem = Cfg<D>::kSmemBytes + (sparse ? static_cast<int>((bits + 127) / 128) * 16 : 0);
     p.pad_staged = 0;
-    if (sparse && p.key_pad != nullptr) {
+    if (p.key_pad != nullptr) {
         auto up16 = [](long long x) { return (x + 15) / 16 * 16; };
         const long long units = p.pad_units;
         const long long rows = units < p.BH / p.H ? units : p.BH / p.H;  // distinct batches at most
@@ -1539,7 +1618,7 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
     p.total_units = static_cast<int>(units);
     p.scale_log2 = scale * kLog2e;
     p.wait_ns = kDefaultWaitNs;
-    p.pad_row_words = 4 * p.n_kv_all;
+    p.pad_row_words = PadRow::words(p.n_kv_all);
     p.pad_staged = 0;
     p.pad_map_off = p.pad_rowb_off = p.pad_rows_off = 0;
     const int grid = static_cast<int>(units < sms ? units : sms);
@@ -1547,16 +1626,18 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool pad = key_padding_mask != nullptr;
-    // a block mask or key padding selects the tile-list loops (only visited
-    // tiles are loaded and multiplied); key padding also masks per key
-    const int mode = (block_mask || pad) ? kModeSparse : causal ? kModeCausal : kModeFull;
+    // a block mask selects the tile-list loops (only visited tiles are loaded
+    // and multiplied); key padding masks per key and, once staged, ends each
+    // Q tile's walk at its batch's last tile holding an unpadded key (with a
+    // block mask: skips every tile made only of padded keys)
+    const int mode = block_mask ? kModeSparse : causal ? kModeCausal : kModeFull;
 #define ATTN_LAUNCH(D_, M_, P_) launch<D_, M_, P_>(mq, mk, mv, o, lse, p, grid, dev, s)
-#define ATTN_BY_MODE(D_)                                                                   \
-    (pad                   ? ATTN_LAUNCH(D_, kModeSparse, true)                            \
-     : mode == kModeSparse ? ATTN_LAUNCH(D_, kModeSparse, false)                           \
-     : mode == kModeCausal ? ATTN_LAUNCH(D_, kModeCausal, false)                           \
-                           : ATTN_LAUNCH(D_, kModeFull, false))
-    return d == 64 ? ATTN_BY_MODE(64) : ATTN_BY_MODE(128);
+#define ATTN_BY_MODE(D_, P_)                                      \
+    (mode == kModeSparse   ? ATTN_LAUNCH(D_, kModeSparse, P_)     \
+     : mode == kModeCausal ? ATTN_LAUNCH(D_, kModeCausal, P_)     \
+                           : ATTN_LAUNCH(D_, kModeFull, P_))
+    if (d == 64) return pad ? ATTN_BY_MODE(64, true) : ATTN_BY_MODE(64, false);
+    return pad ? ATTN_BY_MODE(128, true) : ATTN_BY_MODE(128, false);
 #undef ATTN_BY_MODE
 #undef ATTN_LAUNCH
 }
