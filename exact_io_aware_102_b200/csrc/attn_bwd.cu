@@ -17,10 +17,18 @@
 //   * the main kernel runs a persistent grid, one CTA per SM; a work unit is
 //     one (batch, head, 128-key block).  dK and dV of the block accumulate in
 //     TMEM over the query tiles (128 rows each) the block interacts with;
-//   * warp 12 (one lane) loads K, V once per unit and Q_i, dO_i per query tile
-//     (two stages) by TMA; warp 13 (one lane) issues the tcgen05.mma:
-//     S^T = K Q_i^T and dP^T = V dO_i^T into TMEM, then dV += P^T dO_i,
-//     dK += dS^T Q_i and the dQ partial dS K_j;
+//   * warp 12 loads K, V once per unit and Q_i, dO_i per query tile (three
+//     stages at d = 64, two at d = 128) by TMA, and writes each tile's
+//     offset rows (below); warp 13
+//     (one lane) issues the tcgen05.mma: S^T = K Q_i^T and dP^T = V dO_i^T
+//     into TMEM, then dV += P^T dO_i, dK += dS^T Q_i and the dQ partial
+//     dS K_j;
+//   * the row terms of P = 2^(log2(e) (scale S - LSE)) and of dP - delta
+//     ride on the tensor core: S^T and dP^T take one more K = 16 slice, the
+//     product of a block of ones (keys) with a block holding -LSE/scale
+//     (resp. -delta) of each query row, split into three bf16 parts
+//     (c = h1 + h2 + h3 to 2^-24 |c|), so the accumulators hold S - LSE/scale
+//     and dP - delta and the elementwise warps need no per-column values;
 //   * warps 0-7 (two threads per key row: warps 0-3 query columns 0-63, warps
 //     4-7 columns 64-127, so each SM sub-partition runs two of them) turn the
 //     S^T, dP^T rows into P^T (bf16, into TMEM: the A operand of dV) and dS^T
@@ -32,17 +40,17 @@
 //   * warps 8-11 (one thread per query row) read the dQ partial from TMEM and
 //     add it to the fp32 dQ accumulator in global memory with tensor
 //     reductions (cp.reduce.async.bulk.tensor .add), two [32 x 32] boxes per
-//     warp;
+//     warp through one staging box;
 //   * at the end of a unit warps 0-3 write dV and warps 4-7 dK (times scale)
 //     in bf16.
 //   Every wait is bounded (see sm100_ptx.cuh) and no barrier spans warps
 //   other than mbarriers, so a timeout never leaves a thread blocked.
 //
 // TMEM columns: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
-// dQ [384,448), P^T [448,512) (bf16 pairs).  Shared memory: K, V (16 KB
-// each), two stages of Q and dO (16 KB each), two dS^T buffers (32 KB each,
-// two 64-column halves), dQ staging rows, per-warp LSE / delta rows,
-// barriers.
+// dQ [384,448), P^T [448,512) (bf16 pairs).  Shared memory (226,560 bytes
+// with alignment): K, V (16 KB each), three stages of Q and dO (16 KB each),
+// two dS^T buffers (32 KB each, two 64-column halves), four 4 KB dQ staging
+// boxes, two offset slots and the ones (4 KB each), barriers.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -82,31 +90,40 @@ constexpr int kHalf = 128 * 64 * 2;   // one 64-column half of a [128 x 128] bf1
 // shared-memory map (offsets from the 1 KB aligned base)
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kTile;
-constexpr int kOffQ = kOffV + kTile;          // [2] stages
-constexpr int kOffDO = kOffQ + 2 * kTile;     // [2] stages
-constexpr int kOffDS = kOffDO + 2 * kTile;    // [2] dS^T buffers, each two 64-column halves
+constexpr int kStages = 3;                    // Q / dO stages
+constexpr int kOffQ = kOffV + kTile;          // [kStages]
+constexpr int kOffDO = kOffQ + kStages * kTile;  // [kStages]
+constexpr int kOffDS = kOffDO + kStages * kTile;  // [2] dS^T buffers, each two 64-column halves
 constexpr int kDsBytes = 2 * kHalf;
-constexpr int kOffStage = kOffDS + 2 * kDsBytes;  // dQ staging: per dQ warp two [32 x 32] fp32 boxes
-constexpr int kStageBoxBytes = 32 * 32 * 4;   // 128-byte-swizzled, as the tensor reduction reads them
-constexpr int kStageWarpBytes = 2 * kStageBoxBytes;
-constexpr int kOffRow = kOffStage + 4 * kStageWarpBytes;  // per P/dS warp: lse2[64], delta[64]
-constexpr int kRowWarpBytes = 2 * 64 * 4;
-constexpr int kOffBar = kOffRow + kPdsWarps * kRowWarpBytes;
+constexpr int kOffStage = kOffDS + 2 * kDsBytes;  // dQ staging: per dQ warp one [32 x 32] fp32 box
+constexpr int kStageBoxBytes = 32 * 32 * 4;   // 128-byte-swizzled, as the tensor reduction reads it
+// Offset blocks ([128 x 16] bf16, 32-byte swizzle, one K = 16 slice): two
+// slots, each holding a tile's Q offsets (-LSE / scale, logical columns 0-2)
+// and dO offsets (-delta, columns 8-10), then the block of ones (columns 0-2)
+constexpr int kAugBytes = 128 * 16 * 2;
+constexpr int kOffAug = kOffStage + 4 * kStageBoxBytes;  // [2] slots
+constexpr int kOffOnes = kOffAug + 2 * kAugBytes;
+constexpr int kOffBar = kOffOnes + kAugBytes;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
+static_assert(kOffAug % 1024 == 0 && kSmemBytes <= 227 * 1024, "shared memory map");
 
 struct Bars {
     static constexpr int kKVFull = 0, kKVEmpty = 8;
-    static constexpr int kQFull = 16;    // [2]
-    static constexpr int kQEmpty = 32;   // [2]
-    static constexpr int kSFull = 48, kSFree = 56;
-    static constexpr int kPFull = 64;    // P^T (TMEM) and dS^T (SMEM) of a tile written
-    static constexpr int kPTFree = 72;   // dV of a tile retired: P^T's TMEM columns free
-    static constexpr int kDQFull = 80, kDQEmpty = 88;
-    static constexpr int kDKVFull = 96, kDKVEmpty = 104;
-    static constexpr int kDrain = 112;
-    static constexpr int kDsFree = 120;  // [2] dK and dQ of a tile retired: its dS^T buffer free
-    static constexpr int kTmemSlot = 136, kAbort = 140;
+    static constexpr int kQFull = 16;    // [kStages]
+    static constexpr int kQEmpty = 40;   // [kStages]
+    static constexpr int kSFull = 64, kSFree = 72;
+    static constexpr int kPFull = 80;    // P^T (TMEM) and dS^T (SMEM) of a tile written
+    static constexpr int kPTFree = 88;   // dV of a tile retired: P^T's TMEM columns free
+    static constexpr int kDQFull = 96, kDQEmpty = 104;
+    static constexpr int kDKVFull = 112, kDKVEmpty = 120;
+    static constexpr int kDrain = 128;
+    static constexpr int kDsFree = 136;    // [2] dK and dQ of a tile retired: its dS^T buffer free
+    static constexpr int kAugFull = 152;   // [2] a tile's offset rows written
+    static constexpr int kAugEmpty = 168;  // [2] S^T and dP^T of the tile that used them retired
+    static constexpr int kTmemSlot = 184, kAbort = 188;
 };
+static_assert(Bars::kQFull + 8 * kStages <= Bars::kQEmpty && Bars::kQEmpty + 8 * kStages <= Bars::kSFull,
+              "barrier map");
 
 struct BwdParams {
     int BH, H, N, n_kb, n_qt, total_units, causal;
@@ -114,6 +131,7 @@ struct BwdParams {
     const uint8_t* block_mask;  // [n_bt, n_bt] (nonzero = block computed) or null
     int n_bt;                   // ceil(N / 128)
     float scale, scale_log2;
+    float neg_inv_scale;  // -1 / scale, rounded once
     const float* lse;     // [BH, N]
     const float* delta;   // [BH, N]
     float* dq;            // [BH, N, 64] fp32, accumulated
@@ -170,10 +188,80 @@ __device__ __forceinline__ bool wait_b(const Ctx& c, uint32_t bar, uint32_t pari
     return wait_bounded(bar, parity, c.abort_flag, c.p.wait_ns);
 }
 
+// c = h1 + h2 + h3 with bf16 parts rounded to nearest, |c - (h1 + h2 + h3)|
+// <= 2^-24 |c| (each difference is exact in fp32): packed (h1 | h2 << 16, h3)
+__device__ __forceinline__ uint2 split_bf16x3(float c) {
+    const uint32_t h1 = pack_bf16x2(c, 0.f) & 0xFFFFu;
+    const float r1 = c - __uint_as_float(h1 << 16);
+    const uint32_t h2 = pack_bf16x2(r1, 0.f) & 0xFFFFu;
+    const float r2 = r1 - __uint_as_float(h2 << 16);
+    const uint32_t h3 = pack_bf16x2(r2, 0.f) & 0xFFFFu;
+    return make_uint2(h1 | (h2 << 16), h3);
+}
+
+// The lowest bf16 (-0x1.fep127): the score offset of a query row without
+// probability mass (past N, or LSE = -inf), so that every scaled score of the
+// row is <= -4.8e8 and its P is exactly 0 (scale >= 1e-30).
+constexpr float kNoRowOffset = -0x1.fep127f;
+
+// 32-byte swizzle (K-major, 32-byte rows): logical 16-byte chunk c of row j
+// sits at chunk c ^ ((j >> 2) & 1) -- address bit 4 takes bit 7's value.
+__device__ __forceinline__ uint32_t sw32_off(int j, int c) {
+    return static_cast<uint32_t>(j) * 32u + (static_cast<uint32_t>(c ^ ((j >> 2) & 1)) << 4);
+}
+
+// Offset rows of query tile i into one [rows x 16] block: row j holds
+// split(-LSE_q / scale) in logical columns 0-2 and split(-delta_q) in columns
+// 8-10; the other columns stay zero.  S^T reads the block from its start, dP^T
+// 16 bytes in, so that columns 8-15 come first (its columns 8-15 are then
+// the next row's first ones, finite, and meet the zeros of the ones block).
+// Lane `lane` of the load warp writes rows lane, lane + 32, ...
+template <int ROWS>
+struct OffsetRows {
+    float l[ROWS / 32], d[ROWS / 32];
+    __device__ __forceinline__ void fetch(const BwdParams& p, const float* lse_h, const float* dl_h, int row0,
+                                          int lane) {
+#pragma unroll
+        for (int t = 0; t < ROWS / 32; ++t) {
+            const int q = row0 + lane + 32 * t;
+            l[t] = q < p.N ? lse_h[q] : -INFINITY;
+            d[t] = q < p.N ? dl_h[q] : 0.f;
+        }
+    }
+    __device__ __forceinline__ void store(const BwdParams& p, uint32_t aug, int lane) const {
+#pragma unroll
+        for (int t = 0; t < ROWS / 32; ++t) {
+            const int j = lane + 32 * t;
+            const bool in = l[t] > -INFINITY;
+            const uint2 a = split_bf16x3(in ? l[t] * p.neg_inv_scale : kNoRowOffset);
+            const uint2 b = split_bf16x3(in ? -d[t] : 0.f);
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(aug + sw32_off(j, 0)), "r"(a.x), "r"(a.y) : "memory");
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(aug + sw32_off(j, 1)), "r"(b.x), "r"(b.y) : "memory");
+        }
+    }
+};
+
+// Zeroes `bytes` of offset blocks from `zero` and fills the ones block (bf16
+// 1.0 in logical columns 0-2 of each of `rows` rows, zero elsewhere); all
+// threads of the CTA take part, before the barrier that starts the roles.
+__device__ __forceinline__ void init_offset_blocks(uint8_t* zero, int bytes, uint8_t* ones, int rows) {
+    for (int k = threadIdx.x; k < bytes / 16; k += blockDim.x)
+        reinterpret_cast<uint4*>(zero)[k] = make_uint4(0u, 0u, 0u, 0u);
+    for (int k = threadIdx.x; k < rows * 2; k += blockDim.x) {
+        const int j = k >> 1, c = k & 1;  // logical chunk c of row j
+        *reinterpret_cast<uint4*>(ones + sw32_off(j, c)) =
+            c == 0 ? make_uint4(0x3F803F80u, 0x3F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async();
+}
+
 // ---------------------------------------------------------------- TMA producer
+// The whole warp: lane 0 issues the copies; every lane writes offset rows
+// and arrives on the offset slot's full barrier (count 32).
 __device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, const CUtensorMap* tk,
-                                          const CUtensorMap* tv, const CUtensorMap* tdo) {
+                                          const CUtensorMap* tv, const CUtensorMap* tdo, int lane) {
     const BwdParams& p = c.p;
+    const bool leader = lane == 0;
     uint32_t g = 0;      // query tiles issued
     uint32_t units = 0;  // units whose K / V were issued
     bool ok = true;
@@ -181,32 +269,51 @@ __device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, c
         const BwdUnit w = bwd_unit(u, p);
         int i = next_tile(p, w, w.i0, kBQ);
         if (i >= p.n_qt) continue;  // no query tile meets this key block
-        if (!wait_b(c, c.bar + Bars::kKVEmpty, (units & 1) ^ 1)) {
+        if (!__all_sync(0xffffffffu, wait_b(c, c.bar + Bars::kKVEmpty, (units & 1) ^ 1))) {
             ok = false;
             break;
         }
-        mbar_expect_tx(c.bar + Bars::kKVFull, 2 * kTile);
-        tma_load_4d(c.base + kOffK, tk, c.bar + Bars::kKVFull, 0, w.kb * kBK, w.bh, 0);
-        tma_load_4d(c.base + kOffV, tv, c.bar + Bars::kKVFull, 0, w.kb * kBK, w.bh, 0);
+        if (leader) {
+            mbar_expect_tx(c.bar + Bars::kKVFull, 2 * kTile);
+            tma_load_4d(c.base + kOffK, tk, c.bar + Bars::kKVFull, 0, w.kb * kBK, w.bh, 0);
+            tma_load_4d(c.base + kOffV, tv, c.bar + Bars::kKVFull, 0, w.kb * kBK, w.bh, 0);
+        }
         ++units;
+        const float* lse_h = p.lse + static_cast<size_t>(w.bh) * p.N;
+        const float* dl_h = p.delta + static_cast<size_t>(w.bh) * p.N;
         for (; i < p.n_qt; i = next_tile(p, w, i + 1, kBQ), ++g) {
-            const uint32_t s = g & 1;
-            if (!wait_b(c, c.bar + Bars::kQEmpty + 8 * s, ((g >> 1) & 1) ^ 1)) {
+            const uint32_t s = g % kStages;
+            // the offset rows first: their slot frees when S^T of tile g-2
+            // retires, long before the Q / dO stage (after dK of tile g-3)
+            OffsetRows<kBQ> rows;
+            rows.fetch(p, lse_h, dl_h, i * kBQ, lane);
+            const uint32_t a = g & 1;  // offset slot
+            if (!__all_sync(0xffffffffu, wait_b(c, c.bar + Bars::kAugEmpty + 8 * a, ((g >> 1) & 1) ^ 1))) {
                 ok = false;
                 break;
             }
-            const uint32_t fb = c.bar + Bars::kQFull + 8 * s;
-            mbar_expect_tx(fb, 2 * kTile);
-            tma_load_4d(c.base + kOffQ + s * kTile, tq, fb, 0, i * kBQ, w.bh, 0);
-            tma_load_4d(c.base + kOffDO + s * kTile, tdo, fb, 0, i * kBQ, w.bh, 0);
+            rows.store(p, c.base + kOffAug + a * kAugBytes, lane);
+            fence_proxy_async();  // the tensor core reads what the generic proxy wrote
+            mbar_arrive(c.bar + Bars::kAugFull + 8 * a);
+            if (!__all_sync(0xffffffffu, wait_b(c, c.bar + Bars::kQEmpty + 8 * s, ((g / kStages) & 1) ^ 1))) {
+                ok = false;
+                break;
+            }
+            if (leader) {
+                const uint32_t fb = c.bar + Bars::kQFull + 8 * s;
+                mbar_expect_tx(fb, 2 * kTile);
+                tma_load_4d(c.base + kOffQ + s * kTile, tq, fb, 0, i * kBQ, w.bh, 0);
+                tma_load_4d(c.base + kOffDO + s * kTile, tdo, fb, 0, i * kBQ, w.bh, 0);
+            }
         }
     }
-    if (!ok) {
+    if (!ok && leader) {
         // every issued copy lands before the CTA may exit
         if (units > 0) wait_bounded(c.bar + Bars::kKVFull, (units - 1) & 1, nullptr, kDrainNs);
-        for (uint32_t k = (g > 2 ? g - 2 : 0); k < g; ++k)
-            wait_bounded(c.bar + Bars::kQFull + 8 * (k & 1), (k >> 1) & 1, nullptr, kDrainNs);
+        for (uint32_t k = (g > kStages ? g - kStages : 0); k < g; ++k)
+            wait_bounded(c.bar + Bars::kQFull + 8 * (k % kStages), (k / kStages) & 1, nullptr, kDrainNs);
     }
+    __syncwarp();
 }
 
 // ---------------------------------------------------------------- MMA issuing
@@ -219,12 +326,16 @@ struct BwdMma {
     // M = 128, N = 64, A and B M/N-major (dQ: A = dS read from the dS^T tile)
     static constexpr uint32_t kIdescTT = idesc_bf16_f32(128, 64, true) | (1u << 15);
 
-    // D[128 x 128] = A[128 x 64] B[128 x 64]^T, both K-major tiles
-    __device__ __forceinline__ static void nt(uint32_t d, uint32_t a, uint32_t b) {
+    static constexpr uint32_t kHiAug = sdesc_hi_sw32(256);
+
+    // D[128 x 128] = A[128 x 64] B[128 x 64]^T + ones[128 x 16] aug[128 x 16]^T,
+    // all K-major: the tile product plus each column's offset
+    __device__ __forceinline__ static void nt(uint32_t d, uint32_t a, uint32_t b, uint32_t ones, uint32_t aug) {
         const uint32_t a0 = sdesc_lo(a, 16), b0 = sdesc_lo(b, 16);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
             mma_ss_lo(d, a0 + ((kk * 32) >> 4), b0 + ((kk * 32) >> 4), kHi, kIdescNN, kk > 0 ? 1u : 0u);
+        mma_ss_lo(d, sdesc_lo(ones, 16), sdesc_lo(aug, 16), kHiAug, kIdescNN, 1u);
     }
     // D[128 x 64] (+)= A[128 x 128] B[128 x 64]: A K-major in two 64-column
     // halves, B M/N-major (rows = the 128-long K dimension)
@@ -264,15 +375,19 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
     };
     uint32_t g = 0;       // query tiles of this CTA so far (S issued for tiles < g_s)
     uint32_t units = 0;
-    // S^T and dP^T of tile g into TMEM, once the P/dS warps have loaded tile g-1
+    // S^T - LSE/scale and dP^T - delta of tile g into TMEM, once the P/dS
+    // warps have loaded tile g-1
     auto issue_s = [&](uint32_t gg) {
-        const uint32_t s = gg & 1;
-        if (!wait(c.bar + Bars::kQFull + 8 * s, (gg >> 1) & 1)) return;
+        const uint32_t s = gg % kStages, a = gg & 1;
+        if (!wait(c.bar + Bars::kQFull + 8 * s, (gg / kStages) & 1)) return;
+        if (!wait(c.bar + Bars::kAugFull + 8 * a, (gg >> 1) & 1)) return;
         if (gg > 0 && !wait(c.bar + Bars::kSFree, (gg - 1) & 1)) return;
         tc_fence_after();
-        BwdMma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kTile);
-        BwdMma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kTile);
+        const uint32_t aug = c.base + kOffAug + a * kAugBytes;
+        BwdMma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kTile, c.base + kOffOnes, aug);
+        BwdMma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kTile, c.base + kOffOnes, aug + 16);
         tc_commit(c.bar + Bars::kSFull);
+        tc_commit(c.bar + Bars::kAugEmpty + 8 * a);
     };
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
@@ -287,14 +402,14 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
             if (it == 0 && !wait(c.bar + Bars::kDKVEmpty, (units & 1) ^ 1)) break;
             if (!wait(c.bar + Bars::kDQEmpty, (g & 1) ^ 1)) break;
             tc_fence_after();
-            const uint32_t s = g & 1;
-            const uint32_t ds = c.base + kOffDS + s * kDsBytes;
+            const uint32_t s = g % kStages, b = g & 1;
+            const uint32_t ds = c.base + kOffDS + b * kDsBytes;
             BwdMma::ts(t + kColDV, t + kColP, c.base + kOffDO + s * kTile, it > 0);  // dV += P^T dO
             tc_commit(c.bar + Bars::kPTFree);
             BwdMma::kt(t + kColDK, ds, c.base + kOffQ + s * kTile, it > 0);          // dK += dS^T Q
+            tc_commit(c.bar + Bars::kQEmpty + 8 * s);  // the last read of Q_i and dO_i
             BwdMma::tt(t + kColDQ, ds, c.base + kOffK);                               // dQ_j = dS K
-            tc_commit(c.bar + Bars::kDsFree + 8 * s);
-            tc_commit(c.bar + Bars::kQEmpty + 8 * s);
+            tc_commit(c.bar + Bars::kDsFree + 8 * b);
             tc_commit(c.bar + Bars::kDQFull);
             if (inext >= p.n_qt) {
                 tc_commit(c.bar + Bars::kDKVFull);
@@ -340,7 +455,6 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
     const uint32_t t_s = c.tmem + lane_off + kColS + col0, t_dp = c.tmem + lane_off + kColDP + col0;
     const uint32_t t_acc = c.tmem + lane_off + (half == 0 ? kColDV : kColDK);
     const uint32_t t_p = c.tmem + lane_off + kColP + col0 / 2;  // bf16 pairs
-    const uint32_t rows_smem = c.base + kOffRow + warp * kRowWarpBytes;  // lse2[64], delta[64]
     const float sl2 = p.scale_log2;
     uint32_t g = 0, units = 0;
     bool ok = true;
@@ -349,22 +463,6 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
         const int key = w.kb * kBK + r;
         // padded keys (and rows past N) take no part: P = dS = 0 on their rows
         const bool key_ok = key < p.N && (p.key_pad == nullptr || p.key_pad[static_cast<size_t>(w.bh / p.H) * p.N + key] == 0);
-        const float* lse_h = p.lse + static_cast<size_t>(w.bh) * p.N;
-        const float* dl_h = p.delta + static_cast<size_t>(w.bh) * p.N;
-        // LSE * log2(e) and delta of this lane's two query rows of tile i
-        // (rows past N, and rows that saw no key (LSE = -inf, O = 0): +inf and
-        // delta = 0, so P = dS = 0), fetched one tile ahead
-        float pre_l[2], pre_d[2];
-        auto fetch = [&](int i) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int q = i * kBQ + col0 + lane * 2 + e;
-                const float l = q < p.N ? lse_h[q] : -INFINITY;
-                const bool in = l > -INFINITY;
-                pre_l[e] = in ? l * kLog2eB : INFINITY;
-                pre_d[e] = in ? dl_h[q] : 0.f;
-            }
-        };
         int i = next_tile(p, w, w.i0, kBQ);
         if (i >= p.n_qt) {
             // no query tile meets this key block: its dK and dV rows are zero
@@ -376,17 +474,8 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             }
             continue;
         }
-        fetch(i);
         for (; i < p.n_qt; ++g) {
-            __syncwarp();
-            asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(rows_smem + lane * 8), "f"(pre_l[0]), "f"(pre_l[1])
-                         : "memory");
-            asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(rows_smem + 256 + lane * 8), "f"(pre_d[0]),
-                         "f"(pre_d[1])
-                         : "memory");
-            __syncwarp();
             const int inext = next_tile(p, w, i + 1, kBQ);
-            if (inext < p.n_qt) fetch(inext);
             bool got = wait_b(c, c.bar + Bars::kSFull, g & 1);
             got = __all_sync(0xffffffffu, got);
             if (!got) {
@@ -398,8 +487,10 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             // a warp-uniform fast path when no element of the warp's rows is masked
             const bool masked = __any_sync(0xffffffffu, !key_ok || diag);
             const uint32_t ds_buf = c.base + kOffDS + (g & 1) * kDsBytes;
-            // both 32-column chunks of this thread's S^T and dP^T row, then
-            // release them at once: the next tile's products start now
+            // both 32-column chunks of this thread's row of S^T - LSE/scale
+            // and dP^T - delta, then release them at once: the next tile's
+            // products start now (rows past N, or without any visible key,
+            // carry the lowest offset and give P = dS = 0)
             uint32_t sr[2][32], dr[2][32];
             tmem_ld32(t_s, sr[0]);
             tmem_ld32(t_s + 32, sr[1]);
@@ -417,28 +508,19 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
                 uint32_t pk[16], dk[16];
                 const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const float4 l2 = ld_shared_f4(rows_smem + (c4 * 32 + v * 4) * 4);
-                    const float4 dl = ld_shared_f4(rows_smem + 256 + (c4 * 32 + v * 4) * 4);
-#pragma unroll
-                    for (int e2 = 0; e2 < 2; ++e2) {
-                        const int e = v * 4 + e2 * 2;
-                        const float2 nl = e2 == 0 ? make_float2(-l2.x, -l2.y) : make_float2(-l2.z, -l2.w);
-                        const float2 nd = e2 == 0 ? make_float2(-dl.x, -dl.y) : make_float2(-dl.z, -dl.w);
-                        float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[c4][e]), __uint_as_float(sr[c4][e + 1])),
-                                              sl2x2, nl);
-                        x.x = ex2(x.x);
-                        x.y = ex2(x.y);
-                        if (masked) {
-                            const int q = col0 + c4 * 32 + e;
-                            if (!key_ok || (diag && q < r)) x.x = 0.f;
-                            if (!key_ok || (diag && q + 1 < r)) x.y = 0.f;
-                        }
-                        const float2 dsv = __fmul2_rn(
-                            x, __fadd2_rn(make_float2(__uint_as_float(dr[c4][e]), __uint_as_float(dr[c4][e + 1])), nd));
-                        pk[e >> 1] = pack_bf16x2(x.x, x.y);
-                        dk[e >> 1] = pack_bf16x2(dsv.x, dsv.y);
+                for (int e = 0; e < 32; e += 2) {
+                    float2 x = __fmul2_rn(make_float2(__uint_as_float(sr[c4][e]), __uint_as_float(sr[c4][e + 1])),
+                                          sl2x2);
+                    x.x = ex2(x.x);
+                    x.y = ex2(x.y);
+                    if (masked) {
+                        const int q = col0 + c4 * 32 + e;
+                        if (!key_ok || (diag && q < r)) x.x = 0.f;
+                        if (!key_ok || (diag && q + 1 < r)) x.y = 0.f;
                     }
+                    const float2 dsv = __fmul2_rn(x, make_float2(__uint_as_float(dr[c4][e]), __uint_as_float(dr[c4][e + 1])));
+                    pk[e >> 1] = pack_bf16x2(x.x, x.y);
+                    dk[e >> 1] = pack_bf16x2(dsv.x, dsv.y);
                 }
                 if (c4 == 0 && g > 0) {
                     // P^T's TMEM columns: dV of the previous tile must have retired
@@ -512,17 +594,18 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
 }
 
 // ------------------------------------------------------------- dQ warps (8-11)
-// Thread = query row of the tile = TMEM lane.  Each warp stages its 32 rows
-// as two [32 x 32] fp32 boxes in the 128-byte-swizzled layout and adds them
-// to dQ with two tensor reductions (cp.reduce.async.bulk.tensor .add); the
-// tensor map clips rows past N.
+// Thread = query row of the tile = TMEM lane.  Each warp reads its 32 rows
+// (64 columns) from TMEM, releases the accumulator, and adds them to dQ as
+// two [32 x 32] fp32 boxes, one after the other through one 128-byte-
+// swizzled staging box, with tensor reductions (cp.reduce.async.bulk.tensor
+// .add); the tensor map clips rows past N.
 __device__ __forceinline__ void role_dq(const Ctx& c, const CUtensorMap* tm_dq, int warp, int lane) {
     const BwdParams& p = c.p;
     const int quarter = warp & 3;
     const uint32_t t_dq = c.tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColDQ;
-    const uint32_t stage = c.base + kOffStage + quarter * kStageWarpBytes;
+    const uint32_t stage = c.base + kOffStage + quarter * kStageBoxBytes;
     uint32_t g = 0;
-    bool pending = false;  // lane 0: this warp's last reductions may still read the staging boxes
+    bool pending = false;  // lane 0: this warp's last reduction may still read the staging box
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
@@ -534,41 +617,39 @@ __device__ __forceinline__ void role_dq(const Ctx& c, const CUtensorMap* tm_dq, 
                 break;
             }
             tc_fence_after();
-            if (lane == 0 && pending) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-            pending = false;
-            __syncwarp();
+            uint32_t a[2][32];
+            tmem_ld32(t_dq, a[0]);
+            tmem_ld32(t_dq + 32, a[1]);
+            tmem_wait_ld();
+            reg_fence32(a[0]);
+            reg_fence32(a[1]);
+            tc_fence_before();
+            mbar_arrive(c.bar + Bars::kDQEmpty);
+            const int row0 = i * kBQ + quarter * 32;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                uint32_t a[32];
-                tmem_ld32(t_dq + h * 32, a);
-                tmem_wait_ld();
-                reg_fence32(a);
-                if (h == 1) {
-                    tc_fence_before();
-                    mbar_arrive(c.bar + Bars::kDQEmpty);
-                }
-                // row `lane` of box h: 16-byte chunk v4 at chunk v4 ^ (lane % 8)
+                // the box is free once the previous reduction has read it
+                if (lane == 0 && pending) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                pending = false;
+                __syncwarp();
+                // row `lane` of the box: 16-byte chunk v4 at chunk v4 ^ (lane % 8)
 #pragma unroll
                 for (int v4 = 0; v4 < 8; ++v4)
-                    st_shared_v4(stage + h * kStageBoxBytes + lane * 128 + ((v4 ^ (lane & 7)) << 4),
-                                 __float_as_uint(__uint_as_float(a[v4 * 4]) * p.scale),
-                                 __float_as_uint(__uint_as_float(a[v4 * 4 + 1]) * p.scale),
-                                 __float_as_uint(__uint_as_float(a[v4 * 4 + 2]) * p.scale),
-                                 __float_as_uint(__uint_as_float(a[v4 * 4 + 3]) * p.scale));
-            }
-            fence_proxy_async();
-            __syncwarp();
-            const int row0 = i * kBQ + quarter * 32;
-            if (lane == 0 && row0 < p.N) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
+                    st_shared_v4(stage + lane * 128 + ((v4 ^ (lane & 7)) << 4),
+                                 __float_as_uint(__uint_as_float(a[h][v4 * 4]) * p.scale),
+                                 __float_as_uint(__uint_as_float(a[h][v4 * 4 + 1]) * p.scale),
+                                 __float_as_uint(__uint_as_float(a[h][v4 * 4 + 2]) * p.scale),
+                                 __float_as_uint(__uint_as_float(a[h][v4 * 4 + 3]) * p.scale));
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0 && row0 < p.N) {
                     asm volatile(
                         "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
-                        ::"l"(reinterpret_cast<uint64_t>(tm_dq)), "r"(h * 32), "r"(row0), "r"(w.bh),
-                        "r"(stage + h * kStageBoxBytes)
+                        ::"l"(reinterpret_cast<uint64_t>(tm_dq)), "r"(h * 32), "r"(row0), "r"(w.bh), "r"(stage)
                         : "memory");
-                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                pending = true;
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    pending = true;
+                }
             }
         }
     }
@@ -592,9 +673,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (threadIdx.x == 0) {
         mbar_init(bar + Bars::kKVFull, 1);
         mbar_init(bar + Bars::kKVEmpty, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(bar + Bars::kQFull + 8 * s, 1);
             mbar_init(bar + Bars::kQEmpty + 8 * s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar + Bars::kAugFull + 8 * a, 32);  // the load warp's lanes
+            mbar_init(bar + Bars::kAugEmpty + 8 * a, 1);
         }
         mbar_init(bar + Bars::kSFull, 1);
         mbar_init(bar + Bars::kSFree, kPdsThreads);
@@ -622,6 +707,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_alloc(smem_addr(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
+    init_offset_blocks(gbase + kOffAug, 2 * kAugBytes, gbase + kOffOnes, 128);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -634,9 +720,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         role_dq(ctx, &tm_dq, warp, lane);
     } else {
         regs_decrease<kOtherRegs>();
-        if (lane == 0) {
-            if (warp == kLoadWarp) role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do);
-            else if (warp == kMmaWarp) role_mma(ctx);
+        if (warp == kLoadWarp) {
+            role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do, lane);
+        } else if (warp == kMmaWarp && lane == 0) {
+            role_mma(ctx);
         }
         __syncwarp();
     }
@@ -882,13 +969,12 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
         const bool key_ok = key < p.N && (p.key_pad == nullptr || p.key_pad[static_cast<size_t>(w.bh / p.H) * p.N + key] == 0);
         const float* lse_h = p.lse + static_cast<size_t>(w.bh) * p.N;
         const float* dl_h = p.delta + static_cast<size_t>(w.bh) * p.N;
-        float pre_l, pre_d;
+        // fetched one tile ahead, converted when staged (as at d = 64)
+        float raw_l, raw_d;
         auto fetch = [&](int i) {
             const int q = i * kBQ + col0 + lane;
-            const float l = q < p.N ? lse_h[q] : -INFINITY;
-            const bool in = l > -INFINITY;
-            pre_l = in ? l * kLog2eB : INFINITY;
-            pre_d = in ? dl_h[q] : 0.f;
+            raw_l = q < p.N ? lse_h[q] : -INFINITY;
+            raw_d = q < p.N ? dl_h[q] : 0.f;
         };
         int i = next_tile(p, w, w.i0, kBQ);
         if (i >= p.n_qt) {
@@ -903,6 +989,8 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
         }
         fetch(i);
         for (; i < p.n_qt; ++g) {
+            const bool in = raw_l > -INFINITY;
+            const float pre_l = in ? raw_l * kLog2eB : INFINITY, pre_d = in ? raw_d : 0.f;
             __syncwarp();
             asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + lane * 4), "f"(pre_l) : "memory");
             asm volatile("st.shared.f32 [%0], %1;" ::"r"(rows_smem + 128 + lane * 4), "f"(pre_d) : "memory");
@@ -1381,6 +1469,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     p.causal = causal ? 1 : 0;
     p.scale = scale;
     p.scale_log2 = scale * kLog2eB;
+    p.neg_inv_scale = static_cast<float>(-1.0 / static_cast<double>(scale));
     p.lse = lse;
     p.delta = delta;
     p.dq = dq;

@@ -294,6 +294,11 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
 __host__ __device__ constexpr uint32_t sdesc_hi_sw128(uint32_t sbo_bytes) {
     return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
+// The same for the 32-byte swizzle (layout type 6): K-major rows of 32 bytes
+// (one K = 16 slice of bf16), 8-row atoms of 256 bytes.
+__host__ __device__ constexpr uint32_t sdesc_hi_sw32(uint32_t sbo_bytes) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (6u << 29);
+}
 __device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
     return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
 }
