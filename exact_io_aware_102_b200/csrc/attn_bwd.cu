@@ -97,32 +97,37 @@ constexpr int kOffDS = kOffDO + kStages * kTile;  // [2] dS^T buffers, each two 
 constexpr int kDsBytes = 2 * kHalf;
 constexpr int kOffStage = kOffDS + 2 * kDsBytes;  // dQ staging: per dQ warp one [32 x 32] fp32 box
 constexpr int kStageBoxBytes = 32 * 32 * 4;   // 128-byte-swizzled, as the tensor reduction reads it
-// Offset blocks ([128 x 16] bf16, 32-byte swizzle, one K = 16 slice): two
-// slots, each holding a tile's Q offsets (-LSE / scale, logical columns 0-2)
+// Offset blocks ([128 x 16] bf16, 32-byte swizzle, one K = 16 slice): one
+// per stage, holding the tile's Q offsets (-LSE / scale, logical columns 0-2)
 // and dO offsets (-delta, columns 8-10), then the block of ones (columns 0-2)
 constexpr int kAugBytes = 128 * 16 * 2;
-constexpr int kOffAug = kOffStage + 4 * kStageBoxBytes;  // [2] slots
-constexpr int kOffOnes = kOffAug + 2 * kAugBytes;
+constexpr int kOffAug = kOffStage + 4 * kStageBoxBytes;  // [kStages]
+constexpr int kOffOnes = kOffAug + kStages * kAugBytes;
 constexpr int kOffBar = kOffOnes + kAugBytes;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
 static_assert(kOffAug % 1024 == 0 && kSmemBytes <= 227 * 1024, "shared memory map");
 
+// Barriers.  The tensor-core thread waits on two per query tile (Ready,
+// PFull) and commits three (SFull, PTFree, TileDone): each wait or commit
+// leaves the shallow tensor-instruction queue to drain for tens of cycles.
 struct Bars {
     static constexpr int kKVFull = 0, kKVEmpty = 8;
-    static constexpr int kQFull = 16;    // [kStages]
-    static constexpr int kQEmpty = 40;   // [kStages]
-    static constexpr int kSFull = 64, kSFree = 72;
-    static constexpr int kPFull = 80;    // P^T (TMEM) and dS^T (SMEM) of a tile written
-    static constexpr int kPTFree = 88;   // dV of a tile retired: P^T's TMEM columns free
-    static constexpr int kDQFull = 96, kDQEmpty = 104;
-    static constexpr int kDKVFull = 112, kDKVEmpty = 120;
-    static constexpr int kDrain = 128;
-    static constexpr int kDsFree = 136;    // [2] dK and dQ of a tile retired: its dS^T buffer free
-    static constexpr int kAugFull = 152;   // [2] a tile's offset rows written
-    static constexpr int kAugEmpty = 168;  // [2] S^T and dP^T of the tile that used them retired
-    static constexpr int kTmemSlot = 184, kAbort = 188;
+    // [kStages] tile g may start: its Q, dO (bytes) and offset rows (32 load
+    // lanes) have landed, and the P/dS warps (256) have read S^T of tile g-1
+    static constexpr int kReady = 16;
+    // [kStages] the products of tile g retired: its stage, its dS^T buffer
+    // and (for the dQ warps) its dQ partial in TMEM
+    static constexpr int kTileDone = 40;
+    static constexpr int kSFull = 64;
+    // P^T (TMEM) and dS^T (SMEM) of tile g written (256 P/dS threads), and
+    // the dQ partial of tile g-1 read (128 dQ threads)
+    static constexpr int kPFull = 72;
+    static constexpr int kPTFree = 80;   // dV of a tile retired: P^T's TMEM columns free
+    static constexpr int kDKVFull = 88, kDKVEmpty = 96;
+    static constexpr int kDrain = 104;
+    static constexpr int kTmemSlot = 112, kAbort = 116;
 };
-static_assert(Bars::kQFull + 8 * kStages <= Bars::kQEmpty && Bars::kQEmpty + 8 * kStages <= Bars::kSFull,
+static_assert(Bars::kReady + 8 * kStages <= Bars::kTileDone && Bars::kTileDone + 8 * kStages <= Bars::kSFull,
               "barrier map");
 
 struct BwdParams {
@@ -256,8 +261,9 @@ __device__ __forceinline__ void init_offset_blocks(uint8_t* zero, int bytes, uin
 }
 
 // ---------------------------------------------------------------- TMA producer
-// The whole warp: lane 0 issues the copies; every lane writes offset rows
-// and arrives on the offset slot's full barrier (count 32).
+// The whole warp: lane 0 issues the copies (its arrival on the stage's Ready
+// barrier carries the expected bytes); every lane writes offset rows and
+// arrives on Ready.
 __device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, const CUtensorMap* tk,
                                           const CUtensorMap* tv, const CUtensorMap* tdo, int lane) {
     const BwdParams& p = c.p;
@@ -283,35 +289,32 @@ __device__ __forceinline__ void role_load(const Ctx& c, const CUtensorMap* tq, c
         const float* dl_h = p.delta + static_cast<size_t>(w.bh) * p.N;
         for (; i < p.n_qt; i = next_tile(p, w, i + 1, kBQ), ++g) {
             const uint32_t s = g % kStages;
-            // the offset rows first: their slot frees when S^T of tile g-2
-            // retires, long before the Q / dO stage (after dK of tile g-3)
             OffsetRows<kBQ> rows;
-            rows.fetch(p, lse_h, dl_h, i * kBQ, lane);
-            const uint32_t a = g & 1;  // offset slot
-            if (!__all_sync(0xffffffffu, wait_b(c, c.bar + Bars::kAugEmpty + 8 * a, ((g >> 1) & 1) ^ 1))) {
+            rows.fetch(p, lse_h, dl_h, i * kBQ, lane);  // in flight while the stage drains
+            // the stage (and its offset block) is free once tile g-3 retired
+            if (!__all_sync(0xffffffffu, wait_b(c, c.bar + Bars::kTileDone + 8 * s, ((g / kStages) & 1) ^ 1))) {
                 ok = false;
                 break;
             }
-            rows.store(p, c.base + kOffAug + a * kAugBytes, lane);
+            rows.store(p, c.base + kOffAug + s * kAugBytes, lane);
             fence_proxy_async();  // the tensor core reads what the generic proxy wrote
-            mbar_arrive(c.bar + Bars::kAugFull + 8 * a);
-            if (!__all_sync(0xffffffffu, wait_b(c, c.bar + Bars::kQEmpty + 8 * s, ((g / kStages) & 1) ^ 1))) {
-                ok = false;
-                break;
-            }
+            const uint32_t rb = c.bar + Bars::kReady + 8 * s;
             if (leader) {
-                const uint32_t fb = c.bar + Bars::kQFull + 8 * s;
-                mbar_expect_tx(fb, 2 * kTile);
-                tma_load_4d(c.base + kOffQ + s * kTile, tq, fb, 0, i * kBQ, w.bh, 0);
-                tma_load_4d(c.base + kOffDO + s * kTile, tdo, fb, 0, i * kBQ, w.bh, 0);
+                mbar_expect_tx(rb, 2 * kTile);
+                tma_load_4d(c.base + kOffQ + s * kTile, tq, rb, 0, i * kBQ, w.bh, 0);
+                tma_load_4d(c.base + kOffDO + s * kTile, tdo, rb, 0, i * kBQ, w.bh, 0);
+            } else {
+                mbar_arrive(rb);
             }
         }
     }
     if (!ok && leader) {
-        // every issued copy lands before the CTA may exit
+        // every issued copy lands before the CTA may exit (the Ready phases
+        // also need arrivals that an aborted CTA may never make: these waits
+        // then end at their limit, long after the copies landed)
         if (units > 0) wait_bounded(c.bar + Bars::kKVFull, (units - 1) & 1, nullptr, kDrainNs);
         for (uint32_t k = (g > kStages ? g - kStages : 0); k < g; ++k)
-            wait_bounded(c.bar + Bars::kQFull + 8 * (k % kStages), (k / kStages) & 1, nullptr, kDrainNs);
+            wait_bounded(c.bar + Bars::kReady + 8 * (k % kStages), (k / kStages) & 1, nullptr, kDrainNs);
     }
     __syncwarp();
 }
@@ -373,21 +376,18 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         if (ok && !wait_b(c, bar, parity)) ok = false;
         return ok;
     };
-    uint32_t g = 0;       // query tiles of this CTA so far (S issued for tiles < g_s)
+    uint32_t g = 0;       // query tiles of this CTA so far
     uint32_t units = 0;
-    // S^T - LSE/scale and dP^T - delta of tile g into TMEM, once the P/dS
-    // warps have loaded tile g-1
+    // S^T - LSE/scale and dP^T - delta of tile g into TMEM, once its inputs
+    // have landed and the P/dS warps have read tile g-1's
     auto issue_s = [&](uint32_t gg) {
-        const uint32_t s = gg % kStages, a = gg & 1;
-        if (!wait(c.bar + Bars::kQFull + 8 * s, (gg / kStages) & 1)) return;
-        if (!wait(c.bar + Bars::kAugFull + 8 * a, (gg >> 1) & 1)) return;
-        if (gg > 0 && !wait(c.bar + Bars::kSFree, (gg - 1) & 1)) return;
+        const uint32_t s = gg % kStages;
+        if (!wait(c.bar + Bars::kReady + 8 * s, (gg / kStages) & 1)) return;
         tc_fence_after();
-        const uint32_t aug = c.base + kOffAug + a * kAugBytes;
+        const uint32_t aug = c.base + kOffAug + s * kAugBytes;
         BwdMma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kTile, c.base + kOffOnes, aug);
         BwdMma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kTile, c.base + kOffOnes, aug + 16);
         tc_commit(c.bar + Bars::kSFull);
-        tc_commit(c.bar + Bars::kAugEmpty + 8 * a);
     };
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
@@ -398,19 +398,17 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         for (int it = 0; ok && i < p.n_qt; ++it, ++g) {
             const int inext = next_tile(p, w, i + 1, kBQ);
             if (inext < p.n_qt) issue_s(g + 1);  // overlaps the P/dS work of tile g
+            // P^T, dS^T of tile g written and the dQ partial of tile g-1 read
             if (!wait(c.bar + Bars::kPFull, g & 1)) break;
             if (it == 0 && !wait(c.bar + Bars::kDKVEmpty, (units & 1) ^ 1)) break;
-            if (!wait(c.bar + Bars::kDQEmpty, (g & 1) ^ 1)) break;
             tc_fence_after();
-            const uint32_t s = g % kStages, b = g & 1;
-            const uint32_t ds = c.base + kOffDS + b * kDsBytes;
+            const uint32_t s = g % kStages;
+            const uint32_t ds = c.base + kOffDS + (g & 1) * kDsBytes;
             BwdMma::ts(t + kColDV, t + kColP, c.base + kOffDO + s * kTile, it > 0);  // dV += P^T dO
             tc_commit(c.bar + Bars::kPTFree);
             BwdMma::kt(t + kColDK, ds, c.base + kOffQ + s * kTile, it > 0);          // dK += dS^T Q
-            tc_commit(c.bar + Bars::kQEmpty + 8 * s);  // the last read of Q_i and dO_i
             BwdMma::tt(t + kColDQ, ds, c.base + kOffK);                               // dQ_j = dS K
-            tc_commit(c.bar + Bars::kDsFree + 8 * b);
-            tc_commit(c.bar + Bars::kDQFull);
+            tc_commit(c.bar + Bars::kTileDone + 8 * s);
             if (inext >= p.n_qt) {
                 tc_commit(c.bar + Bars::kDKVFull);
                 tc_commit(c.bar + Bars::kKVEmpty);
@@ -502,7 +500,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             reg_fence32(dr[0]);
             reg_fence32(dr[1]);
             tc_fence_before();
-            mbar_arrive(c.bar + Bars::kSFree);  // S^T / dP^T may be overwritten
+            mbar_arrive(c.bar + Bars::kReady + 8 * ((g + 1) % kStages));  // S^T / dP^T may be overwritten
 #pragma unroll
             for (int c4 = 0; c4 < 2; ++c4) {
                 uint32_t pk[16], dk[16];
@@ -534,7 +532,7 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
                 }
                 if (c4 == 0 && g > 1) {
                     // this dS^T buffer: dK and dQ of tile g-2 must have retired
-                    bool free = wait_b(c, c.bar + Bars::kDsFree + 8 * (g & 1), ((g >> 1) & 1) ^ 1);
+                    bool free = wait_b(c, c.bar + Bars::kTileDone + 8 * ((g - 2) % kStages), ((g - 2) / kStages) & 1);
                     free = __all_sync(0xffffffffu, free);
                     if (!free) {
                         ok = false;
@@ -610,7 +608,7 @@ __device__ __forceinline__ void role_dq(const Ctx& c, const CUtensorMap* tm_dq, 
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
         for (int i = next_tile(p, w, w.i0, kBQ); i < p.n_qt; i = next_tile(p, w, i + 1, kBQ), ++g) {
-            bool got = wait_b(c, c.bar + Bars::kDQFull, g & 1);
+            bool got = wait_b(c, c.bar + Bars::kTileDone + 8 * (g % kStages), (g / kStages) & 1);
             got = __all_sync(0xffffffffu, got);
             if (!got) {
                 ok = false;
@@ -624,7 +622,7 @@ __device__ __forceinline__ void role_dq(const Ctx& c, const CUtensorMap* tm_dq, 
             reg_fence32(a[0]);
             reg_fence32(a[1]);
             tc_fence_before();
-            mbar_arrive(c.bar + Bars::kDQEmpty);
+            mbar_arrive(c.bar + Bars::kPFull);  // counts toward tile g+1
             const int row0 = i * kBQ + quarter * 32;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -674,21 +672,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar + Bars::kKVFull, 1);
         mbar_init(bar + Bars::kKVEmpty, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar + Bars::kQFull + 8 * s, 1);
-            mbar_init(bar + Bars::kQEmpty + 8 * s, 1);
-        }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(bar + Bars::kAugFull + 8 * a, 32);  // the load warp's lanes
-            mbar_init(bar + Bars::kAugEmpty + 8 * a, 1);
+            mbar_init(bar + Bars::kReady + 8 * s, kPdsThreads + 32);  // P/dS threads, load lanes
+            mbar_init(bar + Bars::kTileDone + 8 * s, 1);
         }
         mbar_init(bar + Bars::kSFull, 1);
-        mbar_init(bar + Bars::kSFree, kPdsThreads);
-        mbar_init(bar + Bars::kPFull, kPdsThreads);
+        mbar_init(bar + Bars::kPFull, kPdsThreads + kBQ);  // P/dS threads, dQ threads
         mbar_init(bar + Bars::kPTFree, 1);
-        mbar_init(bar + Bars::kDsFree, 1);
-        mbar_init(bar + Bars::kDsFree + 8, 1);
-        mbar_init(bar + Bars::kDQFull, 1);
-        mbar_init(bar + Bars::kDQEmpty, kBQ);
         mbar_init(bar + Bars::kDKVFull, 1);
         mbar_init(bar + Bars::kDKVEmpty, kPdsThreads);
         mbar_init(bar + Bars::kDrain, 1);
@@ -707,16 +696,18 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_alloc(smem_addr(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
-    init_offset_blocks(gbase + kOffAug, 2 * kAugBytes, gbase + kOffOnes, 128);
+    init_offset_blocks(gbase + kOffAug, kStages * kAugBytes, gbase + kOffOnes, 128);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const Ctx ctx{base, bar, *tmem_slot, abort_flag, gbase, p};
     if (warp < kPdsWarps) {
         regs_increase<kPdsRegs>();
+        mbar_arrive(bar + Bars::kReady);  // tile 0 has no earlier S^T to read
         role_pds(ctx, warp, lane);
     } else if (warp < kDqWarp0 + 4) {
         regs_decrease<kOtherRegs>();
+        mbar_arrive(bar + Bars::kPFull);  // tile 0 has no earlier dQ partial
         role_dq(ctx, &tm_dq, warp, lane);
     } else {
         regs_decrease<kOtherRegs>();
