@@ -19,10 +19,10 @@
 //     TMEM over the query tiles (128 rows each) the block interacts with;
 //   * warp 12 loads K, V once per unit and Q_i, dO_i per query tile (three
 //     stages at d = 64, two at d = 128) by TMA, and writes each tile's
-//     offset rows (below); warp 13
-//     (one lane) issues the tcgen05.mma: S^T = K Q_i^T and dP^T = V dO_i^T
-//     into TMEM, then dV += P^T dO_i, dK += dS^T Q_i and the dQ partial
-//     dS K_j;
+//     offset rows (below); warp 13 issues the tcgen05.mma (the whole warp
+//     runs the loop and one elected lane issues): S^T = K Q_i^T and
+//     dP^T = V dO_i^T into TMEM, then dV += P^T dO_i, dK += dS^T Q_i and the
+//     dQ partial dS K_j;
 //   * the row terms of P = 2^(log2(e) (scale S - LSE)) and of dP - delta
 //     ride on the tensor core: S^T and dP^T take one more K = 16 slice, the
 //     product of a block of ones (keys) with a block holding -LSE/scale
@@ -333,47 +333,54 @@ struct BwdMma {
 
     // D[128 x 128] = A[128 x 64] B[128 x 64]^T + ones[128 x 16] aug[128 x 16]^T,
     // all K-major: the tile product plus each column's offset
-    __device__ __forceinline__ static void nt(uint32_t d, uint32_t a, uint32_t b, uint32_t ones, uint32_t aug) {
+    __device__ __forceinline__ static void nt(uint32_t d, uint32_t a, uint32_t b, uint32_t ones, uint32_t aug,
+                                              uint32_t issue) {
         const uint32_t a0 = sdesc_lo(a, 16), b0 = sdesc_lo(b, 16);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-            mma_ss_lo(d, a0 + ((kk * 32) >> 4), b0 + ((kk * 32) >> 4), kHi, kIdescNN, kk > 0 ? 1u : 0u);
-        mma_ss_lo(d, sdesc_lo(ones, 16), sdesc_lo(aug, 16), kHiAug, kIdescNN, 1u);
+            mma_ss_lo_w(d, a0 + ((kk * 32) >> 4), b0 + ((kk * 32) >> 4), kHi, kIdescNN, kk > 0 ? 1u : 0u,
+                        issue);
+        mma_ss_lo_w(d, sdesc_lo(ones, 16), sdesc_lo(aug, 16), kHiAug, kIdescNN, 1u, issue);
     }
     // D[128 x 64] (+)= A[128 x 128] B[128 x 64]: A K-major in two 64-column
     // halves, B M/N-major (rows = the 128-long K dimension)
-    __device__ __forceinline__ static void kt(uint32_t d, uint32_t a, uint32_t b, bool acc) {
+    __device__ __forceinline__ static void kt(uint32_t d, uint32_t a, uint32_t b, bool acc, uint32_t issue) {
         const uint32_t a0 = sdesc_lo(a, 16), b0 = sdesc_lo(b, kHalf);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ss_lo(d, a0 + (((kk / 4) * kHalf + (kk % 4) * 32) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi,
-                      kIdescKT, (acc || kk > 0) ? 1u : 0u);
+            mma_ss_lo_w(d, a0 + (((kk / 4) * kHalf + (kk % 4) * 32) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi,
+                        kIdescKT, (acc || kk > 0) ? 1u : 0u, issue);
     }
     // D[128 x 64] (+)= A[128 x 128] B[128 x 64]: A bf16 pairs in TMEM (P^T),
     // B M/N-major
-    __device__ __forceinline__ static void ts(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
+    __device__ __forceinline__ static void ts(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc, uint32_t issue) {
         const uint32_t b0 = sdesc_lo(b, kHalf);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ts_lo(d, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), kHi, kIdescKT, (acc || kk > 0) ? 1u : 0u);
+            mma_ts_lo_w(d, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), kHi, kIdescKT, (acc || kk > 0) ? 1u : 0u,
+                        issue);
     }
     // D[128 x 64] = A[128 x 128] B[128 x 64] with A stored transposed (the
     // dS^T tile: rows = K, two 64-wide halves of M), B M/N-major
-    __device__ __forceinline__ static void tt(uint32_t d, uint32_t a_t, uint32_t b) {
+    __device__ __forceinline__ static void tt(uint32_t d, uint32_t a_t, uint32_t b, uint32_t issue) {
         const uint32_t a0 = sdesc_lo(a_t, kHalf), b0 = sdesc_lo(b, kHalf);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ss_lo(d, a0 + ((kk * 16 * 128) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi, kIdescTT,
-                      kk > 0 ? 1u : 0u);
+            mma_ss_lo_w(d, a0 + ((kk * 16 * 128) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi, kIdescTT,
+                        kk > 0 ? 1u : 0u, issue);
     }
 };
 
+// The whole warp runs the issuing loop (warp-uniform control flow, so the
+// descriptors and counters stay on the uniform datapath); one elected lane
+// issues each tcgen05 instruction.  A single-lane loop costs ~8 % here.
 __device__ __forceinline__ void role_mma(const Ctx& c) {
     const BwdParams& p = c.p;
     const uint32_t t = c.tmem;
     bool ok = true;
+    const uint32_t issue = elect_lane();
     auto wait = [&](uint32_t bar, uint32_t parity) {
-        if (ok && !wait_b(c, bar, parity)) ok = false;
+        if (ok && !__all_sync(0xffffffffu, wait_b(c, bar, parity))) ok = false;
         return ok;
     };
     uint32_t g = 0;       // query tiles of this CTA so far
@@ -385,9 +392,9 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         if (!wait(c.bar + Bars::kReady + 8 * s, (gg / kStages) & 1)) return;
         tc_fence_after();
         const uint32_t aug = c.base + kOffAug + s * kAugBytes;
-        BwdMma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kTile, c.base + kOffOnes, aug);
-        BwdMma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kTile, c.base + kOffOnes, aug + 16);
-        tc_commit(c.bar + Bars::kSFull);
+        BwdMma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kTile, c.base + kOffOnes, aug, issue);
+        BwdMma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kTile, c.base + kOffOnes, aug + 16, issue);
+        tc_commit_w(c.bar + Bars::kSFull, issue);
     };
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
@@ -404,21 +411,21 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
             tc_fence_after();
             const uint32_t s = g % kStages;
             const uint32_t ds = c.base + kOffDS + (g & 1) * kDsBytes;
-            BwdMma::ts(t + kColDV, t + kColP, c.base + kOffDO + s * kTile, it > 0);  // dV += P^T dO
-            tc_commit(c.bar + Bars::kPTFree);
-            BwdMma::kt(t + kColDK, ds, c.base + kOffQ + s * kTile, it > 0);          // dK += dS^T Q
-            BwdMma::tt(t + kColDQ, ds, c.base + kOffK);                               // dQ_j = dS K
-            tc_commit(c.bar + Bars::kTileDone + 8 * s);
+            BwdMma::ts(t + kColDV, t + kColP, c.base + kOffDO + s * kTile, it > 0, issue);  // dV += P^T dO
+            tc_commit_w(c.bar + Bars::kPTFree, issue);
+            BwdMma::kt(t + kColDK, ds, c.base + kOffQ + s * kTile, it > 0, issue);  // dK += dS^T Q
+            BwdMma::tt(t + kColDQ, ds, c.base + kOffK, issue);                       // dQ_j = dS K
+            tc_commit_w(c.bar + Bars::kTileDone + 8 * s, issue);
             if (inext >= p.n_qt) {
-                tc_commit(c.bar + Bars::kDKVFull);
-                tc_commit(c.bar + Bars::kKVEmpty);
+                tc_commit_w(c.bar + Bars::kDKVFull, issue);
+                tc_commit_w(c.bar + Bars::kKVEmpty, issue);
             }
             i = inext;
         }
         ++units;
     }
     if (!ok) {
-        tc_commit(c.bar + Bars::kDrain);
+        tc_commit_w(c.bar + Bars::kDrain, issue);
         wait_bounded(c.bar + Bars::kDrain, 0, nullptr, kDrainNs);
     }
 }
@@ -516,7 +523,8 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
                         if (!key_ok || (diag && q < r)) x.x = 0.f;
                         if (!key_ok || (diag && q + 1 < r)) x.y = 0.f;
                     }
-                    const float2 dsv = __fmul2_rn(x, make_float2(__uint_as_float(dr[c4][e]), __uint_as_float(dr[c4][e + 1])));
+                    const float2 dsv =
+                        __fmul2_rn(x, make_float2(__uint_as_float(dr[c4][e]), __uint_as_float(dr[c4][e + 1])));
                     pk[e >> 1] = pack_bf16x2(x.x, x.y);
                     dk[e >> 1] = pack_bf16x2(dsv.x, dsv.y);
                 }
@@ -713,7 +721,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         regs_decrease<kOtherRegs>();
         if (warp == kLoadWarp) {
             role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do, lane);
-        } else if (warp == kMmaWarp && lane == 0) {
+        } else if (warp == kMmaWarp) {
             role_mma(ctx);
         }
         __syncwarp();
@@ -854,35 +862,38 @@ struct Mma {
     static constexpr uint32_t kIdescQ = idesc_bf16_f32(128, 64, true) | (1u << 15);     // dQ^T
     // D[128 x 64] = A[128 x 128] B[64 x 128]^T: A a K / V tile, B a Q / dO tile,
     // both K-major in two 64-column halves
-    __device__ __forceinline__ static void nt(uint32_t d, uint32_t a, uint32_t b) {
+    __device__ __forceinline__ static void nt(uint32_t d, uint32_t a, uint32_t b, uint32_t issue) {
         const uint32_t a0 = sdesc_lo(a, 16), b0 = sdesc_lo(b, 16);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-            mma_ss_lo(d, a0 + (((kk / 4) * kKHalf + (kk % 4) * 32) >> 4),
-                      b0 + (((kk / 4) * kQHalf + (kk % 4) * 32) >> 4), kHi, kIdescS, kk > 0 ? 1u : 0u);
+            mma_ss_lo_w(d, a0 + (((kk / 4) * kKHalf + (kk % 4) * 32) >> 4),
+                      b0 + (((kk / 4) * kQHalf + (kk % 4) * 32) >> 4), kHi, kIdescS, kk > 0 ? 1u : 0u, issue);
     }
     // dV (+)= P^T dO: A = P^T bf16 pairs in TMEM (K = 64 queries), B = the dO
     // tile M/N-major (N = 128 over two 64-column halves)
-    __device__ __forceinline__ static void pv(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
+    __device__ __forceinline__ static void pv(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc, uint32_t issue) {
         const uint32_t b0 = sdesc_lo(b, kQHalf);
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk)
-            mma_ts_lo(d, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), kHi, kIdescKV, (acc || kk > 0) ? 1u : 0u);
+            mma_ts_lo_w(d, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), kHi, kIdescKV, (acc || kk > 0) ? 1u : 0u,
+                        issue);
     }
     // dK (+)= dS^T Q: A = dS^T K-major (one 64-wide half), B = the Q tile M/N-major
-    __device__ __forceinline__ static void dsq(uint32_t d, uint32_t a, uint32_t b, bool acc) {
+    __device__ __forceinline__ static void dsq(uint32_t d, uint32_t a, uint32_t b, bool acc, uint32_t issue) {
         const uint32_t a0 = sdesc_lo(a, 16), b0 = sdesc_lo(b, kQHalf);
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk)
-            mma_ss_lo(d, a0 + ((kk * 32) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi, kIdescKV, (acc || kk > 0) ? 1u : 0u);
+            mma_ss_lo_w(d, a0 + ((kk * 32) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi, kIdescKV,
+                        (acc || kk > 0) ? 1u : 0u, issue);
     }
     // dQ^T = K^T dS^T: A = the K tile read M-major (M = 128 head columns over two
     // halves, K = 128 keys), B = dS^T M/N-major (N = 64 queries)
-    __device__ __forceinline__ static void kds(uint32_t d, uint32_t a, uint32_t b) {
+    __device__ __forceinline__ static void kds(uint32_t d, uint32_t a, uint32_t b, uint32_t issue) {
         const uint32_t a0 = sdesc_lo(a, kKHalf), b0 = sdesc_lo(b, kDsTile);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ss_lo(d, a0 + ((kk * 16 * 128) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi, kIdescQ, kk > 0 ? 1u : 0u);
+            mma_ss_lo_w(d, a0 + ((kk * 16 * 128) >> 4), b0 + ((kk * 16 * 128) >> 4), kHi, kIdescQ, kk > 0 ? 1u : 0u,
+                        issue);
     }
 };
 
@@ -890,8 +901,9 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
     const BwdParams& p = c.p;
     const uint32_t t = c.tmem;
     bool ok = true;
+    const uint32_t issue = elect_lane();
     auto wait = [&](uint32_t bar, uint32_t parity) {
-        if (ok && !wait_b(c, bar, parity)) ok = false;
+        if (ok && !__all_sync(0xffffffffu, wait_b(c, bar, parity))) ok = false;
         return ok;
     };
     uint32_t g = 0, units = 0;
@@ -900,9 +912,9 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         if (!wait(c.bar + Bars::kQFull + 8 * s, (gg >> 1) & 1)) return;
         if (gg > 0 && !wait(c.bar + Bars::kSFree, (gg - 1) & 1)) return;
         tc_fence_after();
-        Mma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kQTile);
-        Mma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kQTile);
-        tc_commit(c.bar + Bars::kSFull);
+        Mma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kQTile, issue);
+        Mma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kQTile, issue);
+        tc_commit_w(c.bar + Bars::kSFull, issue);
     };
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = unit(u, p);
@@ -917,25 +929,25 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
             if (it == 0 && !wait(c.bar + Bars::kDKVEmpty, (units & 1) ^ 1)) break;
             tc_fence_after();
             const uint32_t s = g & 1, ds = c.base + kOffDS + s * kDsTile;
-            Mma::pv(t + kColDV, t + kColP, c.base + kOffDO + s * kQTile, it > 0);   // dV += P^T dO
-            tc_commit(c.bar + Bars::kPTFree);
-            Mma::dsq(t + kColDK, ds, c.base + kOffQ + s * kQTile, it > 0);         // dK += dS^T Q
+            Mma::pv(t + kColDV, t + kColP, c.base + kOffDO + s * kQTile, it > 0, issue);   // dV += P^T dO
+            tc_commit_w(c.bar + Bars::kPTFree, issue);
+            Mma::dsq(t + kColDK, ds, c.base + kOffQ + s * kQTile, it > 0, issue);         // dK += dS^T Q
             if (!wait(c.bar + Bars::kDQEmpty, (g & 1) ^ 1)) break;
             tc_fence_after();
-            Mma::kds(t + kColDQ, c.base + kOffK, ds);                                // dQ^T = K^T dS^T
-            tc_commit(c.bar + Bars::kDsFree + 8 * s);
-            tc_commit(c.bar + Bars::kQEmpty + 8 * s);
-            tc_commit(c.bar + Bars::kDQFull);
+            Mma::kds(t + kColDQ, c.base + kOffK, ds, issue);                                // dQ^T = K^T dS^T
+            tc_commit_w(c.bar + Bars::kDsFree + 8 * s, issue);
+            tc_commit_w(c.bar + Bars::kQEmpty + 8 * s, issue);
+            tc_commit_w(c.bar + Bars::kDQFull, issue);
             if (inext >= p.n_qt) {
-                tc_commit(c.bar + Bars::kDKVFull);
-                tc_commit(c.bar + Bars::kKVEmpty);
+                tc_commit_w(c.bar + Bars::kDKVFull, issue);
+                tc_commit_w(c.bar + Bars::kKVEmpty, issue);
             }
             i = inext;
         }
         ++units;
     }
     if (!ok) {
-        tc_commit(c.bar + Bars::kDrain);
+        tc_commit_w(c.bar + Bars::kDrain, issue);
         wait_bounded(c.bar + Bars::kDrain, 0, nullptr, kDrainNs);
     }
 }
@@ -1221,9 +1233,10 @@ kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         b128::role_dq(ctx, warp, lane);
     } else {
         regs_decrease<kOtherRegs>();
-        if (lane == 0) {
-            if (warp == kLoadWarp) b128::role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do);
-            else if (warp == kMmaWarp) b128::role_mma(ctx);
+        if (warp == kLoadWarp) {
+            if (lane == 0) b128::role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do);
+        } else if (warp == kMmaWarp) {
+            b128::role_mma(ctx);
         }
         __syncwarp();
     }
