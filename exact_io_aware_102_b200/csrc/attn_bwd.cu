@@ -17,32 +17,33 @@
 //   * the main kernel runs a persistent grid, one CTA per SM; a work unit is
 //     one (batch, head, 128-key block).  dK and dV of the block accumulate in
 //     TMEM over the query tiles (128 rows each) the block interacts with;
-//   * warp 12 loads K, V once per unit and Q_i, dO_i per query tile (three
-//     stages at d = 64, two at d = 128) by TMA, and writes each tile's
-//     offset rows (below); warp 13 issues the tcgen05.mma (the whole warp
-//     runs the loop and one elected lane issues): S^T = K Q_i^T and
-//     dP^T = V dO_i^T into TMEM, then dV += P^T dO_i, dK += dS^T Q_i and the
-//     dQ partial dS K_j;
+//   (warp numbers for d = 64; the d = 128 kernel below has its own layout)
+//   * warp 20 loads K, V once per unit and Q_i, dO_i per query tile (three
+//     stages) by TMA, and writes each tile's offset rows (below); warp 21
+//     issues the tcgen05.mma (the whole warp runs the loop and one elected
+//     lane issues): S^T = K Q_i^T and dP^T = V dO_i^T into TMEM, then
+//     dV += P^T dO_i, dK += dS^T Q_i and the dQ partial dS K_j;
 //   * the row terms of P = 2^(log2(e) (scale S - LSE)) and of dP - delta
 //     ride on the tensor core: S^T and dP^T take one more K = 16 slice, the
 //     product of a block of ones (keys) with a block holding -LSE/scale
 //     (resp. -delta) of each query row, split into three bf16 parts
 //     (c = h1 + h2 + h3 to 2^-24 |c|), so the accumulators hold S - LSE/scale
 //     and dP - delta and the elementwise warps need no per-column values;
-//   * warps 0-7 (two threads per key row: warps 0-3 query columns 0-63, warps
-//     4-7 columns 64-127, so each SM sub-partition runs two of them) turn the
-//     S^T, dP^T rows into P^T (bf16, into TMEM: the A operand of dV) and dS^T
+//   * warps 0-15 (four threads per key row: warp w takes query columns
+//     32 (w / 4) .. 32 (w / 4) + 31, so each SM sub-partition runs four of
+//     them, which hide one another's latency) turn the S^T, dP^T rows into
+//     P^T (bf16, into TMEM: the A operand of dV) and dS^T
 //     (bf16, into one of two shared-memory buffers in the 128-byte-swizzled
 //     layout the tensor core reads -- one dS^T tile serves dK (K-major) and,
 //     read transposed, dQ (M-major)).  A tile's P^T and dS^T only wait for
 //     dV of the previous tile, so the products of tile i overlap the
 //     elementwise work of tile i+1;
-//   * warps 8-11 (one thread per query row) read the dQ partial from TMEM and
+//   * warps 16-19 (one thread per query row) read the dQ partial from TMEM and
 //     add it to the fp32 dQ accumulator in global memory with tensor
 //     reductions (cp.reduce.async.bulk.tensor .add), two [32 x 32] boxes per
 //     warp through one staging box;
-//   * at the end of a unit warps 0-3 write dV and warps 4-7 dK (times scale)
-//     in bf16.
+//   * at the end of a unit warps 0-7 write dV and warps 8-15 dK (times
+//     scale) in bf16, 32 columns each.
 //   Every wait is bounded (see sm100_ptx.cuh) and no barrier spans warps
 //   other than mbarriers, so a timeout never leaves a thread blocked.
 //
@@ -67,18 +68,20 @@ namespace {
 constexpr int kD = 64;            // head size handled here
 constexpr int kBK = 128;          // keys per unit (= TMEM lanes)
 constexpr int kBQ = 128;          // query rows per tile
-constexpr int kThreads = 512;     // warps 0-7 P/dS, 8-11 dQ, 12 load, 13 MMA, 14-15 idle
-// Register split (setmaxnreg): the block launches with 512 x 128 registers;
-// the two P/dS warpgroups take 176 each, the dQ and load/MMA warpgroups keep
-// 80 (256 x 176 + 256 x 80 = 512 x 128).
-constexpr int kPdsRegs = 176;
-constexpr int kOtherRegs = 80;
-static_assert(256 * kPdsRegs + 256 * kOtherRegs == kThreads * 128, "setmaxnreg split must equal the launch budget");
-constexpr int kPdsWarps = 8;      // two per SM sub-partition: query columns 0-63 and 64-127
+// Warps: 0-15 P/dS (four per SM sub-partition, 32 query columns each),
+// 16-19 dQ, 20 load, 21 MMA, 22-23 idle.  Register split (setmaxnreg): the
+// block launches with 768 x 80 registers; the four P/dS warpgroups take 88,
+// the dQ warpgroup keeps 80, the load / MMA warpgroup gives back to 48
+// (512 x 88 + 128 x 80 + 128 x 48 = 768 x 80).
+constexpr int kThreads = 768;
+constexpr int kPdsWarps = 16;
 constexpr int kPdsThreads = kPdsWarps * 32;
-constexpr int kDqWarp0 = 8;
-constexpr int kLoadWarp = 12;
-constexpr int kMmaWarp = 13;
+constexpr int kDqWarp0 = 16;
+constexpr int kLoadWarp = 20;
+constexpr int kMmaWarp = 21;
+constexpr int kPdsRegs = 88, kCtlRegs = 48, kLaunchRegs = 80;
+static_assert(kPdsThreads * kPdsRegs + 128 * kLaunchRegs + 128 * kCtlRegs == kThreads * kLaunchRegs,
+              "setmaxnreg split must equal the launch budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384, kColP = 448;
 constexpr float kLog2eB = 1.4426950408889634f;
@@ -448,17 +451,20 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
     return v;
 }
 
-// ---------------------------------------------------------- P / dS warps (0-7)
-// Thread = key row r of the unit's block (TMEM lane r) and one half of the
-// 128 query columns of a tile.
+// ---------------------------------------------------------- P / dS warps (0-15)
+// Thread = key row r of the unit's block (TMEM lane r) and one quarter (32
+// columns) of the 128 query columns of a tile.
 __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
     const BwdParams& p = c.p;
-    const int quarter = warp & 3, half = warp >> 2;
+    const int quarter = warp & 3, part = warp >> 2;
     const int r = quarter * 32 + lane;
-    const int col0 = half * 64;  // first query column of this thread
+    const int col0 = part * 32;  // first query column of this thread
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t t_s = c.tmem + lane_off + kColS + col0, t_dp = c.tmem + lane_off + kColDP + col0;
-    const uint32_t t_acc = c.tmem + lane_off + (half == 0 ? kColDV : kColDK);
+    // unit epilogue: 32 columns of dV (parts 0, 1) or dK (parts 2, 3)
+    const uint32_t t_acc = c.tmem + lane_off + (part < 2 ? kColDV : kColDK) + (part & 1) * 32;
+    uint16_t* const acc_out = part < 2 ? p.dv : p.dk;
+    const int acc_col = (part & 1) * 32;
     const uint32_t t_p = c.tmem + lane_off + kColP + col0 / 2;  // bf16 pairs
     const float sl2 = p.scale_log2;
     uint32_t g = 0, units = 0;
@@ -472,10 +478,10 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
         if (i >= p.n_qt) {
             // no query tile meets this key block: its dK and dV rows are zero
             if (key < p.N) {
-                uint4* dst = reinterpret_cast<uint4*>((half == 0 ? p.dv : p.dk) +
-                                                      (static_cast<size_t>(w.bh) * p.N + key) * kD);
+                uint4* dst =
+                    reinterpret_cast<uint4*>(acc_out + (static_cast<size_t>(w.bh) * p.N + key) * kD + acc_col);
 #pragma unroll
-                for (int v4 = 0; v4 < kD / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+                for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
             }
             continue;
         }
@@ -496,63 +502,54 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             // and dP^T - delta, then release them at once: the next tile's
             // products start now (rows past N, or without any visible key,
             // carry the lowest offset and give P = dS = 0)
-            uint32_t sr[2][32], dr[2][32];
-            tmem_ld32(t_s, sr[0]);
-            tmem_ld32(t_s + 32, sr[1]);
-            tmem_ld32(t_dp, dr[0]);
-            tmem_ld32(t_dp + 32, dr[1]);
+            uint32_t sr[32], dr[32];
+            tmem_ld32(t_s, sr);
+            tmem_ld32(t_dp, dr);
             tmem_wait_ld();
-            reg_fence32(sr[0]);
-            reg_fence32(sr[1]);
-            reg_fence32(dr[0]);
-            reg_fence32(dr[1]);
+            reg_fence32(sr);
+            reg_fence32(dr);
             tc_fence_before();
             mbar_arrive(c.bar + Bars::kReady + 8 * ((g + 1) % kStages));  // S^T / dP^T may be overwritten
+            uint32_t pk[16], dk[16];
+            const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
-            for (int c4 = 0; c4 < 2; ++c4) {
-                uint32_t pk[16], dk[16];
-                const float2 sl2x2 = make_float2(sl2, sl2);
+            for (int e = 0; e < 32; e += 2) {
+                float2 x = __fmul2_rn(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sl2x2);
+                x.x = ex2(x.x);
+                x.y = ex2(x.y);
+                if (masked) {
+                    const int q = col0 + e;
+                    if (!key_ok || (diag && q < r)) x.x = 0.f;
+                    if (!key_ok || (diag && q + 1 < r)) x.y = 0.f;
+                }
+                const float2 dsv = __fmul2_rn(x, make_float2(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])));
+                pk[e >> 1] = pack_bf16x2(x.x, x.y);
+                dk[e >> 1] = pack_bf16x2(dsv.x, dsv.y);
+            }
+            if (g > 0) {
+                // P^T's TMEM columns: dV of the previous tile must have retired
+                bool free = wait_b(c, c.bar + Bars::kPTFree, (g - 1) & 1);
+                free = __all_sync(0xffffffffu, free);
+                if (!free) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            if (g > 1) {
+                // this dS^T buffer: dK and dQ of tile g-2 must have retired
+                bool free = wait_b(c, c.bar + Bars::kTileDone + 8 * ((g - 2) % kStages), ((g - 2) / kStages) & 1);
+                free = __all_sync(0xffffffffu, free);
+                if (!free) {
+                    ok = false;
+                    break;
+                }
+            }
+            tmem_st16(t_p, pk);
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float2 x = __fmul2_rn(make_float2(__uint_as_float(sr[c4][e]), __uint_as_float(sr[c4][e + 1])),
-                                          sl2x2);
-                    x.x = ex2(x.x);
-                    x.y = ex2(x.y);
-                    if (masked) {
-                        const int q = col0 + c4 * 32 + e;
-                        if (!key_ok || (diag && q < r)) x.x = 0.f;
-                        if (!key_ok || (diag && q + 1 < r)) x.y = 0.f;
-                    }
-                    const float2 dsv =
-                        __fmul2_rn(x, make_float2(__uint_as_float(dr[c4][e]), __uint_as_float(dr[c4][e + 1])));
-                    pk[e >> 1] = pack_bf16x2(x.x, x.y);
-                    dk[e >> 1] = pack_bf16x2(dsv.x, dsv.y);
-                }
-                if (c4 == 0 && g > 0) {
-                    // P^T's TMEM columns: dV of the previous tile must have retired
-                    bool free = wait_b(c, c.bar + Bars::kPTFree, (g - 1) & 1);
-                    free = __all_sync(0xffffffffu, free);
-                    if (!free) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                }
-                if (c4 == 0 && g > 1) {
-                    // this dS^T buffer: dK and dQ of tile g-2 must have retired
-                    bool free = wait_b(c, c.bar + Bars::kTileDone + 8 * ((g - 2) % kStages), ((g - 2) / kStages) & 1);
-                    free = __all_sync(0xffffffffu, free);
-                    if (!free) {
-                        ok = false;
-                        break;
-                    }
-                }
-                tmem_st16(t_p + c4 * 16, pk);
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    const uint32_t off = sw128_off(r, col0 + c4 * 32 + q8 * 8);
-                    st_shared_v4(ds_buf + off, dk[q8 * 4], dk[q8 * 4 + 1], dk[q8 * 4 + 2], dk[q8 * 4 + 3]);
-                }
+            for (int q8 = 0; q8 < 4; ++q8) {
+                const uint32_t off = sw128_off(r, col0 + q8 * 8);
+                st_shared_v4(ds_buf + off, dk[q8 * 4], dk[q8 * 4 + 1], dk[q8 * 4 + 2], dk[q8 * 4 + 3]);
             }
             if (!ok) break;
             tmem_wait_st();
@@ -562,7 +559,8 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             i = inext;
         }
         if (!ok) break;
-        // unit epilogue: dV (warps 0-3) or dK times scale (warps 4-7) of this key row
+        // unit epilogue: 32 columns of dV (warps 0-7) or dK times scale
+        // (warps 8-15) of this key row
         bool got = wait_b(c, c.bar + Bars::kDKVFull, units & 1);
         got = __all_sync(0xffffffffu, got);
         if (!got) {
@@ -571,35 +569,30 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
         }
         ++units;
         tc_fence_after();
-        uint32_t a[2][32];
-        tmem_ld32(t_acc, a[0]);
-        tmem_ld32(t_acc + 32, a[1]);
+        uint32_t acc[32];
+        tmem_ld32(t_acc, acc);
         tmem_wait_ld();
-        reg_fence32(a[0]);
-        reg_fence32(a[1]);
+        reg_fence32(acc);
         tc_fence_before();
         mbar_arrive(c.bar + Bars::kDKVEmpty);
         if (key < p.N) {  // padded keys store their (zero) rows too
-            const float f = half == 0 ? 1.f : p.scale;
-            uint4* dst = reinterpret_cast<uint4*>((half == 0 ? p.dv : p.dk) +
-                                                  (static_cast<size_t>(w.bh) * p.N + key) * kD);
+            const float f = part < 2 ? 1.f : p.scale;
+            uint4* dst = reinterpret_cast<uint4*>(acc_out + (static_cast<size_t>(w.bh) * p.N + key) * kD + acc_col);
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int v4 = 0; v4 < 4; ++v4) {
+                uint32_t x[4];
 #pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4) {
-                    uint32_t x[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int cc = v4 * 8 + e * 2;
-                        x[e] = pack_bf16x2(__uint_as_float(a[h][cc]) * f, __uint_as_float(a[h][cc + 1]) * f);
-                    }
-                    dst[h * 4 + v4] = make_uint4(x[0], x[1], x[2], x[3]);
+                for (int e = 0; e < 4; ++e) {
+                    const int cc = v4 * 8 + e * 2;
+                    x[e] = pack_bf16x2(__uint_as_float(acc[cc]) * f, __uint_as_float(acc[cc + 1]) * f);
                 }
+                dst[v4] = make_uint4(x[0], x[1], x[2], x[3]);
+            }
         }
     }
 }
 
-// ------------------------------------------------------------- dQ warps (8-11)
+// ------------------------------------------------------------ dQ warps (16-19)
 // Thread = query row of the tile = TMEM lane.  Each warp reads its 32 rows
 // (64 columns) from TMEM, releases the accumulator, and adds them to dQ as
 // two [32 x 32] fp32 boxes, one after the other through one 128-byte-
@@ -714,11 +707,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_arrive(bar + Bars::kReady);  // tile 0 has no earlier S^T to read
         role_pds(ctx, warp, lane);
     } else if (warp < kDqWarp0 + 4) {
-        regs_decrease<kOtherRegs>();
         mbar_arrive(bar + Bars::kPFull);  // tile 0 has no earlier dQ partial
         role_dq(ctx, &tm_dq, warp, lane);
     } else {
-        regs_decrease<kOtherRegs>();
+        regs_decrease<kCtlRegs>();
         if (warp == kLoadWarp) {
             role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do, lane);
         } else if (warp == kMmaWarp) {
@@ -771,6 +763,18 @@ __global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint1
 // bulk reduction (32 KB, contiguous in dQ) adds to the accumulator.
 namespace b128 {
 
+constexpr int kThreads = 512;     // warps 0-7 P/dS, 8-11 dQ, 12 load, 13 MMA, 14-15 idle
+// Register split (setmaxnreg): the block launches with 512 x 128 registers;
+// the two P/dS warpgroups take 176 each, the dQ and load/MMA warpgroups keep
+// 80 (256 x 176 + 256 x 80 = 512 x 128).
+constexpr int kPdsRegs = 176;
+constexpr int kOtherRegs = 80;
+static_assert(256 * kPdsRegs + 256 * kOtherRegs == kThreads * 128, "setmaxnreg split must equal the launch budget");
+constexpr int kPdsWarps = 8;      // two per SM sub-partition: query columns 0-31 and 32-63
+constexpr int kPdsThreads = kPdsWarps * 32;
+constexpr int kDqWarp0 = 8;
+constexpr int kLoadWarp = 12;
+constexpr int kMmaWarp = 13;
 constexpr int kD = 128;
 constexpr int kBQ = 64;                     // query rows per tile
 constexpr uint32_t kColS = 0, kColDP = 64, kColDV = 128, kColDK = 256, kColDQ = 384, kColP = 448;
@@ -1498,7 +1502,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
         attn_bwd_prep_kernel<128><<<prep_grid, 256, 0, s>>>(o16, do16, delta, dq, static_cast<long long>(rows));
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     const int grid = static_cast<int>(units < sms ? units : sms);
-    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mdo, mdq, p);
+    kern<<<grid, d == 64 ? kThreads : b128::kThreads, smem, s>>>(mq, mk, mv, mdo, mdq, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
