@@ -37,10 +37,10 @@ RMS_TOL = 1e-2
 ABS_FLOOR = 1e-5
 
 
-def run_bwd(B, H, N, causal, seed=0, scale=None, d=64):
+def run_bwd(B, H, N, causal, seed=0, scale=None, d=64, q_mult=1.0):
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dev = torch.device("cuda:0")
-    q, k, v = make_qkv(B, H, N, d, seed=seed)
+    q, k, v = make_qkv(B, H, N, d, seed=seed, q_mult=q_mult)
     do = make_dout(B, H, N, d, seed=seed + 100)
     qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
     o, lse = pkg.forward(qd, kd, vd, scale=scale, causal=causal)
@@ -62,8 +62,8 @@ def compare(got, ref, what):
     return err / max(np.abs(ref).max(), 1e-30)
 
 
-def check_full(B, H, N, causal, seed=0, d=64):
-    ins, (dq, dk, dv), scale = run_bwd(B, H, N, causal, seed, d=d)
+def check_full(B, H, N, causal, seed=0, d=64, scale=None, q_mult=1.0):
+    ins, (dq, dk, dv), scale = run_bwd(B, H, N, causal, seed, scale=scale, d=d, q_mult=q_mult)
     rq, rk, rv = oracle.attention_bwd_rows(*ins, scale, causal)
     shape = (B, H, N, d)
     return [compare(g, r.reshape(shape), n) for g, r, n in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV"))]
@@ -73,6 +73,16 @@ def check_full(B, H, N, causal, seed=0, d=64):
 @pytest.mark.parametrize("N", [1, 2, 17, 127, 128, 129, 255, 256, 300, 700])
 def test_bwd_small_sizes_full(N, causal):
     check_full(1, 2, N, causal, seed=N)
+
+
+# P's row term -LSE/scale and dS's -delta reach the kernel as three bf16 parts
+# added on the tensor core: a small scale makes -LSE/scale large (about 6e3
+# at 1e-3), scale 1 or a 4x Q makes the scores wide and P nearly one-hot
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("scale,q_mult", [(1e-3, 1.0), (1.0, 1.0), (0.125, 4.0)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_bwd_scale_and_logit_range_full(scale, q_mult, causal, d):
+    check_full(1, 2, 333, causal, seed=21, d=d, scale=scale, q_mult=q_mult)
 
 
 def test_bwd_many_heads_and_batches_full():
