@@ -19,10 +19,11 @@
 //     TMEM over the query tiles (128 rows each) the block interacts with;
 //   (warp numbers for d = 64; the d = 128 kernel below has its own layout)
 //   * warp 20 loads K, V once per unit and Q_i, dO_i per query tile (three
-//     stages) by TMA, and writes each tile's offset rows (below); warp 21
-//     issues the tcgen05.mma (the whole warp runs the loop and one elected
-//     lane issues): S^T = K Q_i^T and dP^T = V dO_i^T into TMEM, then
-//     dV += P^T dO_i, dK += dS^T Q_i and the dQ partial dS K_j;
+//     stages) by TMA, and writes each tile's offset rows (below); warps 21
+//     and 22 issue the tcgen05.mma (each runs its loop with the whole warp,
+//     one elected lane issuing): warp 21 S^T = K Q_i^T and dP^T = V dO_i^T
+//     into TMEM, warp 22 dV += P^T dO_i, dK += dS^T Q_i and the dQ partial
+//     dS K_j;
 //   * the row terms of P = 2^(log2(e) (scale S - LSE)) and of dP - delta
 //     ride on the tensor core: S^T and dP^T take one more K = 16 slice, the
 //     product of a block of ones (keys) with a block holding -LSE/scale
@@ -69,7 +70,7 @@ constexpr int kD = 64;            // head size handled here
 constexpr int kBK = 128;          // keys per unit (= TMEM lanes)
 constexpr int kBQ = 128;          // query rows per tile
 // Warps: 0-15 P/dS (four per SM sub-partition, 32 query columns each),
-// 16-19 dQ, 20 load, 21 MMA, 22-23 idle.  Register split (setmaxnreg): the
+// 16-19 dQ, 20 load, 21-22 MMA (S^T / dP^T; dV, dK, dQ), 23 idle.  Register split (setmaxnreg): the
 // block launches with 768 x 80 registers; the four P/dS warpgroups take 88,
 // the dQ warpgroup keeps 80, the load / MMA warpgroup gives back to 48
 // (512 x 88 + 128 x 80 + 128 x 48 = 768 x 80).
@@ -129,6 +130,7 @@ struct Bars {
     static constexpr int kDKVFull = 88, kDKVEmpty = 96;
     static constexpr int kDrain = 104;
     static constexpr int kTmemSlot = 112, kAbort = 116;
+    static constexpr int kDrain2 = 120;  // the second issuing warp's drain
 };
 static_assert(Bars::kReady + 8 * kStages <= Bars::kTileDone && Bars::kTileDone + 8 * kStages <= Bars::kSFull,
               "barrier map");
@@ -374,10 +376,17 @@ struct BwdMma {
     }
 };
 
-// The whole warp runs the issuing loop (warp-uniform control flow, so the
-// descriptors and counters stay on the uniform datapath); one elected lane
-// issues each tcgen05 instruction.  A single-lane loop costs ~8 % here.
-__device__ __forceinline__ void role_mma(const Ctx& c) {
+// Two issuing warps, each running its loop with the whole warp (warp-uniform
+// control flow keeps descriptors and counters on the uniform datapath) and one
+// elected lane issuing: warp 21 the S^T / dP^T products, warp 22 dV, dK, dQ.
+// Either warp's waits, commits and loop overhead then overlap the other's
+// products in the shallow tensor instruction queue.  They touch disjoint TMEM
+// columns; every cross-stream order goes through the P/dS warps (tile g's
+// products need P of tile g, which needs S of tile g).
+
+// S^T - LSE/scale and dP^T - delta of each tile into TMEM, once its inputs
+// have landed and the P/dS warps have read the previous tile's.
+__device__ __forceinline__ void role_mma_s(const Ctx& c) {
     const BwdParams& p = c.p;
     const uint32_t t = c.tmem;
     bool ok = true;
@@ -386,28 +395,49 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         if (ok && !__all_sync(0xffffffffu, wait_b(c, bar, parity))) ok = false;
         return ok;
     };
-    uint32_t g = 0;       // query tiles of this CTA so far
-    uint32_t units = 0;
-    // S^T - LSE/scale and dP^T - delta of tile g into TMEM, once its inputs
-    // have landed and the P/dS warps have read tile g-1's
-    auto issue_s = [&](uint32_t gg) {
-        const uint32_t s = gg % kStages;
-        if (!wait(c.bar + Bars::kReady + 8 * s, (gg / kStages) & 1)) return;
-        tc_fence_after();
-        const uint32_t aug = c.base + kOffAug + s * kAugBytes;
-        BwdMma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kTile, c.base + kOffOnes, aug, issue);
-        BwdMma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kTile, c.base + kOffOnes, aug + 16, issue);
-        tc_commit_w(c.bar + Bars::kSFull, issue);
-    };
+    uint32_t g = 0, units = 0;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
         const BwdUnit w = bwd_unit(u, p);
         int i = next_tile(p, w, w.i0, kBQ);
         if (i >= p.n_qt) continue;  // no query tile meets this key block
         if (!wait(c.bar + Bars::kKVFull, units & 1)) break;
-        issue_s(g);
+        for (; ok && i < p.n_qt; i = next_tile(p, w, i + 1, kBQ), ++g) {
+            const uint32_t s = g % kStages;
+            if (!wait(c.bar + Bars::kReady + 8 * s, (g / kStages) & 1)) break;
+            tc_fence_after();
+            const uint32_t aug = c.base + kOffAug + s * kAugBytes;
+            BwdMma::nt(t + kColS, c.base + kOffK, c.base + kOffQ + s * kTile, c.base + kOffOnes, aug, issue);
+            BwdMma::nt(t + kColDP, c.base + kOffV, c.base + kOffDO + s * kTile, c.base + kOffOnes, aug + 16,
+                       issue);
+            tc_commit_w(c.bar + Bars::kSFull, issue);
+        }
+        ++units;
+    }
+    if (!ok) {
+        tc_commit_w(c.bar + Bars::kDrain, issue);
+        wait_bounded(c.bar + Bars::kDrain, 0, nullptr, kDrainNs);
+    }
+}
+
+// dV += P^T dO, dK += dS^T Q and the dQ partial dS K of each tile once the
+// P/dS warps have written P^T and dS^T (and the dQ warps read the previous
+// partial).
+__device__ __forceinline__ void role_mma_d(const Ctx& c) {
+    const BwdParams& p = c.p;
+    const uint32_t t = c.tmem;
+    bool ok = true;
+    const uint32_t issue = elect_lane();
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+        if (ok && !__all_sync(0xffffffffu, wait_b(c, bar, parity))) ok = false;
+        return ok;
+    };
+    uint32_t g = 0, units = 0;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        const BwdUnit w = bwd_unit(u, p);
+        int i = next_tile(p, w, w.i0, kBQ);
+        if (i >= p.n_qt) continue;
         for (int it = 0; ok && i < p.n_qt; ++it, ++g) {
             const int inext = next_tile(p, w, i + 1, kBQ);
-            if (inext < p.n_qt) issue_s(g + 1);  // overlaps the P/dS work of tile g
             // P^T, dS^T of tile g written and the dQ partial of tile g-1 read
             if (!wait(c.bar + Bars::kPFull, g & 1)) break;
             if (it == 0 && !wait(c.bar + Bars::kDKVEmpty, (units & 1) ^ 1)) break;
@@ -418,6 +448,7 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
             tc_commit_w(c.bar + Bars::kPTFree, issue);
             BwdMma::kt(t + kColDK, ds, c.base + kOffQ + s * kTile, it > 0, issue);  // dK += dS^T Q
             BwdMma::tt(t + kColDQ, ds, c.base + kOffK, issue);                       // dQ_j = dS K
+            // the stage's last reads (S^T, dP^T of tile g retired before its P existed)
             tc_commit_w(c.bar + Bars::kTileDone + 8 * s, issue);
             if (inext >= p.n_qt) {
                 tc_commit_w(c.bar + Bars::kDKVFull, issue);
@@ -428,8 +459,8 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         ++units;
     }
     if (!ok) {
-        tc_commit_w(c.bar + Bars::kDrain, issue);
-        wait_bounded(c.bar + Bars::kDrain, 0, nullptr, kDrainNs);
+        tc_commit_w(c.bar + Bars::kDrain2, issue);
+        wait_bounded(c.bar + Bars::kDrain2, 0, nullptr, kDrainNs);
     }
 }
 
@@ -682,6 +713,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar + Bars::kDKVFull, 1);
         mbar_init(bar + Bars::kDKVEmpty, kPdsThreads);
         mbar_init(bar + Bars::kDrain, 1);
+        mbar_init(bar + Bars::kDrain2, 1);
         *abort_flag = 0u;
         fence_barrier_init();
         fence_proxy_async();
@@ -714,7 +746,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (warp == kLoadWarp) {
             role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do, lane);
         } else if (warp == kMmaWarp) {
-            role_mma(ctx);
+            role_mma_s(ctx);
+        } else if (warp == kMmaWarp + 1) {
+            role_mma_d(ctx);
         }
         __syncwarp();
     }
