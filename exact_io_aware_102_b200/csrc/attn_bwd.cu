@@ -797,7 +797,7 @@ __global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint1
 // bulk reduction (32 KB, contiguous in dQ) adds to the accumulator.
 namespace b128 {
 
-constexpr int kThreads = 512;     // warps 0-7 P/dS, 8-11 dQ, 12 load, 13 MMA, 14-15 idle
+constexpr int kThreads = 512;     // warps 0-7 P/dS, 8-11 dQ, 12 load, 13-14 MMA, 15 idle
 // Register split (setmaxnreg): the block launches with 512 x 128 registers;
 // the two P/dS warpgroups take 176 each, the dQ and load/MMA warpgroups keep
 // 80 (256 x 176 + 256 x 80 = 512 x 128).
@@ -842,6 +842,7 @@ struct Bars {
     static constexpr int kStageFull = 136;           // 128 dQ threads wrote the staging tile
     static constexpr int kStageFree = 144;           // its bulk reduction has read it
     static constexpr int kTmemSlot = 152, kAbort = 156;
+    static constexpr int kDrain2 = 160;
 };
 
 // Causal: key block kb (keys 128 kb ..) meets 64-row query tiles 2 kb ..
@@ -935,7 +936,8 @@ struct Mma {
     }
 };
 
-__device__ __forceinline__ void role_mma(const Ctx& c) {
+// Two issuing warps, as at d = 64: warp 13 S^T / dP^T, warp 14 dV, dK, dQ^T.
+__device__ __forceinline__ void role_mma_s(const Ctx& c) {
     const BwdParams& p = c.p;
     const uint32_t t = c.tmem;
     bool ok = true;
@@ -959,10 +961,31 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         int i = next_tile(p, w, w.i0, kBQ);
         if (i >= p.n_qt) continue;  // no query tile meets this key block
         if (!wait(c.bar + Bars::kKVFull, units & 1)) break;
-        issue_s(g);
+        for (; ok && i < p.n_qt; i = next_tile(p, w, i + 1, kBQ), ++g) issue_s(g);
+        ++units;
+    }
+    if (!ok) {
+        tc_commit_w(c.bar + Bars::kDrain, issue);
+        wait_bounded(c.bar + Bars::kDrain, 0, nullptr, kDrainNs);
+    }
+}
+
+__device__ __forceinline__ void role_mma_d(const Ctx& c) {
+    const BwdParams& p = c.p;
+    const uint32_t t = c.tmem;
+    bool ok = true;
+    const uint32_t issue = elect_lane();
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+        if (ok && !__all_sync(0xffffffffu, wait_b(c, bar, parity))) ok = false;
+        return ok;
+    };
+    uint32_t g = 0, units = 0;
+    for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        const BwdUnit w = unit(u, p);
+        int i = next_tile(p, w, w.i0, kBQ);
+        if (i >= p.n_qt) continue;  // no query tile meets this key block
         for (int it = 0; ok && i < p.n_qt; ++it, ++g) {
             const int inext = next_tile(p, w, i + 1, kBQ);
-            if (inext < p.n_qt) issue_s(g + 1);
             if (!wait(c.bar + Bars::kPFull, g & 1)) break;
             if (it == 0 && !wait(c.bar + Bars::kDKVEmpty, (units & 1) ^ 1)) break;
             tc_fence_after();
@@ -985,8 +1008,8 @@ __device__ __forceinline__ void role_mma(const Ctx& c) {
         ++units;
     }
     if (!ok) {
-        tc_commit_w(c.bar + Bars::kDrain, issue);
-        wait_bounded(c.bar + Bars::kDrain, 0, nullptr, kDrainNs);
+        tc_commit_w(c.bar + Bars::kDrain2, issue);
+        wait_bounded(c.bar + Bars::kDrain2, 0, nullptr, kDrainNs);
     }
 }
 
@@ -1243,6 +1266,7 @@ kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         mbar_init(bar + Bars::kDKVFull, 1);
         mbar_init(bar + Bars::kDKVEmpty, kPdsThreads);
         mbar_init(bar + Bars::kDrain, 1);
+        mbar_init(bar + Bars::kDrain2, 1);
         mbar_init(bar + Bars::kStageFull, 128);
         mbar_init(bar + Bars::kStageFree, 1);
         *abort_flag = 0u;
@@ -1274,7 +1298,9 @@ kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         if (warp == kLoadWarp) {
             if (lane == 0) b128::role_load(ctx, &tm_q, &tm_k, &tm_v, &tm_do);
         } else if (warp == kMmaWarp) {
-            b128::role_mma(ctx);
+            b128::role_mma_s(ctx);
+        } else if (warp == kMmaWarp + 1) {
+            b128::role_mma_d(ctx);
         }
         __syncwarp();
     }
