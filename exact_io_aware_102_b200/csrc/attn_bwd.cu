@@ -529,10 +529,10 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
             // a warp-uniform fast path when no element of the warp's rows is masked
             const bool masked = __any_sync(0xffffffffu, !key_ok || diag);
             const uint32_t ds_buf = c.base + kOffDS + (g & 1) * kDsBytes;
-            // both 32-column chunks of this thread's row of S^T - LSE/scale
-            // and dP^T - delta, then release them at once: the next tile's
-            // products start now (rows past N, or without any visible key,
-            // carry the lowest offset and give P = dS = 0)
+            // this thread's 32 columns of S^T - LSE/scale and dP^T - delta,
+            // then release them: the next tile's products start now (rows
+            // past N, or without any visible key, carry the lowest offset
+            // and give P = dS = 0)
             uint32_t sr[32], dr[32];
             tmem_ld32(t_s, sr);
             tmem_ld32(t_dp, dr);
