@@ -606,9 +606,15 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
         reg_fence32(acc);
         tc_fence_before();
         mbar_arrive(c.bar + Bars::kDKVEmpty);
-        if (key < p.N) {  // padded keys store their (zero) rows too
+        // The warp's 32 rows x 32 columns go out through its own 2 KB of a
+        // dS^T buffer (the same bytes it writes dS^T to; free between units:
+        // the unit's products have retired and this warp's next dS^T comes
+        // later), so that a store covers 64-byte row segments of 8 rows
+        // instead of 32 scattered 16-byte pieces.  Padded keys store their
+        // (zero) rows too.
+        {
             const float f = part < 2 ? 1.f : p.scale;
-            uint4* dst = reinterpret_cast<uint4*>(acc_out + (static_cast<size_t>(w.bh) * p.N + key) * kD + acc_col);
+            const uint32_t scratch = c.base + kOffDS;
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
                 uint32_t x[4];
@@ -617,8 +623,19 @@ __device__ __forceinline__ void role_pds(const Ctx& c, int warp, int lane) {
                     const int cc = v4 * 8 + e * 2;
                     x[e] = pack_bf16x2(__uint_as_float(acc[cc]) * f, __uint_as_float(acc[cc + 1]) * f);
                 }
-                dst[v4] = make_uint4(x[0], x[1], x[2], x[3]);
+                st_shared_v4(scratch + sw128_off(r, col0 + v4 * 8), x[0], x[1], x[2], x[3]);
             }
+            __syncwarp();
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) {
+                const int rr = quarter * 32 + 8 * k8 + (lane >> 2), ch = lane & 3;
+                const uint4 v = lds_u32x4(scratch + sw128_off(rr, col0 + ch * 8));
+                const int key_rr = w.kb * kBK + rr;
+                if (key_rr < p.N)
+                    *reinterpret_cast<uint4*>(acc_out + (static_cast<size_t>(w.bh) * p.N + key_rr) * kD + acc_col +
+                                              ch * 8) = v;
+            }
+            __syncwarp();
         }
     }
 }
