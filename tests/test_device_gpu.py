@@ -16,6 +16,10 @@ def peak_extra_bytes(q, k, v, causal=False):
     as the first page of the pages does it: memory_allocated() as the base,
     reset the peak, run, and read max_memory_allocated()."""
     torch.cuda.synchronize()
+    # an empty cache first: a cached block left by an earlier test can be
+    # handed out whole (the allocator does not split off small remainders),
+    # which would count bytes the call never asked for
+    torch.cuda.empty_cache()
     base = torch.cuda.memory_allocated()
     torch.cuda.reset_peak_memory_stats()
     o, lse = pkg.forward(q, k, v, causal=causal)
