@@ -44,15 +44,17 @@
 //     reductions (cp.reduce.async.bulk.tensor .add), two [32 x 32] boxes per
 //     warp through one staging box;
 //   * at the end of a unit warps 0-7 write dV and warps 8-15 dK (times
-//     scale) in bf16, 32 columns each.
+//     scale) in bf16, 32 columns each, each warp passing its [32 x 32] block
+//     through its own bytes of a (then free) dS^T buffer so that four lanes
+//     store one 64-byte row segment.
 //   Every wait is bounded (see sm100_ptx.cuh) and no barrier spans warps
 //   other than mbarriers, so a timeout never leaves a thread blocked.
 //
 // TMEM columns: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
-// dQ [384,448), P^T [448,512) (bf16 pairs).  Shared memory (226,560 bytes
+// dQ [384,448), P^T [448,512) (bf16 pairs).  Shared memory (230,656 bytes
 // with alignment): K, V (16 KB each), three stages of Q and dO (16 KB each),
 // two dS^T buffers (32 KB each, two 64-column halves), four 4 KB dQ staging
-// boxes, two offset slots and the ones (4 KB each), barriers.
+// boxes, one offset block per stage and the ones (4 KB each), barriers.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
