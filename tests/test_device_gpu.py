@@ -12,19 +12,20 @@ DEV = torch.device("cuda:0")
 
 
 def peak_extra_bytes(q, k, v, causal=False):
-    """Peak device bytes allocated by one call on top of the inputs, measured
-    as the first page of the pages does it: memory_allocated() as the base,
-    reset the peak, run, and read max_memory_allocated()."""
+    """Peak device bytes one call asks the caching allocator for on top of
+    what is already allocated, measured as the first page of the pages does it
+    (a base, reset the peak, run, read the peak) on the allocator's
+    requested-bytes counters.  Its allocated-bytes counters would also count
+    the unsplit remainder of a cached block that an earlier test left behind
+    (the allocator hands out a cached block whole when the rest would be
+    small), which depends on the order of the tests, not on the call; the
+    benchmark, in a fresh process, reports the allocated-bytes figure."""
     torch.cuda.synchronize()
-    # an empty cache first: a cached block left by an earlier test can be
-    # handed out whole (the allocator does not split off small remainders),
-    # which would count bytes the call never asked for
-    torch.cuda.empty_cache()
-    base = torch.cuda.memory_allocated()
+    base = torch.cuda.memory_stats()["requested_bytes.all.current"]
     torch.cuda.reset_peak_memory_stats()
     o, lse = pkg.forward(q, k, v, causal=causal)
     torch.cuda.synchronize()
-    extra = torch.cuda.max_memory_allocated() - base
+    extra = torch.cuda.memory_stats()["requested_bytes.all.peak"] - base
     del o, lse
     return extra
 
