@@ -127,6 +127,19 @@ def profiled_traffic():
         return None
 
 
+# A spin on the device, queued right before a timed loop, while which the
+# host enqueues the first steps: a host stall (interpreter, the clock-sampling
+# thread) then finds the device still busy instead of leaving it idle between
+# a step's start event and its launch, where the stall would count as that
+# step's time.  It runs before the first step's start event (~2 ms).
+HOST_LEAD_CYCLES = 4_000_000
+
+
+def host_lead():
+    import torch
+    torch.cuda._sleep(HOST_LEAD_CYCLES)
+
+
 def reduce_max(value, dist=None, device=None):
     """Max of a float over all ranks (identity on one process)."""
     if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
@@ -282,6 +295,7 @@ def run_cuda(args, rank, world, dist):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clocks:
+        host_lead()
         for i in range(args.steps):
             flush.zero_()
             ev[i][0].record(stream)
@@ -348,6 +362,7 @@ def run_cuda(args, rank, world, dist):
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize()
+        host_lead()
         for i in range(e2e_steps):
             flush.zero_()
             eev[i][0].record(stream)
@@ -424,6 +439,7 @@ def run_cuda_backward(args, rank, world, dist):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clocks:
+        host_lead()
         for i in range(args.steps):
             flush.zero_()
             ev[i][0].record(stream)
@@ -485,6 +501,7 @@ def run_sweep(args):
             pkg.forward(q, k, v, out=o, lse=lse)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         torch.cuda.synchronize()
+        host_lead()
         for i in range(steps):
             flush.zero_()
             ev[i][0].record()
@@ -531,6 +548,7 @@ def run_pad_sweep(args):
             pkg.forward(q, k, v, out=o, lse=lse, key_padding_mask=pad)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         torch.cuda.synchronize()
+        host_lead()
         for i in range(steps):
             flush.zero_()
             ev[i][0].record()
