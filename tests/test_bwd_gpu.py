@@ -133,6 +133,36 @@ def test_bwd_deterministic_dk_dv():
     np.testing.assert_allclose(dq1, dq2, rtol=0, atol=1e-5 * np.abs(dq1).max())
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_bwd_two_streams_at_once_match_one_stream(d):
+    # backward launches on two streams at the same time: dK, dV bit-identical
+    # to the same call alone, dQ (fp32 bulk reductions in any order) equal to
+    # fp32 summation-order noise
+    dev = torch.device("cuda:0")
+    sets = []
+    for seed in (41, 42):
+        q, k, v = (x.to(dev) for x in make_qkv(1, 4, 1000, d, seed=seed))
+        do = make_dout(1, 4, 1000, d, seed=seed + 100).to(dev)
+        o, lse = pkg.forward(q, k, v, causal=True)
+        sets.append((q, k, v, o, lse, do))
+    ref = [pkg.backward(q, k, v, o, lse, do, causal=True) for (q, k, v, o, lse, do) in sets]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for s in streams:
+        s.wait_stream(torch.cuda.current_stream())
+    outs = []
+    for _ in range(3):
+        for i in (0, 1):
+            with torch.cuda.stream(streams[i]):
+                outs.append((i, pkg.backward(*sets[i], causal=True)))
+    torch.cuda.synchronize()
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    for i, (dq, dk, dv) in outs:
+        rq, rk, rv = ref[i]
+        assert torch.equal(dk, rk) and torch.equal(dv, rv)
+        assert float((dq - rq).abs().max()) <= 1e-5 * float(rq.abs().max())
+
+
 # ---- key padding (the forward's mask, nonzero = padded key)
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])

@@ -153,6 +153,29 @@ def test_deterministic_and_stream_ordered():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("d,causal", [(64, False), (128, True)])
+def test_two_streams_at_once_match_one_stream(d, causal):
+    # launches on two streams run at the same time (each kernel keeps its state
+    # in its own shared memory and TMEM; no atomics on the outputs): every
+    # result is bit-identical to the same call alone
+    dev = torch.device("cuda:0")
+    ins = [[x.to(dev) for x in make_qkv(1, 8, 2000, d, seed=s)] for s in (31, 32)]
+    ref = [pkg.forward(*t, causal=causal) for t in ins]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for s in streams:
+        s.wait_stream(torch.cuda.current_stream())
+    outs = []
+    for _ in range(4):
+        for i in (0, 1):
+            with torch.cuda.stream(streams[i]):
+                outs.append((i, pkg.forward(*ins[i], causal=causal)))
+    torch.cuda.synchronize()
+    assert pkg.attn_check_device_status() == pkg.ATTN_OK
+    for i, (o, lse) in outs:
+        assert torch.equal(o, ref[i][0]) and torch.equal(lse, ref[i][1])
+
+
 def test_permuting_keys_and_values_leaves_output_unchanged():
     # a property that holds at any size: exact attention is invariant to a
     # joint permutation of the keys and values
